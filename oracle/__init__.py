@@ -1,0 +1,164 @@
+"""fp64 CPU oracle of the Mesa layer (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product library
+(``test_sequence_layer_b200``) never imports it, and this package imports
+nothing from the product.
+
+The arithmetic lives in ``mesa_oracle.c`` (plain C, fp64). This module only
+compiles it with gcc and marshals numpy arrays through ctypes. Every array is
+converted to contiguous float64 (bf16 and fp32 inputs convert exactly).
+
+Method: "MesaNet: Sequence Modeling by Locally Optimal Test-Time Training"
+(gist.science, ja/ko/hi editions), Technical summary > Method > Mesa layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mesa_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libmesa_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP over independent sequences)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    hdr = os.path.join(_HERE, "mesa_oracle.h")
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < max(os.path.getmtime(_SRC), os.path.getmtime(hdr)))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        # -ffp-contract=off: no fused multiply-adds, so each line rounds as written.
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        D = ctypes.POINTER(ctypes.c_double)
+        I32 = ctypes.POINTER(ctypes.c_int32)
+        i, d = ctypes.c_int, ctypes.c_double
+        lib.oracle_forward_cg.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, I32, D, D]
+        lib.oracle_forward_cholesky.argtypes = [D, D, D, D, D, D, i, i, i, i, i, D, D, D, D, D]
+        lib.oracle_forward_chunked.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, i, d, D, D, D, I32, D, D]
+        lib.oracle_step.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, i, d, D, I32]
+        lib.oracle_cg_dense.argtypes = [i, D, D, i, d, D, I32]
+        for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
+                  lib.oracle_step, lib.oracle_cg_dense):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor -> numpy (exact widening to fp64)
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if a.dtype == np.int32:
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise RuntimeError(f"{name} failed with code {rc}")
+
+
+def _shapes(q, v):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    return B, H, T, dk, dv
+
+
+def forward_cg(q, k, v, gamma, beta, lam, cg_steps, tol=0.0, H0=None, G0=None):
+    """Per-token recurrence + CG. Returns (out, iters, H_final, G_final)."""
+    q, k, v, gamma, beta, lam = map(_f64, (q, k, v, gamma, beta, lam))
+    H0, G0 = _f64(H0), _f64(G0)
+    B, H, T, dk, dv = _shapes(q, v)
+    out = np.zeros((B, H, T, dv))
+    iters = np.zeros((B, H, T), dtype=np.int32)
+    Hf = np.zeros((B, H, dk, dk))
+    Gf = np.zeros((B, H, dv, dk))
+    rc = _load().oracle_forward_cg(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                   B, H, T, dk, dv, int(cg_steps), float(tol), _ptr(H0), _ptr(G0),
+                                   _ptr(out), _ptr(iters), _ptr(Hf), _ptr(Gf))
+    _check(rc, "oracle_forward_cg")
+    return out, iters, Hf, Gf
+
+
+def forward_cholesky(q, k, v, gamma, beta, lam, H0=None, G0=None):
+    """Per-token recurrence + exact solve. Returns (out, H_final, G_final)."""
+    q, k, v, gamma, beta, lam = map(_f64, (q, k, v, gamma, beta, lam))
+    H0, G0 = _f64(H0), _f64(G0)
+    B, H, T, dk, dv = _shapes(q, v)
+    out = np.zeros((B, H, T, dv))
+    Hf = np.zeros((B, H, dk, dk))
+    Gf = np.zeros((B, H, dv, dk))
+    rc = _load().oracle_forward_cholesky(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                         B, H, T, dk, dv, _ptr(H0), _ptr(G0), _ptr(out), _ptr(Hf), _ptr(Gf))
+    _check(rc, "oracle_forward_cholesky")
+    return out, Hf, Gf
+
+
+def forward_chunked(q, k, v, gamma, beta, lam, chunk, cg_steps, tol=0.0, H0=None, G0=None):
+    """Chunked form with the same CG rule. Returns (out, iters, H_final, G_final)."""
+    q, k, v, gamma, beta, lam = map(_f64, (q, k, v, gamma, beta, lam))
+    H0, G0 = _f64(H0), _f64(G0)
+    B, H, T, dk, dv = _shapes(q, v)
+    out = np.zeros((B, H, T, dv))
+    iters = np.zeros((B, H, T), dtype=np.int32)
+    Hf = np.zeros((B, H, dk, dk))
+    Gf = np.zeros((B, H, dv, dk))
+    rc = _load().oracle_forward_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                        B, H, T, dk, dv, int(chunk), int(cg_steps), float(tol),
+                                        _ptr(H0), _ptr(G0), _ptr(out), _ptr(iters), _ptr(Hf), _ptr(Gf))
+    _check(rc, "oracle_forward_chunked")
+    return out, iters, Hf, Gf
+
+
+def step(q, k, v, gamma, beta, lam, Hstate, Gstate, cg_steps, tol=0.0):
+    """One decode step. q,k,v: [B,H,d]; gamma,beta: [B,H]. States are copied
+    (not modified). Returns (out, iters, H_new, G_new)."""
+    q, k, v, gamma, beta, lam = map(_f64, (q, k, v, gamma, beta, lam))
+    Hs = _f64(Hstate).copy()
+    Gs = _f64(Gstate).copy()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((B, H, dv))
+    iters = np.zeros((B, H), dtype=np.int32)
+    rc = _load().oracle_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                             B, H, dk, dv, _ptr(Hs), _ptr(Gs), int(cg_steps), float(tol),
+                             _ptr(out), _ptr(iters))
+    _check(rc, "oracle_step")
+    return out, iters, Hs, Gs
+
+
+def cg_dense(A, b, cg_steps, tol=0.0):
+    """CG on one dense SPD system. Returns (x, iters)."""
+    A, b = _f64(A), _f64(b)
+    n = b.shape[0]
+    x = np.zeros(n)
+    it = np.zeros(1, dtype=np.int32)
+    rc = _load().oracle_cg_dense(n, _ptr(A), _ptr(b), int(cg_steps), float(tol), _ptr(x), _ptr(it))
+    _check(rc, "oracle_cg_dense")
+    return x, int(it[0])
