@@ -1,0 +1,324 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the Mesa layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One "step" is one mesa_forward over the whole workload (all tokens of every
+(b, h) sequence), with inputs resident in HBM. The default workload is the
+long-context bf16 forward (B=8, H=16, T=8192, d=128, chunk 64, 15 CG steps).
+Under torchrun every rank runs its own copy of the workload on its own GPU
+(sequences are independent: weak scaling, no data-path collective); the
+timed region is bracketed by a barrier and a device synchronisation, and the
+slowest rank's time is reported. Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0
+only), each step on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mesa_inputs as mi  # noqa: E402
+
+# fp32 FMA peak on CUDA cores: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz.
+SIMT_FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def flops_per_token_iter(d, C):
+    """Useful causal flops of one CG matvec per token: inter-chunk 2d^2 plus
+    the masked intra-chunk scores and their read-back, 2d(C+1)."""
+    return 2 * d * d + 2 * d * (C + 1)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_sample(w, n_seq, T_s):
+    """Times the oracle on n_seq sequences x T_s tokens of workload w; returns tokens/s."""
+    import oracle
+    oracle.build()
+    pairs = [(i // w.H, i % w.H) for i in range(n_seq)]
+    x = mi.batch(w, T=T_s, seqs=pairs)
+    t0 = time.perf_counter()
+    oracle.forward_cg(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], w.cg_steps, w.tol)
+    dt = time.perf_counter() - t0
+    return n_seq * T_s / dt, dt
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    cores = host_cores()
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    n_seq, T_s = min(cores, w.B * w.H), 256
+    rates = []
+    for s in range(args.warmup + args.steps):
+        rate, _ = cpu_oracle_sample(w, n_seq, T_s)
+        if s >= args.warmup:
+            rates.append(rate)
+    value = statistics.median(rates)
+    sample = f"{n_seq} sequences x first {T_s} tokens of {w.name} per step (OpenMP over sequences)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * n_seq * T_s / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.dk, "chunk": w.chunk,
+                   "cg_steps": w.cg_steps, "tol": w.tol},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "Mesa-layer fwd tokens/s (B*H*T) at T=8192,d=128,15 CG steps; % tensor peak"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="bf16_T8192", choices=[k for k in mi.WORKLOADS if k != "decode"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3 or args.impl == "reference" or os.environ.get("MESA_BENCH_ALLOW_SHORT"), \
+        "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = mi.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from test_sequence_layer_b200 import build as mbuild, mesa
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    x = mi.device_batch(w, dev, seed_offset=rank)
+    B, H, T, d, C = w.B, w.H, w.T, w.dk, w.chunk
+    tokens = B * H * T
+    out = torch.empty((B, H, T, d), device=dev)
+    iters = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+    ws = torch.empty(max(mesa.workspace_size(B, H, T, d, d, C, x["q"].dtype), 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mesa.forward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], chunk=C, cg_steps=w.cg_steps,
+                     tol=w.tol, out=out, return_iters=True, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert mesa.get_error(stream) == 0
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    mesa.timing_enable(False)
+    kernels = mesa.timing_read()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert mesa.get_error(stream) == 0
+    ms_per_step = ms / args.steps
+    value = world * tokens / (ms_per_step / 1e3)
+    total_iters = int(iters.sum().item())
+
+    # dominant kernel and its roofline
+    name, (launches, kms) = max(kernels.items(), key=lambda kv: kv[1][1])
+    gpu_launches = sum(v[0] for v in kernels.values())
+    avg_ms = kms / max(launches, 1)
+    peaks = load_peaks()
+    fti = flops_per_token_iter(d, C)
+    if name in ("tc_cg", "simt_cg"):
+        # CG matvecs actually needed (sum of per-token iteration counts) + one read-out per token
+        flops = (total_iters + tokens) * fti
+    else:
+        flops = tokens * 2 * (d * d + d * d)
+    achieved = flops / (avg_ms / 1e3) / 1e12
+    if name.startswith("tc_"):
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "peak_kind": f"{peaks['_source']} bf16 dense burst (fp16 operands run at the bf16 rate)"}
+    else:
+        roof = {"bound": "alu", "achieved": achieved, "peak": SIMT_FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "peak_kind": "fp32 FMA: 148 SM x 128 FMA/clk x 2 x 1.965 GHz"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = name
+    roof["avg_ms"] = avg_ms
+
+    # end to end through the host-buffer C-ABI call (copies inside the timed region)
+    e2e = None
+    if not args.no_e2e:
+        hx = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "gamma", "beta", "lam")}
+        hout = torch.empty((B, H, T, d)).pin_memory()
+        hws = torch.empty(mesa.mesa._load().mesa_forward_host_workspace_size(
+            B, H, T, d, d, C, 1 if x["q"].dtype == torch.bfloat16 else 0), dtype=torch.uint8, device=dev)
+        del ws
+        e_steps = max(3, args.steps // 4)
+
+        def hstep():
+            mesa.forward_host(hx["q"], hx["k"], hx["v"], hx["gamma"], hx["beta"], hx["lam"], chunk=C,
+                              cg_steps=w.cg_steps, tol=w.tol, out=hout, workspace=hws, device=dev,
+                              stream=stream)
+        hstep()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            hstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = sum(hx[n].numel() * hx[n].element_size() for n in ("q", "k", "v", "gamma", "beta", "lam"))
+        e2e = {"value": world * tokens / (ems / e_steps / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = host_cores()
+        n_seq = min(w.B * w.H, max(cores, 1))
+        T_s = min(w.T, 1024)
+        rate, dt = cpu_oracle_sample(w, n_seq, T_s)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n_seq} sequences x first {T_s} tokens of {w.name} ({dt:.1f} s, OpenMP over sequences)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    path = "tensor-core (tcgen05)" if name.startswith("tc_") else "fp32 CUDA-core"
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16-in/f16-mma/f32-acc" if name.startswith("tc_") else "bf16-in/f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "T": T, "d": d, "chunk": C, "cg_steps": w.cg_steps,
+                   "tol": w.tol, "path": path, "per_gpu_tokens": tokens,
+                   "l2": "inputs larger than L2 (%.2f GB per step)" % ((x["q"].numel() * 3 * x["q"].element_size()
+                                                                       + out.numel() * 4) / 1e9),
+                   "cg_iters_total": total_iters},
+        "roofline": roof,
+        "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
+        "gpu_launches": gpu_launches,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

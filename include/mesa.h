@@ -1,0 +1,190 @@
+/*
+ * mesa.h -- C ABI of the B200 (sm_100a) Mesa layer library (libmesa_b200.so).
+ *
+ * The Mesa layer of "MesaNet: Sequence Modeling by Locally Optimal Test-Time
+ * Training" (gist.science, ja/ko/hi editions; Technical summary > Method >
+ * Mesa layer). For every sequence (b, h) and token t it keeps the gated
+ * statistics
+ *     H_t = gamma_t H_{t-1} + beta_t k_t k_t^T        (dk x dk)
+ *     G_t = gamma_t G_{t-1} + beta_t v_t k_t^T        (dv x dk)
+ * (the page's cumulative forget factors zeta read as
+ *  zeta_{tt'} = beta_t' prod_{s=t'+1..t} gamma_s), solves
+ *     (H_t + Lambda) x_t = q_t
+ * by conjugate gradient (the page's "optimal query response"), and emits the
+ * locally optimal read-out o_t = G_t x_t (the page's Delta_t = Phi_t q_t with
+ * Phi_t = G_t (H_t + Lambda)^-1, the minimiser of its Mesa objective).
+ *
+ * CG rule (identical in every entry point): x_0 = 0, r_0 = p_0 = q_t; before
+ * each of at most cg_steps updates the token stops if tol > 0 and
+ * |r|_2 <= tol |q_t|_2 (the page's per-token stopping criterion under
+ * "Dynamic compute"); it also stops, keeping its x, if r.r <= 0 or
+ * p.(H+Lambda)p <= 0 or is not finite. iters = number of updates applied.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller (except
+ *     mesa_forward_host, whose tensors are host pointers). The library
+ *     allocates no device memory in any call; scratch space is the caller's
+ *     workspace.
+ *   - Layouts are contiguous row-major: q, k [B,H,T,dk]; v, out [B,H,T,dv];
+ *     gamma, beta, iters [B,H,T]; lambda [H,dk] (the diagonal of Lambda for
+ *     each head, shared by the batch); H states [B,H,dk,dk]; G states
+ *     [B,H,dv,dk].
+ *   - Preconditions on values (not checked, the caller's contract):
+ *     0 < gamma <= 1, beta >= 0, lambda > 0, all finite. Non-finite inputs
+ *     give non-finite outputs for the affected tokens but never hang.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Device calls are asynchronous on it.
+ *   - Argument errors are returned synchronously and nothing is launched.
+ *     A failed launch returns MESA_ERR_CUDA. A kernel that gives up a bounded
+ *     wait records MESA_ERR_DEVICE_TIMEOUT in a per-device error word that
+ *     mesa_get_error() reads and clears.
+ */
+#ifndef MESA_H
+#define MESA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MESA_OK = 0,
+    MESA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misalignment, bad tol */
+    MESA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (dk, dv, chunk) */
+    MESA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
+    MESA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+    MESA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait (see mesa_get_error) */
+} mesa_status;
+
+typedef enum {
+    MESA_F32 = 0,    /* q, k, v are float32 */
+    MESA_BF16 = 1    /* q, k, v are bfloat16 (gamma, beta, lambda stay float32) */
+} mesa_dtype;
+
+/*
+ * Bytes of device workspace mesa_forward needs for these sizes (0 if the
+ * sizes are invalid or unsupported). The workspace holds the chunk-start
+ * states {H_c, G_c} of every chunk (the layer's carried inter-chunk state).
+ */
+size_t mesa_forward_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                   mesa_dtype dtype);
+
+/*
+ * Chunkwise-parallel forward of the Mesa layer over a whole sequence.
+ * Source: the MesaNet page, Technical summary > Method > Mesa layer
+ * (objective; CG solve of q*_t) and its "Parallelisation" paragraph (CG over
+ * many time steps is gated linear attention; the layer keeps G_t and H_t
+ * and solves the systems of a chunk in parallel).
+ *
+ *   q, k, v      input tensors, element type `dtype`, 16-byte aligned.
+ *   gamma, beta  float32 [B,H,T], 4-byte aligned.
+ *   lambda       float32 [H,dk], > 0.
+ *   B, H, T      batch, heads, tokens; B,H >= 1, T >= 0 (T = 0: only the
+ *                final-state outputs are written, as copies of the initial
+ *                state or zeros).
+ *   dk, dv       key and value width. Supported: dk == dv in {16,32,64,128}.
+ *   chunk        chunk length C in {16,32,64}; T need not be a multiple of C
+ *                (the tail behaves as if padded with beta = 0, gamma = 1).
+ *                The tensor-core path serves dtype = MESA_BF16,
+ *                dk = dv = 128, chunk = 64; every other supported shape runs
+ *                the fp32 CUDA-core path.
+ *   cg_steps     maximum CG updates per token, 0..1024.
+ *   tol          relative residual tolerance; <= 0 runs exactly cg_steps
+ *                updates (unless breakdown). NaN is an argument error.
+ *   out          float32 [B,H,T,dv], 16-byte aligned (written).
+ *   iters_out    int32 [B,H,T] or NULL: CG updates applied per token.
+ *   H_in, G_in   float32 initial states or NULL (zero), 16-byte aligned.
+ *   H_out, G_out float32 final states (after token T-1) or NULL. May not
+ *                alias H_in / G_in.
+ *   workspace    device memory of at least mesa_forward_workspace_size()
+ *                bytes, 256-byte aligned. Its contents on entry do not
+ *                matter; calls sharing a workspace must not overlap.
+ */
+mesa_status mesa_forward(const void* q, const void* k, const void* v,
+                         const float* gamma, const float* beta, const float* lambda,
+                         int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                         int cg_steps, float tol,
+                         float* out, int32_t* iters_out,
+                         const float* H_in, const float* G_in,
+                         float* H_out, float* G_out,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Bytes of device workspace mesa_forward_host needs: the mesa_forward
+ * workspace plus device staging for every tensor argument.
+ */
+size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                        mesa_dtype dtype);
+
+/*
+ * The same forward with every tensor in HOST memory (page-locked memory is
+ * recommended for overlap; pageable memory works but is slower). The call
+ * enqueues one host-to-device copy per input, the forward, and one
+ * device-to-host copy per requested output on `stream`, then synchronises
+ * the stream before returning, so the host outputs are valid on MESA_OK.
+ * No host alignment is required. `workspace` is DEVICE memory of at least
+ * mesa_forward_host_workspace_size() bytes, 256-byte aligned.
+ */
+mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
+                              const float* gamma, const float* beta, const float* lambda,
+                              int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                              int cg_steps, float tol,
+                              float* out, int32_t* iters_out,
+                              const float* H_in, const float* G_in,
+                              float* H_out, float* G_out,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * One recurrent decode step on explicit state, O(1) per token (the MesaNet
+ * page, "Parallelisation": O(1) inference with the state variables G_t, H_t).
+ * For every (b, h): H <- gamma H + beta k k^T, G <- gamma G + beta v k^T,
+ * x = CG(H + Lambda, q), out = G x.
+ *
+ *   q, k         float32 [B,H,dk];  v float32 [B,H,dv]; 16-byte aligned.
+ *   gamma, beta  float32 [B,H].     lambda float32 [H,dk].
+ *   dk == dv in {16,32,64,128}.
+ *   Hstate       float32 [B,H,dk,dk], read and overwritten in place.
+ *   Gstate       float32 [B,H,dv,dk], read and overwritten in place.
+ *   cg_steps, tol as in mesa_forward.
+ *   out          float32 [B,H,dv] (written).  iters_out int32 [B,H] or NULL.
+ * No workspace is needed.
+ */
+mesa_status mesa_step(const float* q, const float* k, const float* v,
+                      const float* gamma, const float* beta, const float* lambda,
+                      int B, int H, int dk, int dv,
+                      float* Hstate, float* Gstate,
+                      int cg_steps, float tol,
+                      float* out, int32_t* iters_out, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error
+ * word. Returns MESA_OK if no kernel recorded an error since the last call,
+ * MESA_ERR_DEVICE_TIMEOUT if one gave up a bounded wait, MESA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+mesa_status mesa_get_error(void* stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* mesa_status_string(mesa_status s);
+
+/*
+ * Kernel timing (a profiling aid, off by default). While enabled, every
+ * kernel the library launches is bracketed by CUDA events recorded on the
+ * call's stream, and counted. mesa_timing_read() synchronises those events
+ * and returns, for up to `max` kernel kinds, the kind's name, its number of
+ * launches and its summed device time in milliseconds since the last read;
+ * it then clears the records. Returns the number of kinds written, or -1 on
+ * a CUDA error. Not thread-safe; enable it only in one host thread.
+ */
+mesa_status mesa_timing_enable(int on);
+int mesa_timing_read(const char** names, int* launches, double* total_ms, int max);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int mesa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MESA_H */

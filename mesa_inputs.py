@@ -145,3 +145,48 @@ def batch(w: Workload, T: int | None = None, B: int | None = None, H: int | None
     # each carrying the lambda row of its own head
     lam_rows = np.stack([lam[h] for (_, h) in pairs])
     return dict(q=q[None], k=k[None], v=v[None], gamma=g[None], beta=be[None], lam=lam_rows)
+
+
+def device_batch(w: Workload, device, T: int | None = None, B: int | None = None,
+                 H: int | None = None, seed_offset: int = 0):
+    """The same distributions drawn on the device with a seeded torch generator
+    (for full-size runs where drawing every sequence on the host is too slow).
+    Returns torch tensors: q, k, v in the workload dtype, gamma, beta, lam float32."""
+    import torch
+    T = w.T + w.decode_steps if T is None else T
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    g = torch.Generator(device=device)
+    g.manual_seed(1_000_003 * w.seed + seed_offset)
+    f32 = torch.float32
+    q = torch.randn((B, H, T, w.dk), generator=g, device=device, dtype=f32)
+    k = torch.randn((B, H, T, w.dk), generator=g, device=device, dtype=f32)
+    v = torch.randn((B, H, T, w.dv), generator=g, device=device, dtype=f32)
+    zg = torch.randn((B, H, T), generator=g, device=device, dtype=f32)
+    zb = torch.randn((B, H, T), generator=g, device=device, dtype=f32)
+    if w.mixture:
+        coin = torch.rand((B, H, T), generator=g, device=device, dtype=f32)
+        gamma = torch.where(coin < 0.5, torch.sigmoid(zg + 5.0), torch.sigmoid(zg))
+    else:
+        gamma = torch.sigmoid(zg + 3.0)
+    beta = torch.sigmoid(zb)
+    q = q / q.norm(dim=-1, keepdim=True)
+    k = k / k.norm(dim=-1, keepdim=True)
+    dt = torch.bfloat16 if w.dtype == "bf16" else f32
+    lam = torch.from_numpy(lambdas(w.seed, w.H, w.dk)[:H].copy()).to(device)
+    return dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), gamma=gamma.contiguous(), beta=beta.contiguous(), lam=lam)
+
+
+def plant_sequences(dev: dict, w: Workload, pairs, T: int | None = None):
+    """Overwrites the (b, h) sequences listed in ``pairs`` of a device batch with
+    their host per-sequence streams, so those sequences match ``batch(w, seqs=pairs)``."""
+    import torch
+    T = dev["q"].shape[2] if T is None else T
+    host = batch(w, T=T, seqs=pairs)
+    dt = dev["q"].dtype
+    for i, (b, h) in enumerate(pairs):
+        for name in ("q", "k", "v"):
+            dev[name][b, h].copy_(torch.from_numpy(host[name][0, i]).to(dt))
+        dev["gamma"][b, h].copy_(torch.from_numpy(host["gamma"][0, i]))
+        dev["beta"][b, h].copy_(torch.from_numpy(host["beta"][0, i]))
+    return host

@@ -1,0 +1,314 @@
+// api.cu -- the extern "C" entry points of libmesa_b200.so (declared in mesa.h):
+// argument validation, workspace carving, kernel dispatch, the host-buffer
+// variant and the per-device error word.
+#include <math.h>
+#include <string.h>
+
+#include <vector>
+
+#include "mesa_common.cuh"
+#include "mesa_internal.h"
+
+namespace mesa {
+
+__device__ unsigned g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices] = {nullptr};
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool supported_width(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// Shape checks shared by every forward entry point (no pointers involved).
+mesa_status check_shape(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                        int cg_steps, float tol) {
+    if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1 || chunk < 1) return MESA_ERR_INVALID_ARG;
+    if (dtype != MESA_F32 && dtype != MESA_BF16) return MESA_ERR_INVALID_ARG;
+    if (cg_steps < 0 || cg_steps > 1024 || isnan(tol)) return MESA_ERR_INVALID_ARG;
+    if ((long long)B * H > 65535) return MESA_ERR_UNSUPPORTED;           // grid.y limit
+    if (!supported_width(dk) || dk != dv) return MESA_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return MESA_ERR_UNSUPPORTED;
+    if ((long long)(T + chunk - 1) / chunk > 0x7fffffffLL) return MESA_ERR_UNSUPPORTED;
+    return MESA_OK;
+}
+
+size_t workspace_bytes(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
+    if (tc_supported(dk, dv, chunk, dtype)) return tc_workspace_bytes(B, H, T);
+    return simt_workspace_bytes(B, H, T, dk, dv, chunk);
+}
+
+size_t elem_size(mesa_dtype d) { return d == MESA_BF16 ? 2 : 4; }
+
+mesa_status launch_forward(const ForwardArgs& a, cudaStream_t st) {
+    const size_t sbytes = (size_t)a.B * a.H * a.dk * a.dk * sizeof(float);
+    const size_t gbytes = (size_t)a.B * a.H * a.dv * a.dk * sizeof(float);
+    if (a.T == 0) {
+        // Nothing to read out; the final state is the initial state.
+        if (a.H_out) {
+            cudaError_t e = a.H_in ? cudaMemcpyAsync(a.H_out, a.H_in, sbytes, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(a.H_out, 0, sbytes, st);
+            if (e != cudaSuccess) return MESA_ERR_CUDA;
+        }
+        if (a.G_out) {
+            cudaError_t e = a.G_in ? cudaMemcpyAsync(a.G_out, a.G_in, gbytes, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(a.G_out, 0, gbytes, st);
+            if (e != cudaSuccess) return MESA_ERR_CUDA;
+        }
+        return MESA_OK;
+    }
+    cudaError_t e = tc_supported(a.dk, a.dv, a.chunk, a.dtype) ? forward_tc(a, st) : forward_simt(a, st);
+    return e == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+// ---- kernel timing records ----
+const char* const kKindNames[kKindCount] = {"simt_scan", "simt_cg", "decode_step", "tc_scan", "tc_cg"};
+struct TimingRec {
+    int kind;
+    cudaEvent_t start, stop;
+};
+bool g_timing_on = false;
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+constexpr size_t kMaxRecs = 1 << 16;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+}  // namespace
+
+LaunchTimer::LaunchTimer(int kind, cudaStream_t st) : slot_(-1), st_(st) {
+    if (!g_timing_on || g_recs.size() >= kMaxRecs) return;
+    TimingRec r{kind, take_event(), take_event()};
+    if (!r.start || !r.stop || cudaEventRecord(r.start, st) != cudaSuccess) {
+        if (r.start) g_event_pool.push_back(r.start);
+        if (r.stop) g_event_pool.push_back(r.stop);
+        return;
+    }
+    slot_ = (int)g_recs.size();
+    g_recs.push_back(r);
+}
+
+LaunchTimer::~LaunchTimer() {
+    if (slot_ >= 0) cudaEventRecord(g_recs[slot_].stop, st_);
+}
+
+unsigned* error_word_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned*>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+}  // namespace mesa
+
+using namespace mesa;
+
+extern "C" {
+
+int mesa_version(void) { return 10000; }
+
+const char* mesa_status_string(mesa_status s) {
+    switch (s) {
+        case MESA_OK: return "MESA_OK";
+        case MESA_ERR_INVALID_ARG: return "MESA_ERR_INVALID_ARG";
+        case MESA_ERR_UNSUPPORTED: return "MESA_ERR_UNSUPPORTED";
+        case MESA_ERR_WORKSPACE: return "MESA_ERR_WORKSPACE";
+        case MESA_ERR_CUDA: return "MESA_ERR_CUDA";
+        case MESA_ERR_DEVICE_TIMEOUT: return "MESA_ERR_DEVICE_TIMEOUT";
+    }
+    return "MESA_ERR_UNKNOWN";
+}
+
+size_t mesa_forward_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
+    if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
+    return workspace_bytes(B, H, T, dk, dv, chunk, dtype);
+}
+
+mesa_status mesa_forward(const void* q, const void* k, const void* v,
+                         const float* gamma, const float* beta, const float* lambda,
+                         int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                         int cg_steps, float tol,
+                         float* out, int32_t* iters_out,
+                         const float* H_in, const float* G_in,
+                         float* H_out, float* G_out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+    mesa_status s = check_shape(B, H, T, dk, dv, chunk, dtype, cg_steps, tol);
+    if (s != MESA_OK) return s;
+    if (!lambda || !aligned(lambda, 4)) return MESA_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!q || !k || !v || !gamma || !beta || !out) return MESA_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return MESA_ERR_INVALID_ARG;
+        if (!aligned(gamma, 4) || !aligned(beta, 4)) return MESA_ERR_INVALID_ARG;
+        if (iters_out && !aligned(iters_out, 4)) return MESA_ERR_INVALID_ARG;
+    }
+    for (const void* p : {(const void*)H_in, (const void*)G_in, (const void*)H_out, (const void*)G_out})
+        if (p && !aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    if ((H_out && H_out == H_in) || (G_out && G_out == G_in)) return MESA_ERR_INVALID_ARG;
+    const size_t need = workspace_bytes(B, H, T, dk, dv, chunk, dtype);
+    if (T > 0 && need > 0) {
+        if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
+    }
+    ForwardArgs a{q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps, tol,
+                  out, iters_out, H_in, G_in, H_out, G_out, workspace, ws_bytes};
+    return launch_forward(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
+    if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
+    const size_t tok = (size_t)B * H * T;
+    const size_t es = elem_size(dtype);
+    size_t n = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256);
+    n += round_up(tok * dk * es, 256) * 2 + round_up(tok * dv * es, 256);      // q, k, v
+    n += round_up(tok * 4, 256) * 2 + round_up((size_t)H * dk * 4, 256);      // gamma, beta, lambda
+    n += round_up(tok * dv * 4, 256) + round_up(tok * 4, 256);                // out, iters
+    n += (round_up((size_t)B * H * dk * dk * 4, 256) + round_up((size_t)B * H * dv * dk * 4, 256)) * 2;
+    return n;
+}
+
+mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
+                              const float* gamma, const float* beta, const float* lambda,
+                              int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                              int cg_steps, float tol,
+                              float* out, int32_t* iters_out,
+                              const float* H_in, const float* G_in,
+                              float* H_out, float* G_out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    mesa_status s = check_shape(B, H, T, dk, dv, chunk, dtype, cg_steps, tol);
+    if (s != MESA_OK) return s;
+    if (!lambda) return MESA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !gamma || !beta || !out)) return MESA_ERR_INVALID_ARG;
+    if ((H_out && H_out == H_in) || (G_out && G_out == G_in)) return MESA_ERR_INVALID_ARG;
+    const size_t need = mesa_forward_host_workspace_size(B, H, T, dk, dv, chunk, dtype);
+    if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    const size_t tok = (size_t)B * H * T;
+    const size_t es = elem_size(dtype);
+    char* w = static_cast<char*>(workspace);
+    const size_t fws = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256);
+    char* cur = w + fws;
+    auto carve = [&](size_t bytes) { char* p = cur; cur += round_up(bytes, 256); return p; };
+    void* dq = carve(tok * dk * es);
+    void* dk_ = carve(tok * dk * es);
+    void* dv_ = carve(tok * dv * es);
+    float* dg = reinterpret_cast<float*>(carve(tok * 4));
+    float* db = reinterpret_cast<float*>(carve(tok * 4));
+    float* dl = reinterpret_cast<float*>(carve((size_t)H * dk * 4));
+    float* dout = reinterpret_cast<float*>(carve(tok * dv * 4));
+    int32_t* dit = reinterpret_cast<int32_t*>(carve(tok * 4));
+    const size_t sb = (size_t)B * H * dk * dk * 4, gb = (size_t)B * H * dv * dk * 4;
+    float* dHi = reinterpret_cast<float*>(carve(sb));
+    float* dGi = reinterpret_cast<float*>(carve(gb));
+    float* dHo = reinterpret_cast<float*>(carve(sb));
+    float* dGo = reinterpret_cast<float*>(carve(gb));
+
+    auto h2d = [&](void* dst, const void* src, size_t bytes) {
+        return bytes == 0 || cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    };
+    auto d2h = [&](void* dst, const void* src, size_t bytes) {
+        return bytes == 0 || cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    };
+    bool ok = true;
+    if (T > 0) {
+        ok = ok && h2d(dq, q, tok * dk * es) && h2d(dk_, k, tok * dk * es) && h2d(dv_, v, tok * dv * es);
+        ok = ok && h2d(dg, gamma, tok * 4) && h2d(db, beta, tok * 4);
+    }
+    ok = ok && h2d(dl, lambda, (size_t)H * dk * 4);
+    if (H_in) ok = ok && h2d(dHi, H_in, sb);
+    if (G_in) ok = ok && h2d(dGi, G_in, gb);
+    if (!ok) return MESA_ERR_CUDA;
+    ForwardArgs a{dq, dk_, dv_, dg, db, dl, B, H, T, dk, dv, chunk, dtype, cg_steps, tol,
+                  dout, iters_out ? dit : nullptr, H_in ? dHi : nullptr, G_in ? dGi : nullptr,
+                  H_out ? dHo : nullptr, G_out ? dGo : nullptr, w, fws};
+    s = launch_forward(a, st);
+    if (s != MESA_OK) return s;
+    if (T > 0) ok = ok && d2h(out, dout, tok * dv * 4);
+    if (T > 0 && iters_out) ok = ok && d2h(iters_out, dit, tok * 4);
+    if (H_out) ok = ok && d2h(H_out, dHo, sb);
+    if (G_out) ok = ok && d2h(G_out, dGo, gb);
+    if (!ok) return MESA_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+mesa_status mesa_step(const float* q, const float* k, const float* v,
+                      const float* gamma, const float* beta, const float* lambda,
+                      int B, int H, int dk, int dv,
+                      float* Hstate, float* Gstate,
+                      int cg_steps, float tol,
+                      float* out, int32_t* iters_out, void* stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return MESA_ERR_INVALID_ARG;
+    if (cg_steps < 0 || cg_steps > 1024 || isnan(tol)) return MESA_ERR_INVALID_ARG;
+    if (!supported_width(dk) || dk != dv) return MESA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL) return MESA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gamma || !beta || !lambda || !Hstate || !Gstate || !out) return MESA_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)q, (const void*)k, (const void*)v, (const void*)Hstate,
+                          (const void*)Gstate, (const void*)out})
+        if (!aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    if (!aligned(gamma, 4) || !aligned(beta, 4) || !aligned(lambda, 4)) return MESA_ERR_INVALID_ARG;
+    if (iters_out && !aligned(iters_out, 4)) return MESA_ERR_INVALID_ARG;
+    if (Hstate == Gstate) return MESA_ERR_INVALID_ARG;
+    StepArgs a{q, k, v, gamma, beta, lambda, B, H, dk, dv, Hstate, Gstate, cg_steps, tol, out, iters_out};
+    return step_launch(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+mesa_status mesa_timing_enable(int on) {
+    g_timing_on = on != 0;
+    return MESA_OK;
+}
+
+int mesa_timing_read(const char** names, int* launches, double* total_ms, int max) {
+    int counts[kKindCount] = {0};
+    double ms[kKindCount] = {0.0};
+    int rc = 0;
+    for (const TimingRec& r : g_recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            rc = -1;
+        counts[r.kind] += 1;
+        ms[r.kind] += t;
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.stop);
+    }
+    g_recs.clear();
+    if (rc < 0) return -1;
+    int n = 0;
+    for (int k = 0; k < kKindCount && n < max; ++k) {
+        if (counts[k] == 0) continue;
+        if (names) names[n] = kKindNames[k];
+        if (launches) launches[n] = counts[k];
+        if (total_ms) total_ms[n] = ms[k];
+        ++n;
+    }
+    return n;
+}
+
+mesa_status mesa_get_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MESA_ERR_CUDA;
+    unsigned w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return MESA_ERR_CUDA;
+    if (w == 0) return MESA_OK;
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return MESA_ERR_CUDA;
+    return MESA_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

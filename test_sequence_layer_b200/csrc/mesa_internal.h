@@ -1,0 +1,80 @@
+// mesa_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mesa.h"
+
+namespace mesa {
+
+// Validated arguments of one forward call (device pointers).
+struct ForwardArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* gamma;
+    const float* beta;
+    const float* lambda;
+    int B, H, T, dk, dv, chunk;
+    mesa_dtype dtype;
+    int cg_steps;
+    float tol;
+    float* out;
+    int32_t* iters;
+    const float* H_in;
+    const float* G_in;
+    float* H_out;
+    float* G_out;
+    void* workspace;
+    size_t ws_bytes;
+};
+
+// Device address of the calling device's error word (nullptr on failure).
+unsigned* error_word_ptr();
+
+// Kernel kinds for the optional timing records (mesa_timing_enable).
+enum KernelKind : int { kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindCount };
+
+// Brackets one launch with CUDA events on `st` while timing is enabled.
+class LaunchTimer {
+  public:
+    LaunchTimer(int kind, cudaStream_t st);
+    ~LaunchTimer();
+    LaunchTimer(const LaunchTimer&) = delete;
+    LaunchTimer& operator=(const LaunchTimer&) = delete;
+
+  private:
+    int slot_;
+    cudaStream_t st_;
+};
+
+// fp32 CUDA-core path (simt_forward.cu).
+size_t simt_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
+cudaError_t forward_simt(const ForwardArgs& a, cudaStream_t st);
+
+// Tensor-core path (tc_forward.cu): bf16 inputs, dk = dv = 128, chunk = 64.
+bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype);
+size_t tc_workspace_bytes(int B, int H, int T);
+cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st);
+
+// Decode step (decode.cu).
+struct StepArgs {
+    const float* q;
+    const float* k;
+    const float* v;
+    const float* gamma;
+    const float* beta;
+    const float* lambda;
+    int B, H, dk, dv;
+    float* Hs;
+    float* Gs;
+    int cg_steps;
+    float tol;
+    float* out;
+    int32_t* iters;
+};
+cudaError_t step_launch(const StepArgs& a, cudaStream_t st);
+
+}  // namespace mesa

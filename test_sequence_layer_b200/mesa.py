@@ -1,0 +1,195 @@
+"""ctypes binding of libmesa_b200.so (argument marshalling only).
+
+Every step of the layer runs in the library's CUDA kernels; this module only
+turns torch tensors into the pointers, sizes and stream the C ABI takes
+(include/mesa.h) and turns status codes into exceptions. There is no
+fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmesa_b200.so")
+_lib = None
+
+MESA_F32, MESA_BF16 = 0, 1
+_STATUS = {0: "MESA_OK", 1: "MESA_ERR_INVALID_ARG", 2: "MESA_ERR_UNSUPPORTED", 3: "MESA_ERR_WORKSPACE",
+           4: "MESA_ERR_CUDA", 5: "MESA_ERR_DEVICE_TIMEOUT"}
+
+
+class MesaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing; build it with `python -m test_sequence_layer_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    fwd = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, Z, P]
+    lib.mesa_forward.argtypes = fwd
+    lib.mesa_forward.restype = I
+    lib.mesa_forward_host.argtypes = fwd
+    lib.mesa_forward_host.restype = I
+    lib.mesa_forward_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.mesa_forward_workspace_size.restype = Z
+    lib.mesa_forward_host_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.mesa_forward_host_workspace_size.restype = Z
+    lib.mesa_step.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, I, F, P, P, P]
+    lib.mesa_step.restype = I
+    lib.mesa_get_error.argtypes = [P]
+    lib.mesa_get_error.restype = I
+    lib.mesa_status_string.argtypes = [I]
+    lib.mesa_status_string.restype = ctypes.c_char_p
+    lib.mesa_version.argtypes = []
+    lib.mesa_version.restype = I
+    lib.mesa_timing_enable.argtypes = [I]
+    lib.mesa_timing_enable.restype = I
+    lib.mesa_timing_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(I),
+                                     ctypes.POINTER(ctypes.c_double), I]
+    lib.mesa_timing_read.restype = I
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MESA_F32
+    if t.dtype == torch.bfloat16:
+        return MESA_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise MesaError(rc, where)
+
+
+def workspace_size(B, H, T, dk, dv, chunk, dtype=torch.bfloat16) -> int:
+    code = MESA_BF16 if dtype == torch.bfloat16 else MESA_F32
+    return int(_load().mesa_forward_workspace_size(B, H, T, dk, dv, chunk, code))
+
+
+def forward(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None,
+            return_iters=False, H_in=None, G_in=None, return_state=False, workspace=None,
+            stream=None):
+    """Chunkwise-parallel Mesa forward on CUDA tensors.
+
+    q, k: [B,H,T,dk]; v: [B,H,T,dv] (float32 or bfloat16, same dtype);
+    gamma, beta: [B,H,T] float32; lam: [H,dk] float32.
+    Returns out [B,H,T,dv] float32, plus iters [B,H,T] int32 if return_iters,
+    plus (H_out, G_out) if return_state.
+    """
+    lib = _load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32, device=dev)
+    iters = torch.empty((B, H, T), dtype=torch.int32, device=dev) if return_iters else None
+    H_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev) if return_state else None
+    G_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev) if return_state else None
+    need = int(lib.mesa_forward_workspace_size(B, H, T, dk, dv, chunk, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.mesa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                          B, H, T, dk, dv, chunk, code, int(cg_steps), float(tol),
+                          _ptr(out), _ptr(iters), _ptr(H_in), _ptr(G_in), _ptr(H_out), _ptr(G_out),
+                          _ptr(workspace), ws_bytes, _stream(stream, dev))
+    _check(rc, "mesa_forward")
+    res = (out,)
+    if return_iters:
+        res += (iters,)
+    if return_state:
+        res += (H_out, G_out)
+    return res[0] if len(res) == 1 else res
+
+
+def forward_host(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None,
+                 iters=None, H_in=None, G_in=None, H_out=None, G_out=None, workspace=None,
+                 device=None, stream=None):
+    """Forward with HOST (CPU, ideally pinned) tensors; the library copies them to the
+    device, runs the forward and copies results back before returning."""
+    lib = _load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32)
+    need = int(lib.mesa_forward_host_workspace_size(B, H, T, dk, dv, chunk, code))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.mesa_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                               B, H, T, dk, dv, chunk, code, int(cg_steps), float(tol),
+                               _ptr(out), _ptr(iters), _ptr(H_in), _ptr(G_in), _ptr(H_out), _ptr(G_out),
+                               _ptr(workspace), ws_bytes, _stream(stream, device))
+    _check(rc, "mesa_forward_host")
+    return out
+
+
+def step(q, k, v, gamma, beta, lam, Hstate, Gstate, *, cg_steps=15, tol=0.0, out=None,
+         iters=None, stream=None):
+    """One decode step; Hstate [B,H,dk,dk] and Gstate [B,H,dv,dk] (float32) are
+    updated in place. q, k: [B,H,dk]; v: [B,H,dv]; gamma, beta: [B,H]."""
+    lib = _load()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=torch.float32, device=q.device)
+    rc = lib.mesa_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam), B, H, dk, dv,
+                       _ptr(Hstate), _ptr(Gstate), int(cg_steps), float(tol), _ptr(out), _ptr(iters),
+                       _stream(stream, q.device))
+    _check(rc, "mesa_step")
+    return out
+
+
+def get_error(stream=None) -> int:
+    """Synchronises the stream and reads/clears the device error word (0 = none)."""
+    lib = _load()
+    s = ctypes.c_void_p(None) if stream is None else ctypes.c_void_p(stream.cuda_stream)
+    return int(lib.mesa_get_error(s))
+
+
+def timing_enable(on: bool = True):
+    """Bracket every library kernel launch with CUDA events on its stream."""
+    _load().mesa_timing_enable(1 if on else 0)
+
+
+def timing_read() -> dict:
+    """{kernel kind: (launches, total device ms)} since the last read (synchronises)."""
+    lib = _load()
+    n = 16
+    names = (ctypes.c_char_p * n)()
+    launches = (ctypes.c_int * n)()
+    ms = (ctypes.c_double * n)()
+    k = lib.mesa_timing_read(names, launches, ms, n)
+    if k < 0:
+        raise MesaError(4, "mesa_timing_read")
+    return {names[i].decode(): (int(launches[i]), float(ms[i])) for i in range(k)}

@@ -1,0 +1,118 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+symbol include/mesa.h declares, and rejects bad arguments on the host before
+any launch (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from test_sequence_layer_b200 import build, mesa
+    build.build()
+    return mesa._load()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(mesa_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"mesa_forward", "mesa_step", "mesa_forward_workspace_size", "mesa_get_error",
+            "mesa_status_string", "mesa_forward_host"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["MESA_OK", "MESA_ERR_INVALID_ARG", "MESA_ERR_UNSUPPORTED",
+                                 "MESA_ERR_WORKSPACE", "MESA_ERR_CUDA", "MESA_ERR_DEVICE_TIMEOUT"]):
+        assert lib.mesa_status_string(code).decode() == name
+    assert lib.mesa_status_string(99).decode() == "MESA_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    f = lib.mesa_forward_workspace_size
+    assert f(1, 1, 64, 16, 16, 16, 0) == 4 * (16 * 16 * 2) * 4            # 4 chunks x (H + G) fp32
+    assert f(1, 1, 65, 16, 16, 16, 0) == 5 * (16 * 16 * 2) * 4            # ragged tail adds a chunk
+    assert f(8, 16, 8192, 128, 128, 64, 1) > 0
+    assert f(0, 1, 64, 16, 16, 16, 0) == 0                                # invalid
+    assert f(1, 1, 64, 48, 48, 16, 0) == 0                                # unsupported width
+    assert f(1, 1, 64, 16, 32, 16, 0) == 0                                # dk != dv
+    assert f(1, 1, 64, 16, 16, 24, 0) == 0                                # unsupported chunk
+    assert lib.mesa_forward_host_workspace_size(1, 1, 64, 16, 16, 16, 0) > f(1, 1, 64, 16, 16, 16, 0)
+
+
+FAKE = 1 << 20   # aligned, never dereferenced: every call below is rejected first
+
+
+def fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gamma=FAKE, beta=FAKE, lam=FAKE, B=1, H=1, T=64, dk=16, dv=16,
+             chunk=16, dtype=0, N=8, tol=0.0, out=FAKE, iters=None, Hi=None, Gi=None, Ho=None, Go=None,
+             ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return lib.mesa_forward(a["q"], a["k"], a["v"], a["gamma"], a["beta"], a["lam"], a["B"], a["H"], a["T"],
+                            a["dk"], a["dv"], a["chunk"], a["dtype"], a["N"], ctypes.c_float(a["tol"]),
+                            a["out"], a["iters"], a["Hi"], a["Gi"], a["Ho"], a["Go"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(gamma=None), 1), (dict(beta=None), 1),
+    (dict(lam=None), 1), (dict(out=None), 1),
+    (dict(B=0), 1), (dict(H=-1), 1), (dict(T=-5), 1), (dict(dtype=7), 1),
+    (dict(N=-1), 1), (dict(N=5000), 1), (dict(tol=float("nan")), 1),
+    (dict(dk=48, dv=48), 2), (dict(dk=16, dv=32), 2), (dict(chunk=24), 2), (dict(B=300, H=300), 2),
+    (dict(q=FAKE + 8), 1), (dict(out=FAKE + 4), 1), (dict(gamma=FAKE + 2), 1), (dict(iters=FAKE + 2), 1),
+    (dict(Hi=FAKE + 4), 1), (dict(Ho=FAKE, Hi=FAKE), 1),
+    (dict(ws=None), 3), (dict(wsb=100), 3), (dict(ws=FAKE + 16), 1),
+])
+def test_forward_rejects_bad_arguments(lib, kw, code):
+    assert fwd(lib, **kw) == code
+
+
+def step(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gamma=FAKE, beta=FAKE, lam=FAKE, B=2, H=2, dk=16, dv=16,
+             Hs=FAKE, Gs=FAKE + 4096, N=8, tol=0.0, out=FAKE, iters=None)
+    a.update(kw)
+    return lib.mesa_step(a["q"], a["k"], a["v"], a["gamma"], a["beta"], a["lam"], a["B"], a["H"], a["dk"],
+                         a["dv"], a["Hs"], a["Gs"], a["N"], ctypes.c_float(a["tol"]), a["out"], a["iters"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(Hs=None), 1), (dict(Gs=None), 1), (dict(out=None), 1), (dict(lam=None), 1),
+    (dict(B=0), 1), (dict(N=-2), 1), (dict(tol=float("nan")), 1),
+    (dict(dk=24, dv=24), 2), (dict(dk=16, dv=64), 2),
+    (dict(q=FAKE + 4), 1), (dict(Hs=FAKE + 8), 1), (dict(Gs=FAKE), 1),
+])
+def test_step_rejects_bad_arguments(lib, kw, code):
+    assert step(lib, **kw) == code
+
+
+def test_host_variant_rejects_bad_arguments(lib):
+    f = lib.mesa_forward_host
+    args = [FAKE] * 6 + [1, 1, 64, 16, 16, 16, 0, 8, ctypes.c_float(0.0), FAKE, None, None, None, None, None]
+    assert f(*args, None, 0, None) == 3                               # no workspace
+    bad = list(args)
+    bad[8] = -1
+    assert f(*bad, FAKE, 1 << 30, None) == 1
+    assert f(*args, FAKE + 64, 1 << 30, None) == 1                    # misaligned workspace
+
+
+def test_product_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "test_sequence_layer_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert "oracle" not in src.lower().replace("oracles", ""), fn
