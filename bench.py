@@ -196,7 +196,7 @@ def main():
 
     def step():
         mesa.forward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], chunk=C, cg_steps=w.cg_steps,
-                     tol=w.tol, out=out, return_iters=True, workspace=ws, stream=stream)
+                     tol=w.tol, out=out, iters=iters, return_iters=True, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -288,8 +288,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = host_cores()
-        n_seq = min(w.B * w.H, max(cores, 1))
-        T_s = min(w.T, 1024)
+        n_seq = min(w.B * w.H, 8 * max(cores, 1))
+        T_s = min(w.T, 4096)
         rate, dt = cpu_oracle_sample(w, n_seq, T_s)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n_seq} sequences x first {T_s} tokens of {w.name} ({dt:.1f} s, OpenMP over sequences)"}

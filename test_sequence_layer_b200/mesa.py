@@ -94,14 +94,14 @@ def workspace_size(B, H, T, dk, dv, chunk, dtype=torch.bfloat16) -> int:
 
 
 def forward(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None,
-            return_iters=False, H_in=None, G_in=None, return_state=False, workspace=None,
+            return_iters=False, iters=None, H_in=None, G_in=None, return_state=False, workspace=None,
             stream=None):
     """Chunkwise-parallel Mesa forward on CUDA tensors.
 
     q, k: [B,H,T,dk]; v: [B,H,T,dv] (float32 or bfloat16, same dtype);
     gamma, beta: [B,H,T] float32; lam: [H,dk] float32.
-    Returns out [B,H,T,dv] float32, plus iters [B,H,T] int32 if return_iters,
-    plus (H_out, G_out) if return_state.
+    Returns out [B,H,T,dv] float32, plus iters [B,H,T] int32 if return_iters
+    (written into `iters` when given), plus (H_out, G_out) if return_state.
     """
     lib = _load()
     B, H, T, dk = q.shape
@@ -110,7 +110,8 @@ def forward(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=No
     dev = q.device
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=torch.float32, device=dev)
-    iters = torch.empty((B, H, T), dtype=torch.int32, device=dev) if return_iters else None
+    if return_iters and iters is None:
+        iters = torch.empty((B, H, T), dtype=torch.int32, device=dev)
     H_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev) if return_state else None
     G_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev) if return_state else None
     need = int(lib.mesa_forward_workspace_size(B, H, T, dk, dv, chunk, code))
