@@ -1,0 +1,193 @@
+// tc_common.cuh -- thin wrappers over the sm_100a tensor-core instructions used
+// by the tensor-core path (tcgen05 MMA/TMEM, mbarriers, bulk async copies).
+//
+// Layout facts these wrappers rely on (checked on B200 before use):
+//   * Shared-memory matrix descriptors use the 128-byte swizzle. A K-major
+//     tile is stored as blocks of 64 16-bit elements per 128-byte row, 8-row
+//     atoms of 1024 bytes (SBO = 1024); the K=16 slice s of a block starts
+//     32*s bytes in. An MN-major tile stores 64 MN elements per 128-byte row
+//     with one row per K index; LBO is the byte stride between 64-wide MN
+//     blocks, SBO = 1024 between groups of 8 K rows, and a K=16 step
+//     advances 2048 bytes.
+//   * An M=128 accumulator puts row m in TMEM lane m, column n in column n.
+//     An M=64 accumulator puts rows 16g..16g+15 in lanes 32g..32g+15.
+//   * tcgen05.ld/st .16x256b: thread t of the warp gets lanes (base + t/4)
+//     and (base + t/4 + 8), columns 2*(t%4) and 2*(t%4)+1 of each 8-column
+//     group; registers 4g..4g+3 of the .xN form hold group g as
+//     (lane t/4, col), (lane t/4, col+1), (lane t/4+8, col), (lane t/4+8, col+1).
+//   * tcgen05.ld .32x32b: thread t gets lane base + t, consecutive columns.
+#pragma once
+
+#include <stdint.h>
+
+namespace mesa {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;                      // descriptor version for sm_100
+    d |= 2ull << 61;                      // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                                    // D format: f32
+           | (0u << 7) | (0u << 10)                     // A, B format: f16
+           | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16)
+           | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// Waits until the phase of `bar` with the given parity has completed, for at
+// most ~2e9 cycles. Returns false if the wait gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_addr(bar);
+    uint32_t done = 0;
+    const long long t0 = clock64();
+    while (true) {
+        asm volatile(
+            "{\n .reg .pred w;\n mbarrier.try_wait.parity.shared::cta.b64 w, [%1], %2;\n selp.u32 %0, 1, 0, w;\n}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > 2000000000ll) return false;
+    }
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk (non-tensor) asynchronous copy global -> shared, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Warp-wide TMEM allocation; the base address is written to *slot.
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D (+)= A * B^T with both operands in shared memory.
+__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on `bar` when every previously issued MMA of this thread is done.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+#define MESA_R4(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3])
+
+__device__ __forceinline__ void tmem_ld16_x4(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : MESA_R4(0), MESA_R4(4), MESA_R4(8), MESA_R4(12)
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld16_x8(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : MESA_R4(0), MESA_R4(4), MESA_R4(8), MESA_R4(12), MESA_R4(16), MESA_R4(20), MESA_R4(24), MESA_R4(28)
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+#define MESA_W4(i) "r"(__float_as_uint(v[i])), "r"(__float_as_uint(v[i + 1])), "r"(__float_as_uint(v[i + 2])), \
+                   "r"(__float_as_uint(v[i + 3]))
+
+__device__ __forceinline__ void tmem_st16_x8(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        MESA_W4(0), MESA_W4(4), MESA_W4(8), MESA_W4(12), MESA_W4(16), MESA_W4(20), MESA_W4(24), MESA_W4(28)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16_x4(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        MESA_W4(0), MESA_W4(4), MESA_W4(8), MESA_W4(12)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive columns (thread t: lane base + t).
+__device__ __forceinline__ void tmem_ld32_x32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : MESA_R4(0), MESA_R4(4), MESA_R4(8), MESA_R4(12), MESA_R4(16), MESA_R4(20), MESA_R4(24), MESA_R4(28)
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+#undef MESA_R4
+#undef MESA_W4
+
+// Byte offset of element (row, col) in a K-major 128-byte-swizzled tile of
+// 16-bit elements whose rows hold `row_blocks` rows per 64-column block.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int col, int rows_per_block) {
+    const int blk = col >> 6, c = col & 63;
+    return static_cast<uint32_t>(blk * rows_per_block * 128 + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) +
+                                 ((c & 7) << 1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace tc
+}  // namespace mesa
