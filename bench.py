@@ -258,8 +258,7 @@ def main():
     if not args.no_e2e:
         hx = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "gamma", "beta", "lam")}
         hout = torch.empty((B, H, T, d)).pin_memory()
-        hws = torch.empty(mesa.mesa._load().mesa_forward_host_workspace_size(
-            B, H, T, d, d, C, 1 if x["q"].dtype == torch.bfloat16 else 0), dtype=torch.uint8, device=dev)
+        hws = torch.empty(mesa.host_workspace_size(B, H, T, d, d, C, x["q"].dtype), dtype=torch.uint8, device=dev)
         del ws
         e_steps = max(3, args.steps // 4)
 

@@ -93,6 +93,11 @@ def workspace_size(B, H, T, dk, dv, chunk, dtype=torch.bfloat16) -> int:
     return int(_load().mesa_forward_workspace_size(B, H, T, dk, dv, chunk, code))
 
 
+def host_workspace_size(B, H, T, dk, dv, chunk, dtype=torch.bfloat16) -> int:
+    code = MESA_BF16 if dtype == torch.bfloat16 else MESA_F32
+    return int(_load().mesa_forward_host_workspace_size(B, H, T, dk, dv, chunk, code))
+
+
 def forward(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None,
             return_iters=False, iters=None, H_in=None, G_in=None, return_state=False, workspace=None,
             stream=None):
