@@ -112,6 +112,42 @@ mesa_status mesa_forward(const void* q, const void* k, const void* v,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Size of the fixed device scratch array behind mesa_forward_noalloc.
+ */
+#define MESA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * mesa_forward without a workspace argument, for callers that cannot
+ * allocate device memory at all: plug-in code inside a host framework that
+ * owns every device allocation and passes in only its tensors, or latency-
+ * bound loops that must never call cudaMalloc (which can synchronise the
+ * device). The MesaNet pages have no counterpart to this entry point; it
+ * exists for those callers only.
+ *
+ * Arguments, layouts and results are exactly those of mesa_forward minus
+ * `workspace` and `ws_bytes`. The scratch the forward needs (chunk-start
+ * states) comes from a library-owned device array of
+ * MESA_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU loading the library
+ * holds until the process exits. Nothing is allocated by the call.
+ *   - Sizes whose scratch (mesa_forward_workspace_size) exceeds
+ *     MESA_NOALLOC_SCRATCH_BYTES are refused with MESA_ERR_WORKSPACE before
+ *     any device work.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the previous call's
+ *     contents; every byte is written before it is read, so no clearing is
+ *     needed. Calls that overlap on the GPU (different streams, or host
+ *     threads without ordering) race on the array: serialise them.
+ */
+mesa_status mesa_forward_noalloc(const void* q, const void* k, const void* v,
+                                 const float* gamma, const float* beta, const float* lambda,
+                                 int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                                 int cg_steps, float tol,
+                                 float* out, int32_t* iters_out,
+                                 const float* H_in, const float* G_in,
+                                 float* H_out, float* G_out, void* stream);
+
+/*
  * Bytes of device workspace mesa_forward_host needs: the mesa_forward
  * workspace plus device staging for every tensor argument.
  */

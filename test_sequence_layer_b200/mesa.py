@@ -199,3 +199,25 @@ def timing_read() -> dict:
     if k < 0:
         raise MesaError(4, "mesa_timing_read")
     return {names[i].decode(): (int(launches[i]), float(ms[i])) for i in range(k)}
+
+
+def forward_noalloc(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None, iters=None,
+                    H_in=None, G_in=None, H_out=None, G_out=None, stream=None):
+    """mesa_forward_noalloc: the forward for callers that cannot allocate device
+    memory; its scratch is a fixed library-owned device array (sizes beyond it
+    raise MesaError MESA_ERR_WORKSPACE)."""
+    lib = _load()
+    if not getattr(lib, "_noalloc_typed", False):
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.mesa_forward_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, P, P, P, P]
+        lib.mesa_forward_noalloc.restype = I
+        lib._noalloc_typed = True
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32, device=q.device)
+    rc = lib.mesa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam), B, H, T, dk, dv,
+                                  chunk, _dtype_code(q), int(cg_steps), float(tol), _ptr(out), _ptr(iters),
+                                  _ptr(H_in), _ptr(G_in), _ptr(H_out), _ptr(G_out), _stream(stream, q.device))
+    _check(rc, "mesa_forward_noalloc")
+    return out
