@@ -60,6 +60,14 @@ __device__ __forceinline__ float pow2_ceil_at_least_one(float m) {
     return ldexpf(1.f, f == 0.5f ? e - 1 : e);
 }
 
+// Power of two 2^floor(e/2) with 2^e <= rr < 2^(e+1): a scale within a factor
+// sqrt(2) of |r| whose reciprocal is exact (1 for rr <= 0 or denormal rr).
+__device__ __forceinline__ float pow2_sqrt_scale(float rr) {
+    const int e = ((__float_as_int(rr) >> 23) & 0xff) - 127;
+    if (!(rr > 0.f) || e <= -126 || e >= 127) return 1.f;
+    return __int_as_float((((e >> 1) + 127) & 0xff) << 23);
+}
+
 // Inclusive log-cumsum of gamma over a 64-token chunk by warp 0 (padded
 // tokens count as gamma = 1).
 __device__ __forceinline__ void chunk_gates(const float* __restrict__ gamma, size_t base, int n, float* b) {
@@ -318,11 +326,13 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             }
             mma_commit(bar_mma);
         }
-        // bound update (every thread, same order -> identical value)
+        // bound update: every warp reduces the same 64 terms in the same order,
+        // so every thread of every CTA of this sequence gets the same value
         {
             const float* km = m ? kmax : amax;
-            float add = 0.f;
-            for (int j = 0; j < n; ++j) add = fmaf(sw[j], amax[j] * km[j], add);
+            float add = sw[lane] * (amax[lane] * km[lane]) + sw[lane + 32] * (amax[lane + 32] * km[lane + 32]);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) add += __shfl_xor_sync(0xffffffffu, add, off);
             bound = fmaf(expf(blast), bound, add);
         }
         if (tid == 0 && !mbar_wait(bar_mma, mma_phase & 1)) red[15] = 1.f;
@@ -373,8 +383,8 @@ struct CgSmem {
     static constexpr int oB = oEb + 256;          // b_t [64]
     static constexpr int oRed = oB + 256;         // [2 halves][64 tokens][4] partial sums
     static constexpr int oMisc = oRed + 2048;     // 16 floats / flags
-    static constexpr int oBar = oMisc + 64;       // 2 mbarriers
-    static constexpr int oSlot = oBar + 16;
+    static constexpr int oBar = oMisc + 64;       // 3 mbarriers
+    static constexpr int oSlot = oBar + 32;
     static constexpr int bytes = oSlot + 16;
 };
 
@@ -437,6 +447,14 @@ __device__ __forceinline__ bool wait_mma_cta(uint64_t* bar, uint32_t parity, int
     return *abort_flag == 0.f;
 }
 
+// Every thread waits on the MMA barrier itself (no CTA barrier); a thread
+// whose bounded wait gave up raises the abort flag, which the next CTA
+// barrier makes visible to all.
+__device__ __forceinline__ void wait_mma_each(uint64_t* bar, uint32_t parity, float* abort_flag) {
+    if (!mbar_wait(bar, parity)) *abort_flag = 1.f;
+    tc_fence_after();
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
 tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
              const __nv_bfloat16* __restrict__ v, const float* __restrict__ gamma,
@@ -458,7 +476,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     float* misc = reinterpret_cast<float*>(smem + CgSmem::oMisc);
     float* abort_flag = misc + 15;
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + CgSmem::oBar);
-    uint64_t* bar_mma = bar_ld + 1;
+    uint64_t* bar_s = bar_ld + 1;        // scores S ready
+    uint64_t* bar_y = bar_ld + 2;        // Y = U + Z ready
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + CgSmem::oSlot);
 
     const int c = blockIdx.x, bh = blockIdx.y, head = bh % H;
@@ -482,7 +501,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     // ---- set-up: barriers, TMEM, async load of the H_c image ----
     if (tid == 0) {
         mbar_init(bar_ld, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_y, 1);
         fence_mbar_init();
         *abort_flag = 0.f;
     }
@@ -491,7 +511,12 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *slot;
+    // TMEM: columns [0,128) lanes 16g..16g+15 (M=64 rows) hold Y = U + Z; the
+    // idle lanes 16g+16..16g+31 of the same columns hold x (same token order);
+    // columns [128,192) hold the scores S.
     const uint32_t tq = tbase + ((uint32_t)(32 * q4) << 16);    // this warp's lane quadrant
+    const uint32_t tx = tq + (16u << 16);                        // ... and its x lanes
+    constexpr uint32_t kColS = 128;
     if (tid == 0) {
         mbar_arrive_expect_tx(bar_ld, kImgBytes);
         bulk_g2s(Hs, Himg, kImgBytes, bar_ld);
@@ -533,7 +558,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.f;
-        tmem_st16_x8(tq + 128 + 64 * hh, z);
+        tmem_st16_x8(tx + 64 * hh, z);
         tmem_wait_st();
     }
     float rr0, rr1;
@@ -552,9 +577,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     bool act0 = tok0 < n, act1 = tok1 < n;
     int it0 = 0, it1 = 0;
     const float eb0 = seb[tok0], eb1 = seb[tok1];
-    float s0 = rr0 > 0.f ? sqrtf(rr0) : 1.f, s1 = rr1 > 0.f ? sqrtf(rr1) : 1.f;
-    store_rows(Ps + row0, Ps + row1, phase, p0, p1, 1.f / s0, 1.f / s1);
-    store_rows(Pt + row0, Pt + row1, phase, p0, p1, eb0 / s0, eb1 / s1);
+    float s0 = pow2_sqrt_scale(rr0), s1 = pow2_sqrt_scale(rr1);
+    float is0 = 1.f / s0, is1 = 1.f / s1;                   // exact: powers of two
+    store_rows(Ps + row0, Ps + row1, phase, p0, p1, is0, is1);
+    store_rows(Pt + row0, Pt + row1, phase, p0, p1, eb0 * is0, eb1 * is1);
 
     // MMA issue (one thread). Descriptor address fields are the low 14 bits,
     // so byte offsets (>> 4) add directly.
@@ -566,25 +592,27 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint32_t ko = ((ks >> 2) * 8192 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase, dA + ko, dK + ko, kIdS, ks > 0 ? 1u : 0u);
+            mma_f16(tbase + kColS, dA + ko, dK + ko, kIdS, ks > 0 ? 1u : 0u);
         }
     };
-    auto issue_UZ = [&](const uint8_t* A) {  // Y = A Hs^T + W Kmn: M=64, N=128
-        const uint64_t dA = sdesc(smem_addr(A), 16, 1024), dH = sdesc(smem_addr(Hs), 16, 1024);
-        const uint64_t dW = sdesc(smem_addr(Ws), 16, 1024), dKmn = sdesc(smem_addr(Ks), 8192, 1024);
+    auto issue_U = [&](const uint8_t* A, const uint8_t* B) {   // Y = A B^T: M=64, N=128, K=128
+        const uint64_t dA = sdesc(smem_addr(A), 16, 1024), dB = sdesc(smem_addr(B), 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint32_t ka = ((ks >> 2) * 8192 + (ks & 3) * 32) >> 4;
             const uint32_t kb = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase, dA + ka, dH + kb, kIdU, ks > 0 ? 1u : 0u);
+            mma_f16(tbase, dA + ka, dB + kb, kIdU, ks > 0 ? 1u : 0u);
         }
+    };
+    auto issue_Z = [&]() {                   // Y += W Kmn: M=64, N=128, K=64
+        const uint64_t dW = sdesc(smem_addr(Ws), 16, 1024), dKmn = sdesc(smem_addr(Ks), 8192, 1024);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) mma_f16(tbase, dW + ((ks * 32) >> 4), dKmn + ((ks * 2048) >> 4), kIdZ, 1u);
     };
     // S (in TMEM) -> masked, scaled scores -> fp16 image
     auto masked_scores = [&](float extra) {
         float sv[16];
-        tmem_ld16_x4(tq + 32 * hh, sv);
+        tmem_ld16_x4(tq + kColS + 32 * hh, sv);
         tmem_wait_ld();
         const float2 ex = make_float2(extra, extra);
 #pragma unroll
@@ -613,22 +641,24 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tc_fence_after();
         if (!any || *abort_flag != 0.f) break;
 
+        // S first, then U straight behind it: U runs while the scores are masked
         if (tid == 0) {
             issue_S(Ps);
-            mma_commit(bar_mma);
+            mma_commit(bar_s);
+            issue_U(Pt, Hs);
         }
-        if (!wait_mma_cta(bar_mma, mma_phase & 1, tid, abort_flag)) break;
-        ++mma_phase;
+        wait_mma_each(bar_s, mma_phase & 1, abort_flag);
         masked_scores(1.f);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (*abort_flag != 0.f) break;
         if (tid == 0) {
-            issue_UZ(Pt);
-            mma_commit(bar_mma);
+            issue_Z();
+            mma_commit(bar_y);
         }
-        if (!wait_mma_cta(bar_mma, mma_phase & 1, tid, abort_flag)) break;
+        wait_mma_each(bar_y, mma_phase & 1, abort_flag);
         ++mma_phase;
 
         // y = (s sH) Y + lambda p, written back over Y; partials p.y, r.y, y.y, r.r
@@ -682,7 +712,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
         for (int half = 0; half < 2; ++half) {   // x += alpha p (TMEM), r -= alpha y, p = r + rho p
             float xv[16], yv[16];
-            const uint32_t xa = tq + 128 + 64 * hh + 32 * half;
+            const uint32_t xa = tx + 64 * hh + 32 * half;
             tmem_ld16_x4(xa, xv);
             tmem_ld16_x4(tq + 64 * hh + 32 * half, yv);
             tmem_wait_ld();
@@ -706,23 +736,25 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         if (act0) {
             rr0 = rn0;
             ++it0;
-            s0 = rr0 > 0.f ? sqrtf(rr0) : 1.f;
+            s0 = pow2_sqrt_scale(rr0);
+            is0 = 1.f / s0;
         }
         if (act1) {
             rr1 = rn1;
             ++it1;
-            s1 = rr1 > 0.f ? sqrtf(rr1) : 1.f;
+            s1 = pow2_sqrt_scale(rr1);
+            is1 = 1.f / s1;
         }
         tmem_wait_st();
-        store_rows(Ps + row0, Ps + row1, phase, p0, p1, 1.f / s0, 1.f / s1);
-        store_rows(Pt + row0, Pt + row1, phase, p0, p1, eb0 / s0, eb1 / s1);
+        store_rows(Ps + row0, Ps + row1, phase, p0, p1, is0, is1);
+        store_rows(Pt + row0, Pt + row1, phase, p0, p1, eb0 * is0, eb1 * is1);
     }
 
     // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V ----
     float2 xr0[8], xr1[8];
     {
         float xv[32];
-        tmem_ld16_x8(tq + 128 + 64 * hh, xv);
+        tmem_ld16_x8(tx + 64 * hh, xv);
         tmem_wait_ld();
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
@@ -778,10 +810,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             mbar_arrive_expect_tx(bar_ld, kImgBytes);
             bulk_g2s(Hs, Gimg, kImgBytes, bar_ld);
             issue_S(Ps);                       // S' = X-hat K^T
-            mma_commit(bar_mma);
+            mma_commit(bar_s);
         }
-        ok = wait_mma_cta(bar_mma, mma_phase & 1, tid, abort_flag);
-        ++mma_phase;
+        ok = wait_mma_cta(bar_s, mma_phase & 1, tid, abort_flag);
     }
     if (ok) {
         masked_scores(sH * sV / sG);           // mask holds 1/sH
@@ -802,11 +833,12 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             if (!mbar_wait(bar_ld, 1)) {
                 *abort_flag = 1.f;
             } else {
-                issue_UZ(Pt);
-                mma_commit(bar_mma);
+                issue_U(Pt, Hs);               // O = X-tilde G^T + W' V
+                issue_Z();
+                mma_commit(bar_y);
             }
         }
-        ok = wait_mma_cta(bar_mma, mma_phase & 1, tid, abort_flag);
+        ok = wait_mma_cta(bar_y, mma_phase & 1, tid, abort_flag);
         ++mma_phase;
     }
     if (ok) {
@@ -831,7 +863,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     } else {
         if (tid == 0) {
             record_error(err, kErrTimeout);
-            mbar_wait(bar_mma, mma_phase & 1);   // one more bounded chance for in-flight MMAs to drain
+            // one more bounded chance for every MMA issued so far to drain
+            mma_commit(bar_ld);
+            mbar_wait(bar_ld, 0);
+            mbar_wait(bar_ld, 1);
         }
     }
     tc_fence_before();
