@@ -47,6 +47,32 @@ def load_peaks():
     return d
 
 
+# DRAM bytes moved per token by each kernel, from one ncu capture
+# (profiles/tc_kernels_bf16_T2048.md: dram__bytes_read.sum + dram__bytes_write.sum
+# of one launch / tokens of that launch). Reported only while the kernel
+# source still hashes to the captured version; otherwise the field is null.
+MEASURED_TRAFFIC = {
+    "tc_cg": {"src_sha16": "6cb7cfa309f72f83", "bytes_per_token": (471.978752e6 + 117.958912e6) / 262144},
+    "tc_scan": {"src_sha16": "6cb7cfa309f72f83", "bytes_per_token": (136.758016e6 + 213.465856e6) / 262144},
+}
+
+
+def kernel_source_sha16():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("tc_forward.cu", "tc_common.cuh"):
+        with open(os.path.join(ROOT, "test_sequence_layer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel, tokens):
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if rec is None or rec["src_sha16"] != kernel_source_sha16():
+        return None
+    return rec["bytes_per_token"] * tokens
+
+
 def flops_per_token_iter(d, C):
     """Useful causal flops of one CG matvec per token: inter-chunk 2d^2 plus
     the masked intra-chunk scores and their read-back, 2d(C+1)."""
@@ -148,6 +174,97 @@ def run_reference(args, w, rank):
 
 
 METRIC = "Mesa-layer fwd tokens/s (B*H*T) at T=8192,d=128,15 CG steps; % tensor peak"
+DECODE_METRIC = "Mesa decode tokens/s (sequences x heads per mesa_step), d=128, 15 CG steps; % HBM peak"
+
+
+def run_decode(args, w, world, rank, local):
+    """Recurrent decode: a 4096-token prefill through mesa_forward's final
+    state, then timed mesa_step calls (one new token for every head)."""
+    import torch
+    import torch.distributed as dist
+    from test_sequence_layer_b200 import build as mbuild, mesa
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    B, H, d = w.B, w.H, w.dk
+    steps_total = args.warmup + args.steps
+    Hs = torch.empty((B, H, d, d), device=dev)
+    Gs = torch.empty((B, H, d, d), device=dev)
+    dec = {n: [] for n in ("q", "k", "v", "gamma", "beta")}
+    slab = 32
+    for b0 in range(0, B, slab):
+        x = mi.device_batch(w, dev, T=w.T + steps_total, B=slab, seed_offset=1000 * rank + b0)
+        _, Hp, Gp = mesa.forward(*(x[n][:, :, :w.T].contiguous() for n in ("q", "k", "v", "gamma", "beta")),
+                                 x["lam"], chunk=w.chunk, cg_steps=w.cg_steps, return_state=True)
+        Hs[b0:b0 + slab].copy_(Hp)
+        Gs[b0:b0 + slab].copy_(Gp)
+        for n in dec:
+            dec[n].append(x[n][:, :, w.T:].float())
+        del x, Hp, Gp
+    dec = {n: torch.cat(v, 0) for n, v in dec.items()}
+    # one contiguous [steps, B, H, ...] block per input, resident before timing
+    tok = {n: dec[n].movedim(2, 0).contiguous() for n in dec}
+    del dec
+    lam = torch.from_numpy(mi.lambdas(w.seed, w.H, w.dk)).to(dev)
+    out = torch.empty((B, H, d), device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for s in range(args.warmup):
+        mesa.step(tok["q"][s], tok["k"][s], tok["v"][s], tok["gamma"][s], tok["beta"][s], lam, Hs, Gs,
+                  cg_steps=w.cg_steps, out=out, stream=stream)
+    torch.cuda.synchronize()
+    assert mesa.get_error(stream) == 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for s in range(args.warmup, steps_total):
+        mesa.step(tok["q"][s], tok["k"][s], tok["v"][s], tok["gamma"][s], tok["beta"][s], lam, Hs, Gs,
+                  cg_steps=w.cg_steps, out=out, stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    mesa.timing_enable(False)
+    kernels = mesa.timing_read()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.destroy_process_group()
+    assert mesa.get_error(stream) == 0
+    if rank != 0:
+        return
+    heads = B * H
+    launches, kms = kernels["decode_step"]
+    avg_ms = kms / launches
+    # state read + write (H and G, fp32) plus q, k, v, gamma, beta in and out per head
+    bytes_per_launch = heads * (4 * d * d * 4 + (3 * d + 2) * 4 + d * 4)
+    peaks = load_peaks()
+    achieved = bytes_per_launch / (avg_ms / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": world * heads * args.steps / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "sequences": B, "H": H, "d": d, "prefill_tokens": w.T,
+                   "cg_steps": w.cg_steps, "l2": "state larger than L2 (%.2f GB)" % (2 * Hs.numel() * 4 / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "decode_step",
+                     "avg_ms": avg_ms, "peak_kind": f"{peaks['_source']} HBM copy bandwidth"},
+        "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
+        "gpu_launches": sum(v[0] for v in kernels.values()),
+        "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def main():
@@ -155,7 +272,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="bf16_T8192", choices=[k for k in mi.WORKLOADS if k != "decode"])
+    ap.add_argument("--workload", default="bf16_T8192", choices=list(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -170,6 +287,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, rank)
+        return
+    if w.decode_steps > 0:
+        run_decode(args, w, world, rank, local)
         return
 
     import torch
@@ -249,7 +369,7 @@ def main():
         roof = {"bound": "alu", "achieved": achieved, "peak": SIMT_FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                 "peak_kind": "fp32 FMA: 148 SM x 128 FMA/clk x 2 x 1.965 GHz"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(name, tokens)
     roof["kernel"] = name
     roof["avg_ms"] = avg_ms
 
