@@ -129,6 +129,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(value, world, device):
+    """Slowest rank's value (the benchmark's clock for N > 1); identity for N = 1."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Weak scaling: every rank processes `units_per_rank` in `ms` (slowest rank)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def cpu_oracle_sample(w, n_seq, T_s):
     """Times the oracle on n_seq sequences x T_s tokens of workload w; returns tokens/s."""
     import oracle
@@ -235,11 +251,8 @@ def run_decode(args, w, world, rank, local):
     mesa.timing_enable(False)
     kernels = mesa.timing_read()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.destroy_process_group()
     assert mesa.get_error(stream) == 0
     if rank != 0:
@@ -252,7 +265,7 @@ def run_decode(args, w, world, rank, local):
     peaks = load_peaks()
     achieved = bytes_per_launch / (avg_ms / 1e3) / 1e9
     line = {
-        "metric": DECODE_METRIC, "value": world * heads * args.steps / (ms / 1e3), "unit": "tokens/s",
+        "metric": DECODE_METRIC, "value": whole_job_rate(heads * args.steps, world, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "sequences": B, "H": H, "d": d, "prefill_tokens": w.T,
@@ -340,14 +353,10 @@ def main():
     mesa.timing_enable(False)
     kernels = mesa.timing_read()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     assert mesa.get_error(stream) == 0
     ms_per_step = ms / args.steps
-    value = world * tokens / (ms_per_step / 1e3)
+    value = whole_job_rate(tokens, world, ms_per_step)
     total_iters = int(iters.sum().item())
 
     # dominant kernel and its roofline
@@ -395,13 +404,9 @@ def main():
             hstep()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d = sum(hx[n].numel() * hx[n].element_size() for n in ("q", "k", "v", "gamma", "beta", "lam"))
-        e2e = {"value": world * tokens / (ems / e_steps / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(tokens, world, ems / e_steps), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": e_steps}
 
     cpu = None
