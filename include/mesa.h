@@ -30,8 +30,10 @@
  *     each head, shared by the batch); H states [B,H,dk,dk]; G states
  *     [B,H,dv,dk].
  *   - Preconditions on values (not checked, the caller's contract):
- *     0 < gamma <= 1, beta >= 0, lambda > 0, all finite. Non-finite inputs
- *     give non-finite outputs for the affected tokens but never hang.
+ *     0 < gamma <= 1, beta >= 0, lambda > 0, all finite. A non-finite input
+ *     makes the outputs of its chunk (on the tensor-core path: of its pair
+ *     of chunks, which share every MMA) and of every later token of its
+ *     sequence non-finite; it never hangs and touches no other sequence.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Device calls are asynchronous on it.
  *   - Argument errors are returned synchronously and nothing is launched.

@@ -43,6 +43,22 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _configure(lib):
+    """Declares the C signatures on a loaded oracle library."""
+    D = ctypes.POINTER(ctypes.c_double)
+    I32 = ctypes.POINTER(ctypes.c_int32)
+    i, d = ctypes.c_int, ctypes.c_double
+    lib.oracle_forward_cg.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, I32, D, D]
+    lib.oracle_forward_cholesky.argtypes = [D, D, D, D, D, D, i, i, i, i, i, D, D, D, D, D]
+    lib.oracle_forward_chunked.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, i, d, D, D, D, I32, D, D]
+    lib.oracle_step.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, i, d, D, I32]
+    lib.oracle_cg_dense.argtypes = [i, D, D, i, d, D, I32]
+    for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
+              lib.oracle_step, lib.oracle_cg_dense):
+        f.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:

@@ -367,86 +367,6 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     if (w == 0) tmem_dealloc(tbase, 64);
 }
 
-// =====================================================================
-// Fused CG iterations + read-out, one chunk per CTA
-// =====================================================================
-struct CgSmem {
-    static constexpr int oH = 0;                  // H_c image, later G_c   32 KB
-    static constexpr int oK = 32768;              // key image, later value image   16 KB
-    static constexpr int oP = 49152;              // P-hat image, later X-hat  16 KB
-    static constexpr int oPt = 65536;             // P-tilde image, later X-tilde  16 KB
-    static constexpr int oW = 81920;              // masked scores image  8 KB
-    static constexpr int kMStride = 72;           // padded row stride of the decay mask
-    static constexpr int oM = 90112;              // decay mask / sH, fp32 [64][72]
-    static constexpr int oLam = oM + kC * kMStride * 4;   // lambda [128]
-    static constexpr int oEb = oLam + 512;        // e^{b_t} [64]
-    static constexpr int oB = oEb + 256;          // b_t [64]
-    static constexpr int oRed = oB + 256;         // [2 halves][64 tokens][4] partial sums
-    static constexpr int oMisc = oRed + 2048;     // 16 floats / flags
-    static constexpr int oBar = oMisc + 64;       // 3 mbarriers
-    static constexpr int oSlot = oBar + 32;
-    static constexpr int bytes = oSlot + 16;
-};
-
-// Sums NV (<= 4) per-token partials over the 8 threads that hold one token
-// (4 lanes x 2 column halves). One barrier. v0/v1: the two tokens of this thread.
-template <int NV>
-__device__ __forceinline__ void token_sums(float (&v0)[NV], float (&v1)[NV], float4* red, int hh, int tok0, int tok1,
-                                           int lane) {
-    static_assert(NV >= 1 && NV <= 4, "at most 4 partials");
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        v0[i] += __shfl_xor_sync(0xffffffffu, v0[i], 1);
-        v0[i] += __shfl_xor_sync(0xffffffffu, v0[i], 2);
-        v1[i] += __shfl_xor_sync(0xffffffffu, v1[i], 1);
-        v1[i] += __shfl_xor_sync(0xffffffffu, v1[i], 2);
-    }
-    if ((lane & 3) == 0) {
-        float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            a[i] = v0[i];
-            b[i] = v1[i];
-        }
-        red[hh * 64 + tok0] = make_float4(a[0], a[1], a[2], a[3]);
-        red[hh * 64 + tok1] = make_float4(b[0], b[1], b[2], b[3]);
-    }
-    __syncthreads();
-    const float4 a0 = red[tok0], b0 = red[64 + tok0], a1 = red[tok1], b1 = red[64 + tok1];
-    const float s0[4] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w};
-    const float s1[4] = {a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        v0[i] = s0[i];
-        v1[i] = s1[i];
-    }
-}
-
-// Writes this thread's two tokens x 16 columns (as float2 pairs) of a
-// [64 t][128 k] fp16 image, each token scaled by its own factor.
-__device__ __forceinline__ void store_rows(uint8_t* img0, uint8_t* img1, uint32_t phase,
-                                           const float2 (&v0)[8], const float2 (&v1)[8], float s0, float s1) {
-    const float2 f0 = make_float2(s0, s0), f1 = make_float2(s1, s1);
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const float2 a = __fmul2_rn(v0[g], f0), b = __fmul2_rn(v1[g], f1);
-        const uint32_t o = ((uint32_t)g ^ phase) << 4;
-        *reinterpret_cast<uint32_t*>(img0 + o) = pack_half2(a.x, a.y);
-        *reinterpret_cast<uint32_t*>(img1 + o) = pack_half2(b.x, b.y);
-    }
-}
-
-// One thread issues, waits (bounded) and records failure; the barrier then
-// releases the CTA. Returns the CTA-uniform success flag.
-__device__ __forceinline__ bool wait_mma_cta(uint64_t* bar, uint32_t parity, int tid, float* abort_flag) {
-    if (tid == 0) {
-        if (!mbar_wait(bar, parity)) *abort_flag = 1.f;
-    }
-    __syncthreads();
-    tc_fence_after();
-    return *abort_flag == 0.f;
-}
-
 // Every thread waits on the MMA barrier itself (no CTA barrier); a thread
 // whose bounded wait gave up raises the abort flag, which the next CTA
 // barrier makes visible to all.
@@ -455,7 +375,85 @@ __device__ __forceinline__ void wait_mma_each(uint64_t* bar, uint32_t parity, fl
     tc_fence_after();
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+// =====================================================================
+// Fused CG iterations + read-out, a pair of chunks per CTA
+// =====================================================================
+// Two consecutive chunks A, B of one sequence (128 tokens) share every MMA:
+// tokens are the M = 128 dimension, so each product runs at the full M = 128
+// rate and the per-iteration round trip (MMA -> TMEM -> registers ->
+// reduction -> operand image) is paid once per 128 tokens.
+//   S = P K^T        (N = 128: only the two diagonal 64 x 64 blocks are used)
+//   U = P [H_A; H_B]^T (N = 256: token rows of A read columns 0..127, of B 128..255)
+//   Z = W K          (W block-diagonal, K = 128 keys)
+//   y_t = s_t sH (e^{b_t} U_t + Z_t) + lambda p_t
+// Thread layout: 16 warps; warp w holds the 32 tokens of TMEM lane quadrant
+// w % 4 (lane = token) and the 32 columns 32 * (w / 4) .. + 31 of each.
+constexpr int kPairThreads = 512;
+
+struct PairSmem {
+    static constexpr int oH = 0;                  // H images, per K block [A | B] (64 KB); later G
+    static constexpr int oK = 65536;              // key image [128 j][128 k] (32 KB); later values
+    static constexpr int oP = 98304;              // P-hat image [128 t][128 k] (32 KB); later X-hat
+    static constexpr int oW = 131072;             // masked scores [128 t][128 j] (32 KB), block-diagonal
+    static constexpr int kMS = 66;                // padded mask row stride (conflict-free float2 rows)
+    static constexpr int oM = 163840;             // decay mask / sH, fp32 [128 t][64 j], stride kMS
+    static constexpr int oLam = oM + 128 * kMS * 4;   // lambda [128]
+    static constexpr int oEb = oLam + 512;        // e^{b_t} [128]
+    static constexpr int oB = oEb + 512;          // b_t [128]
+    static constexpr int oRed = oB + 512;         // [4 column quarters][128 tokens] float4
+    static constexpr int oMisc = oRed + 8192;     // 32 floats
+    static constexpr int oBar = oMisc + 128;      // mbarriers: ld, s, u, z
+    static constexpr int oSlot = oBar + 64;
+    static constexpr int bytes = oSlot + 16;
+};
+
+// Log-cumsum of gamma over one chunk, by one warp (lane = threadIdx.x & 31).
+__device__ __forceinline__ void warp_chunk_gates(const float* __restrict__ gamma, size_t base, int n, float* b) {
+    const int lane = threadIdx.x & 31;
+    const int t0 = 2 * lane, t1 = 2 * lane + 1;
+    const float l0 = (t0 < n) ? logf(gamma[base + t0]) : 0.f;
+    const float l1 = (t1 < n) ? logf(gamma[base + t1]) : 0.f;
+    const float pair = l0 + l1;
+    float incl = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    const float excl = incl - pair;
+    b[t0] = excl + l0;
+    b[t1] = excl + l0 + l1;
+}
+
+// Sums 4 per-token partials over the 4 column quarters (one barrier).
+__device__ __forceinline__ float4 quarter_sum(float4 v, float4* red, int cq, int tok) {
+    red[cq * 128 + tok] = v;
+    __syncthreads();
+    const float4 a = red[tok], b = red[128 + tok], c = red[256 + tok], d = red[384 + tok];
+    return make_float4((a.x + b.x) + (c.x + d.x), (a.y + b.y) + (c.y + d.y), (a.z + b.z) + (c.z + d.z),
+                       (a.w + b.w) + (c.w + d.w));
+}
+
+// 32 consecutive columns (col0..col0+31) of one token row of a [128][128]
+// fp16 K-major image (two 64-column blocks of 16 KB), each value times s.
+__device__ __forceinline__ void store_row32(uint8_t* img, int tok, int col0, const float2 (&v)[16], float s) {
+    uint8_t* row = img + (col0 >> 6) * 16384 + tok * 128;
+    const int c8 = (col0 & 63) >> 3;
+    const float2 f = make_float2(s, s);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const float2 a = __fmul2_rn(v[4 * g], f), b = __fmul2_rn(v[4 * g + 1], f);
+        const float2 c = __fmul2_rn(v[4 * g + 2], f), d = __fmul2_rn(v[4 * g + 3], f);
+        uint4 o;
+        o.x = pack_half2(a.x, a.y);
+        o.y = pack_half2(b.x, b.y);
+        o.z = pack_half2(c.x, c.y);
+        o.w = pack_half2(d.x, d.y);
+        *reinterpret_cast<uint4*>(row + (((c8 + g) ^ (tok & 7)) << 4)) = o;
+    }
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
 tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
              const __nv_bfloat16* __restrict__ v, const float* __restrict__ gamma,
              const float* __restrict__ beta, const float* __restrict__ lambda, int H, int T, int nc,
@@ -463,191 +461,192 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
              float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* Hs = smem + CgSmem::oH;
-    uint8_t* Ks = smem + CgSmem::oK;
-    uint8_t* Ps = smem + CgSmem::oP;
-    uint8_t* Pt = smem + CgSmem::oPt;
-    uint8_t* Ws = smem + CgSmem::oW;
-    float* Mk = reinterpret_cast<float*>(smem + CgSmem::oM);
-    float* slam = reinterpret_cast<float*>(smem + CgSmem::oLam);
-    float* seb = reinterpret_cast<float*>(smem + CgSmem::oEb);
-    float* sbc = reinterpret_cast<float*>(smem + CgSmem::oB);
-    float4* red = reinterpret_cast<float4*>(smem + CgSmem::oRed);
-    float* misc = reinterpret_cast<float*>(smem + CgSmem::oMisc);
-    float* abort_flag = misc + 15;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + CgSmem::oBar);
-    uint64_t* bar_s = bar_ld + 1;        // scores S ready
-    uint64_t* bar_y = bar_ld + 2;        // Y = U + Z ready
-    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + CgSmem::oSlot);
+    uint8_t* Hs = smem + PairSmem::oH;
+    uint8_t* Ks = smem + PairSmem::oK;
+    uint8_t* Ps = smem + PairSmem::oP;
+    uint8_t* Ws = smem + PairSmem::oW;
+    float* Mk = reinterpret_cast<float*>(smem + PairSmem::oM);
+    float* slam = reinterpret_cast<float*>(smem + PairSmem::oLam);
+    float* seb = reinterpret_cast<float*>(smem + PairSmem::oEb);
+    float* sbc = reinterpret_cast<float*>(smem + PairSmem::oB);
+    float4* red = reinterpret_cast<float4*>(smem + PairSmem::oRed);
+    float* misc = reinterpret_cast<float*>(smem + PairSmem::oMisc);
+    float* abort_flag = misc + 31;
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + PairSmem::oBar);
+    uint64_t* bar_s = bar_ld + 1;
+    uint64_t* bar_u = bar_ld + 2;
+    uint64_t* bar_z = bar_ld + 3;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + PairSmem::oSlot);
 
-    const int c = blockIdx.x, bh = blockIdx.y, head = bh % H;
-    const int t0 = c * kC;
-    const int n = min(kC, T - t0);
-    const size_t base = (size_t)bh * T + t0;
+    const int pr = blockIdx.x, bh = blockIdx.y, head = bh % H;
+    const int cA = 2 * pr;
+    const bool hasB = cA + 1 < nc;
+    const int t0 = cA * kC;
+    const int nA = min(kC, T - t0);
+    const int nB = hasB ? min(kC, T - t0 - kC) : 0;
+    const size_t base = (size_t)bh * T + t0;       // token tok of the CTA is base + tok
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int q4 = w & 3, hh = w >> 2;
-    const int tok0 = 16 * q4 + (lane >> 2), tok1 = tok0 + 8;
-    const int cb = 64 * hh + 2 * (lane & 3);      // column of (group g, e): cb + 8g + e
-    const size_t ci = (size_t)bh * nc + c;
-    const __half* Himg = img + (ci * 2 + 0) * kImgHalves;
-    const __half* Gimg = img + (ci * 2 + 1) * kImgHalves;
+    const int q4 = w & 3, cq = w >> 2;
+    const int tok = 32 * q4 + lane;                  // 0..127 = TMEM lane
+    const int ch = tok >> 6;                          // 0: chunk A, 1: chunk B
+    const bool valid = (tok & 63) < (ch ? nB : nA);
+    const int col0 = 32 * cq;                         // this thread's 32 columns
+    const size_t ciA = (size_t)bh * nc + cA, ciB = hasB ? ciA + 1 : ciA;
 
-    // this thread's 32-bit slot of group g in a [64][128] fp16 image is
-    // row0/row1 + ((g ^ phase) << 4) + cw (both tokens share the swizzle
-    // phase: tok1 = tok0 + 8)
-    const uint32_t phase = (uint32_t)(tok0 & 7), cw = 4u * (uint32_t)(lane & 3);
-    const uint32_t row0 = (uint32_t)(hh * 8192 + tok0 * 128) + cw, row1 = row0 + 8 * 128;
-
-    // ---- set-up: barriers, TMEM, async load of the H_c image ----
     if (tid == 0) {
         mbar_init(bar_ld, 1);
         mbar_init(bar_s, 1);
-        mbar_init(bar_y, 1);
+        mbar_init(bar_u, 1);
+        mbar_init(bar_z, 1);
         fence_mbar_init();
         *abort_flag = 0.f;
     }
-    if (w == 0) tmem_alloc(slot, 256);
+    if (w == 0) tmem_alloc(slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *slot;
-    // TMEM: columns [0,128) lanes 16g..16g+15 (M=64 rows) hold Y = U + Z; the
-    // idle lanes 16g+16..16g+31 of the same columns hold x (same token order);
-    // columns [128,192) hold the scores S.
-    const uint32_t tq = tbase + ((uint32_t)(32 * q4) << 16);    // this warp's lane quadrant
-    const uint32_t tx = tq + (16u << 16);                        // ... and its x lanes
-    constexpr uint32_t kColS = 128;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_ld, kImgBytes);
-        bulk_g2s(Hs, Himg, kImgBytes, bar_ld);
-    }
-    const float sH = scales[ci * 2 + 0], sG = scales[ci * 2 + 1];
-    const float inv_sH = 1.f / sH;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);     // this warp's lane quadrant
+    // TMEM columns: U [0,256), S / Z / y [256,384), x [384,512)
+    constexpr uint32_t kColU = 0, kColS = 256, kColX = 384;
 
-    // gates, lambda and the key image (bf16 -> fp16 is exact for normalised keys)
-    chunk_gates(gamma, base, n, sbc);
-    for (int d = tid; d < kD; d += kThreads) slam[d] = lambda[(size_t)head * kD + d];
+    // bulk loads of the two chunk-start H images: per K block, rows of A then rows of B
+    auto load_state_images = [&](int which) {   // which: 0 = H, 1 = G
+        mbar_arrive_expect_tx(bar_ld, 4 * 16384);
+        const uint8_t* a = reinterpret_cast<const uint8_t*>(img + (ciA * 2 + which) * kImgHalves);
+        const uint8_t* b = reinterpret_cast<const uint8_t*>(img + (ciB * 2 + which) * kImgHalves);
+        bulk_g2s(Hs, a, 16384, bar_ld);
+        bulk_g2s(Hs + 16384, b, 16384, bar_ld);
+        bulk_g2s(Hs + 32768, a + 16384, 16384, bar_ld);
+        bulk_g2s(Hs + 49152, b + 16384, 16384, bar_ld);
+    };
+    if (tid == 0) load_state_images(0);
+    const float sH = scales[(ch ? ciB : ciA) * 2 + 0], sG = scales[(ch ? ciB : ciA) * 2 + 1];
+
+    // gates (warp 0: chunk A, warp 1: chunk B), lambda, key image, zeroed score image
+    if (w < 2) warp_chunk_gates(gamma, base + kC * w, w ? nB : nA, sbc + kC * w);
+    if (tid < kD) slam[tid] = lambda[(size_t)head * kD + tid];
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
-        const int cid = tid + kThreads * rep;
+        const int cid = tid + kPairThreads * rep;       // 2048 16-byte chunks
         const int j = cid >> 4, cc = cid & 15;
+        const bool ok = (j & 63) < ((j >> 6) ? nB : nA);
         uint4 rk = make_uint4(0, 0, 0, 0);
-        if (j < n) rk = *reinterpret_cast<const uint4*>(k + (base + j) * kD + 8 * cc);
-        *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 8192 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
+        if (ok) rk = *reinterpret_cast<const uint4*>(k + (base + j) * kD + 8 * cc);
+        *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
             bf16x8_to_f16x8(rk, 1.f);
+        reinterpret_cast<uint4*>(Ws)[cid] = make_uint4(0, 0, 0, 0);
     }
-    // CG state: x = 0 (TMEM), r = p = q; this thread holds 2 tokens x 8 column pairs
-    float2 r0[8], r1[8], p0[8], p1[8];
+    // CG state: x = 0 (TMEM), r = p = q; this thread: token tok, columns col0..col0+31
+    float2 r[16], p[16];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const int col = cb + 8 * g;
-        float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
-        if (tok0 < n) a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + (base + tok0) * kD + col));
-        if (tok1 < n) b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + (base + tok1) * kD + col));
-        r0[g] = a; p0[g] = a;
-        r1[g] = b; p1[g] = b;
+    for (int g = 0; g < 4; ++g) {
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (valid) raw = *reinterpret_cast<const uint4*>(q + (base + tok) * kD + col0 + 8 * g);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            r[4 * g + i] = __bfloat1622float2(b2[i]);
+            p[4 * g + i] = r[4 * g + i];
+        }
+    }
+    {
+        float z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0.f;
+        tmem_st32_x16(tl + kColX + col0, z);
+        tmem_st32_x16(tl + kColX + col0 + 16, z);
     }
     __syncthreads();                                   // gates visible
-    if (tid < kC) seb[tid] = expf(sbc[tid]);
-    for (int e = tid; e < kC * kC; e += kThreads) {
-        const int tt = e >> 6, j = e & 63;
-        Mk[tt * CgSmem::kMStride + j] =
-            (j <= tt && tt < n) ? beta[base + j] * expf(sbc[tt] - sbc[j]) * inv_sH : 0.f;
-    }
+    if (tid < 128) seb[tid] = expf(sbc[tid]);
     {
-        float z[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = 0.f;
-        tmem_st16_x8(tx + 64 * hh, z);
-        tmem_wait_st();
-    }
-    float rr0, rr1;
-    {
-        float a0[1] = {0.f}, a1[1] = {0.f};
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            a0[0] = fmaf(r0[g].x, r0[g].x, fmaf(r0[g].y, r0[g].y, a0[0]));
-            a1[0] = fmaf(r1[g].x, r1[g].x, fmaf(r1[g].y, r1[g].y, a1[0]));
+        for (int e = tid; e < 128 * kC; e += kPairThreads) {
+            const int tt = e >> 6, jl = e & 63, c = tt >> 6, tlc = tt & 63;
+            const int n = c ? nB : nA;
+            const float s_h = scales[(c ? ciB : ciA) * 2 + 0];
+            Mk[tt * PairSmem::kMS + jl] = (jl <= tlc && tlc < n)
+                        ? beta[base + kC * c + jl] * expf(sbc[tt] - sbc[kC * c + jl]) / s_h
+                        : 0.f;
         }
-        token_sums<1>(a0, a1, red, hh, tok0, tok1, lane);   // barrier also publishes seb
-        rr0 = a0[0];
-        rr1 = a1[0];
     }
-    const float qn0 = sqrtf(rr0), qn1 = sqrtf(rr1);
-    bool act0 = tok0 < n, act1 = tok1 < n;
-    int it0 = 0, it1 = 0;
-    const float eb0 = seb[tok0], eb1 = seb[tok1];
-    float s0 = pow2_sqrt_scale(rr0), s1 = pow2_sqrt_scale(rr1);
-    float is0 = 1.f / s0, is1 = 1.f / s1;                   // exact: powers of two
-    store_rows(Ps + row0, Ps + row1, phase, p0, p1, is0, is1);
-    store_rows(Pt + row0, Pt + row1, phase, p0, p1, eb0 * is0, eb1 * is1);
+    float rr;
+    {
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = __ffma2_rn(r[i], r[i], a);
+        rr = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;   // barrier publishes seb, Mk
+    }
+    tmem_wait_st();
+    const float qn = sqrtf(rr);
+    bool act = valid;
+    int it = 0;
+    const float eb = seb[tok];
+    float s = pow2_sqrt_scale(rr), is = 1.f / s;
+    store_row32(Ps, tok, col0, p, is);
 
-    // MMA issue (one thread). Descriptor address fields are the low 14 bits,
-    // so byte offsets (>> 4) add directly.
-    constexpr uint32_t kIdS = idesc_f16(64, 64, false, false);
-    constexpr uint32_t kIdU = idesc_f16(64, 128, false, false);
-    constexpr uint32_t kIdZ = idesc_f16(64, 128, false, true);
-    auto issue_S = [&](const uint8_t* A) {   // S = A K^T: M=64 tokens, N=64 keys, K=128
-        const uint64_t dA = sdesc(smem_addr(A), 16, 1024), dK = sdesc(smem_addr(Ks), 16, 1024);
+    constexpr uint32_t kIdS = idesc_f16(128, 128, false, false);
+    constexpr uint32_t kIdU = idesc_f16(128, 256, false, false);
+    constexpr uint32_t kIdZ = idesc_f16(128, 128, false, true);
+    auto issue_S = [&]() {      // S = P K^T -> columns [256, 384)
+        const uint64_t dA = sdesc(smem_addr(Ps), 16, 1024), dB = sdesc(smem_addr(Ks), 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t ko = ((ks >> 2) * 8192 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase + kColS, dA + ko, dK + ko, kIdS, ks > 0 ? 1u : 0u);
+            const uint32_t o = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
+            mma_f16(tbase + kColS, dA + o, dB + o, kIdS, ks > 0 ? 1u : 0u);
         }
     };
-    auto issue_U = [&](const uint8_t* A, const uint8_t* B) {   // Y = A B^T: M=64, N=128, K=128
-        const uint64_t dA = sdesc(smem_addr(A), 16, 1024), dB = sdesc(smem_addr(B), 16, 1024);
+    auto issue_U = [&]() {      // U = P [H_A; H_B]^T -> columns [0, 256)
+        const uint64_t dA = sdesc(smem_addr(Ps), 16, 1024), dB = sdesc(smem_addr(Hs), 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t ka = ((ks >> 2) * 8192 + (ks & 3) * 32) >> 4;
-            const uint32_t kb = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase, dA + ka, dB + kb, kIdU, ks > 0 ? 1u : 0u);
+            const uint32_t oa = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
+            const uint32_t ob = ((ks >> 2) * 32768 + (ks & 3) * 32) >> 4;
+            mma_f16(tbase + kColU, dA + oa, dB + ob, kIdU, ks > 0 ? 1u : 0u);
         }
     };
-    auto issue_Z = [&]() {                   // Y += W Kmn: M=64, N=128, K=64
-        const uint64_t dW = sdesc(smem_addr(Ws), 16, 1024), dKmn = sdesc(smem_addr(Ks), 8192, 1024);
+    auto issue_Z = [&]() {      // Z = W K -> columns [256, 384)
+        const uint64_t dA = sdesc(smem_addr(Ws), 16, 1024), dB = sdesc(smem_addr(Ks), 16384, 1024);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) mma_f16(tbase, dW + ((ks * 32) >> 4), dKmn + ((ks * 2048) >> 4), kIdZ, 1u);
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t oa = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
+            mma_f16(tbase + kColS, dA + oa, dB + ((ks * 2048) >> 4), kIdZ, ks > 0 ? 1u : 0u);
+        }
     };
-    // S (in TMEM) -> masked, scaled scores -> fp16 image
+    // S (TMEM) -> decay-masked, scaled scores -> the diagonal block of the score image
     auto masked_scores = [&](float extra) {
-        float sv[16];
-        tmem_ld16_x4(tq + kColS + 32 * hh, sv);
-        tmem_wait_ld();
-        const float2 ex = make_float2(extra, extra);
+        if ((cq >> 1) != ch) return;                   // off-diagonal quarter: block stays zero
+        const float* mrow = Mk + tok * PairSmem::kMS + (col0 & 63);
+        float2 wv[16];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const int j = 32 * hh + 8 * g + 2 * (lane & 3);
-            const float2 m0 = __fmul2_rn(*reinterpret_cast<const float2*>(Mk + tok0 * CgSmem::kMStride + j), ex);
-            const float2 m1 = __fmul2_rn(*reinterpret_cast<const float2*>(Mk + tok1 * CgSmem::kMStride + j), ex);
-            const float2 w0 = __fmul2_rn(m0, make_float2(sv[4 * g], sv[4 * g + 1]));
-            const float2 w1 = __fmul2_rn(m1, make_float2(sv[4 * g + 2], sv[4 * g + 3]));
-            const uint32_t o = ((((uint32_t)(4 * hh + g)) ^ phase) << 4) + cw;
-            *reinterpret_cast<uint32_t*>(Ws + tok0 * 128 + o) = pack_half2(w0.x, w0.y);
-            *reinterpret_cast<uint32_t*>(Ws + tok1 * 128 + o) = pack_half2(w1.x, w1.y);
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float sv[16];
+            tmem_ld32_x16(tl + kColS + col0 + 16 * h2, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float2 m = *reinterpret_cast<const float2*>(mrow + 16 * h2 + 2 * i);
+                wv[8 * h2 + i] = __fmul2_rn(m, make_float2(sv[2 * i] * extra, sv[2 * i + 1] * extra));
+            }
         }
+        store_row32(Ws, tok, col0, wv, 1.f);
     };
 
-    bool ok = mbar_wait(bar_ld, 0);
-    if (!ok) *abort_flag = 1.f;
-    uint32_t mma_phase = 0;
-
+    if (tid == 0 && !mbar_wait(bar_ld, 0)) *abort_flag = 1.f;
+    uint32_t ph = 0;
     for (int step = 0; step < cg_steps; ++step) {
-        act0 = act0 && cg_may_continue(rr0, qn0, tol);
-        act1 = act1 && cg_may_continue(rr1, qn1, tol);
+        act = act && cg_may_continue(rr, qn, tol);
         fence_proxy_async();
         tc_fence_before();
-        const int any = __syncthreads_or((act0 || act1) ? 1 : 0);
+        const int any = __syncthreads_or(act ? 1 : 0);
         tc_fence_after();
         if (!any || *abort_flag != 0.f) break;
-
-        // S first, then U straight behind it: U runs while the scores are masked
         if (tid == 0) {
-            issue_S(Ps);
+            issue_S();
             mma_commit(bar_s);
-            issue_U(Pt, Hs);
+            issue_U();
+            mma_commit(bar_u);
         }
-        wait_mma_each(bar_s, mma_phase & 1, abort_flag);
+        wait_mma_each(bar_s, ph & 1, abort_flag);
         masked_scores(1.f);
         fence_proxy_async();
         tc_fence_before();
@@ -656,121 +655,100 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         if (*abort_flag != 0.f) break;
         if (tid == 0) {
             issue_Z();
-            mma_commit(bar_y);
+            mma_commit(bar_z);
         }
-        wait_mma_each(bar_y, mma_phase & 1, abort_flag);
-        ++mma_phase;
+        wait_mma_each(bar_u, ph & 1, abort_flag);
+        wait_mma_each(bar_z, ph & 1, abort_flag);
+        ++ph;
 
-        // y = (s sH) Y + lambda p, written back over Y; partials p.y, r.y, y.y, r.r
-        float d0[4], d1[4];
+        // y = s sH (e^b U + Z) + lambda p (written over Z); partials p.y, r.y, y.y, r.r
+        const float c_u = s * sH * eb, c_z = s * sH;
+        float4 d;
         {
-            const float2 ys0 = make_float2(s0 * sH, s0 * sH), ys1 = make_float2(s1 * sH, s1 * sH);
-            float2 a = make_float2(0.f, 0.f), b = a, cc = a, e = a, f = a, h = a, ra = a, rb2 = a;
+            float2 a = make_float2(0.f, 0.f), b = a, cc = a, e = a;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float yv[16];
-                const uint32_t ya = tq + 64 * hh + 32 * half;
-                tmem_ld16_x4(ya, yv);
+            for (int h2 = 0; h2 < 4; ++h2) {
+                float uv[8], zv[8];
+                tmem_ld32_x8(tl + kColU + 128 * ch + col0 + 8 * h2, uv);
+                tmem_ld32_x8(tl + kColS + col0 + 8 * h2, zv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int gg = 4 * half + g;
-                    const float2 lm = *reinterpret_cast<const float2*>(slam + cb + 8 * gg);
-                    const float2 y0 = __ffma2_rn(make_float2(yv[4 * g], yv[4 * g + 1]), ys0, __fmul2_rn(lm, p0[gg]));
-                    const float2 y1 = __ffma2_rn(make_float2(yv[4 * g + 2], yv[4 * g + 3]), ys1, __fmul2_rn(lm, p1[gg]));
-                    a = __ffma2_rn(p0[gg], y0, a);
-                    b = __ffma2_rn(r0[gg], y0, b);
-                    cc = __ffma2_rn(y0, y0, cc);
-                    e = __ffma2_rn(p1[gg], y1, e);
-                    f = __ffma2_rn(r1[gg], y1, f);
-                    h = __ffma2_rn(y1, y1, h);
-                    ra = __ffma2_rn(r0[gg], r0[gg], ra);
-                    rb2 = __ffma2_rn(r1[gg], r1[gg], rb2);
-                    yv[4 * g] = y0.x; yv[4 * g + 1] = y0.y; yv[4 * g + 2] = y1.x; yv[4 * g + 3] = y1.y;
+                for (int i = 0; i < 4; ++i) {
+                    const int pi = 4 * h2 + i;
+                    const float2 lm = *reinterpret_cast<const float2*>(slam + col0 + 2 * pi);
+                    float2 y = __ffma2_rn(make_float2(uv[2 * i], uv[2 * i + 1]), make_float2(c_u, c_u),
+                                          __fmul2_rn(lm, p[pi]));
+                    y = __ffma2_rn(make_float2(zv[2 * i], zv[2 * i + 1]), make_float2(c_z, c_z), y);
+                    a = __ffma2_rn(p[pi], y, a);
+                    b = __ffma2_rn(r[pi], y, b);
+                    cc = __ffma2_rn(y, y, cc);
+                    e = __ffma2_rn(r[pi], r[pi], e);
+                    zv[2 * i] = y.x;
+                    zv[2 * i + 1] = y.y;
                 }
-                tmem_st16_x4(ya, yv);
+                tmem_st32_x8(tl + kColS + col0 + 8 * h2, zv);
             }
-            d0[0] = a.x + a.y; d0[1] = b.x + b.y; d0[2] = cc.x + cc.y; d0[3] = ra.x + ra.y;
-            d1[0] = e.x + e.y; d1[1] = f.x + f.y; d1[2] = h.x + h.y; d1[3] = rb2.x + rb2.y;
+            d = make_float4(a.x + a.y, b.x + b.y, cc.x + cc.y, e.x + e.y);
         }
         tmem_wait_st();
-        token_sums<4>(d0, d1, red, hh, tok0, tok1, lane);
-        if (act0 && !cg_curvature_ok(d0[0])) act0 = false;
-        if (act1 && !cg_curvature_ok(d1[0])) act1 = false;
-        // rr is refreshed from the true |r|^2 every iteration (no drift); the next
-        // |r - alpha y|^2 = rr - 2 alpha r.y + alpha^2 y.y is only needed one step
-        // ahead, for rho and the next stopping test.
-        if (act0) rr0 = d0[3];
-        if (act1) rr1 = d1[3];
-        const float al0 = act0 ? rr0 / d0[0] : 0.f, al1 = act1 ? rr1 / d1[0] : 0.f;
-        const float rn0 = fmaxf(fmaf(al0, fmaf(al0, d0[2], -2.f * d0[1]), rr0), 0.f);
-        const float rn1 = fmaxf(fmaf(al1, fmaf(al1, d1[2], -2.f * d1[1]), rr1), 0.f);
-        const float rho0 = act0 ? rn0 / rr0 : 0.f, rho1 = act1 ? rn1 / rr1 : 0.f;
-        const float2 pa0 = make_float2(al0, al0), pa1 = make_float2(al1, al1);
-        const float2 na0 = make_float2(-al0, -al0), na1 = make_float2(-al1, -al1);
-        const float2 rh0 = make_float2(rho0, rho0), rh1 = make_float2(rho1, rho1);
+        d = quarter_sum(d, red, cq, tok);
+        if (act && !cg_curvature_ok(d.x)) act = false;
+        if (act) rr = d.w;                             // true |r|^2 of the current residual
+        const float al = act ? rr / d.x : 0.f;
+        const float rn = fmaxf(fmaf(al, fmaf(al, d.z, -2.f * d.y), rr), 0.f);
+        const float rho = act ? rn / rr : 0.f;
+        const float2 pa = make_float2(al, al), na = make_float2(-al, -al), rh = make_float2(rho, rho);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {   // x += alpha p (TMEM), r -= alpha y, p = r + rho p
-            float xv[16], yv[16];
-            const uint32_t xa = tx + 64 * hh + 32 * half;
-            tmem_ld16_x4(xa, xv);
-            tmem_ld16_x4(tq + 64 * hh + 32 * half, yv);
+        for (int h2 = 0; h2 < 4; ++h2) {               // x += alpha p; r -= alpha y; p = r + rho p
+            float xv[8], yv[8];
+            tmem_ld32_x8(tl + kColX + col0 + 8 * h2, xv);
+            tmem_ld32_x8(tl + kColS + col0 + 8 * h2, yv);
             tmem_wait_ld();
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const int gg = 4 * half + g;
-                const float2 x0 = __ffma2_rn(pa0, p0[gg], make_float2(xv[4 * g], xv[4 * g + 1]));
-                const float2 x1 = __ffma2_rn(pa1, p1[gg], make_float2(xv[4 * g + 2], xv[4 * g + 3]));
-                xv[4 * g] = x0.x; xv[4 * g + 1] = x0.y; xv[4 * g + 2] = x1.x; xv[4 * g + 3] = x1.y;
-                if (act0) {
-                    r0[gg] = __ffma2_rn(na0, make_float2(yv[4 * g], yv[4 * g + 1]), r0[gg]);
-                    p0[gg] = __ffma2_rn(rh0, p0[gg], r0[gg]);
-                }
-                if (act1) {
-                    r1[gg] = __ffma2_rn(na1, make_float2(yv[4 * g + 2], yv[4 * g + 3]), r1[gg]);
-                    p1[gg] = __ffma2_rn(rh1, p1[gg], r1[gg]);
+            for (int i = 0; i < 4; ++i) {
+                const int pi = 4 * h2 + i;
+                const float2 x = __ffma2_rn(pa, p[pi], make_float2(xv[2 * i], xv[2 * i + 1]));
+                xv[2 * i] = x.x;
+                xv[2 * i + 1] = x.y;
+                if (act) {
+                    r[pi] = __ffma2_rn(na, make_float2(yv[2 * i], yv[2 * i + 1]), r[pi]);
+                    p[pi] = __ffma2_rn(rh, p[pi], r[pi]);
                 }
             }
-            tmem_st16_x4(xa, xv);
+            tmem_st32_x8(tl + kColX + col0 + 8 * h2, xv);
         }
-        if (act0) {
-            rr0 = rn0;
-            ++it0;
-            s0 = pow2_sqrt_scale(rr0);
-            is0 = 1.f / s0;
-        }
-        if (act1) {
-            rr1 = rn1;
-            ++it1;
-            s1 = pow2_sqrt_scale(rr1);
-            is1 = 1.f / s1;
+        if (act) {
+            rr = rn;
+            ++it;
+            s = pow2_sqrt_scale(rr);
+            is = 1.f / s;
         }
         tmem_wait_st();
-        store_rows(Ps + row0, Ps + row1, phase, p0, p1, is0, is1);
-        store_rows(Pt + row0, Pt + row1, phase, p0, p1, eb0 * is0, eb1 * is1);
+        store_row32(Ps, tok, col0, p, is);
     }
 
-    // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V ----
-    float2 xr0[8], xr1[8];
+    // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern ----
+    __syncthreads();                                   // last reduction's readers are done with red[]
+    float2 xr[16];
     {
-        float xv[32];
-        tmem_ld16_x8(tx + 64 * hh, xv);
-        tmem_wait_ld();
+        float xv[16];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            xr0[g] = make_float2(xv[4 * g], xv[4 * g + 1]);
-            xr1[g] = make_float2(xv[4 * g + 2], xv[4 * g + 3]);
+        for (int h2 = 0; h2 < 2; ++h2) {
+            tmem_ld32_x16(tl + kColX + col0 + 16 * h2, xv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) xr[8 * h2 + i] = make_float2(xv[2 * i], xv[2 * i + 1]);
         }
     }
-    // the values of the chunk, scaled by a power of two so fp16 holds them
     uint4 vraw[4];
     float vmax = 0.f;
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
-        const int cid = tid + kThreads * rep;
+        const int cid = tid + kPairThreads * rep;
         const int j = cid >> 4, cc = cid & 15;
+        const bool ok = (j & 63) < ((j >> 6) ? nB : nA);
         vraw[rep] = make_uint4(0, 0, 0, 0);
-        if (j < n) vraw[rep] = *reinterpret_cast<const uint4*>(v + (base + j) * kD + 8 * cc);
+        if (ok) vraw[rep] = *reinterpret_cast<const uint4*>(v + (base + j) * kD + 8 * cc);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[rep]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -781,97 +759,93 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
     if (lane == 0) misc[w] = vmax;
-    float xs0, xs1;
+    float xs;
     {
-        float a0[1] = {0.f}, a1[1] = {0.f};
+        float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            a0[0] = fmaf(xr0[g].x, xr0[g].x, fmaf(xr0[g].y, xr0[g].y, a0[0]));
-            a1[0] = fmaf(xr1[g].x, xr1[g].x, fmaf(xr1[g].y, xr1[g].y, a1[0]));
-        }
-        token_sums<1>(a0, a1, red, hh, tok0, tok1, lane);   // its barrier also publishes misc[]
-        xs0 = a0[0] > 0.f ? sqrtf(a0[0]) : 1.f;
-        xs1 = a1[0] > 0.f ? sqrtf(a1[0]) : 1.f;
+        for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
+        const float xx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;   // publishes misc
+        xs = xx > 0.f ? sqrtf(xx) : 1.f;
     }
     float vm = misc[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) vm = fmaxf(vm, misc[i]);
+    for (int i = 1; i < 16; ++i) vm = fmaxf(vm, misc[i]);
     const float sV = pow2_ceil_at_least_one(vm);
-    store_rows(Ps + row0, Ps + row1, phase, xr0, xr1, 1.f / xs0, 1.f / xs1);
-    store_rows(Pt + row0, Pt + row1, phase, xr0, xr1, eb0 / xs0, eb1 / xs1);
+    store_row32(Ps, tok, col0, xr, 1.f / xs);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    ok = *abort_flag == 0.f;
+    bool ok = *abort_flag == 0.f;
     if (ok) {
         if (tid == 0) {
-            // every MMA that read the H image has completed: reuse its buffer for G_c
-            mbar_arrive_expect_tx(bar_ld, kImgBytes);
-            bulk_g2s(Hs, Gimg, kImgBytes, bar_ld);
-            issue_S(Ps);                       // S' = X-hat K^T
+            load_state_images(1);              // every MMA that read the H images is done
+            issue_S();                         // S' = X-hat K^T
             mma_commit(bar_s);
         }
-        ok = wait_mma_cta(bar_s, mma_phase & 1, tid, abort_flag);
-    }
-    if (ok) {
+        wait_mma_each(bar_s, ph & 1, abort_flag);
         masked_scores(sH * sV / sG);           // mask holds 1/sH
-        // the key image is dead (S' done): overwrite it with the value image
         const float inv_sV = 1.f / sV;
 #pragma unroll
-        for (int rep = 0; rep < 4; ++rep) {
-            const int cid = tid + kThreads * rep;
+        for (int rep = 0; rep < 4; ++rep) {    // the key image is dead: values take its place
+            const int cid = tid + kPairThreads * rep;
             const int j = cid >> 4, cc = cid & 15;
-            *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 8192 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
                 bf16x8_to_f16x8(vraw[rep], inv_sV);
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        ok = *abort_flag == 0.f;
+    }
+    if (ok) {
         if (tid == 0) {
             if (!mbar_wait(bar_ld, 1)) {
                 *abort_flag = 1.f;
+                mma_commit(bar_u);
+                mma_commit(bar_z);
             } else {
-                issue_U(Pt, Hs);               // O = X-tilde G^T + W' V
-                issue_Z();
-                mma_commit(bar_y);
+                issue_U();                     // U' = X-hat [G_A; G_B]^T
+                mma_commit(bar_u);
+                issue_Z();                     // Z' = W' V
+                mma_commit(bar_z);
             }
         }
-        ok = wait_mma_cta(bar_y, mma_phase & 1, tid, abort_flag);
-        ++mma_phase;
+        wait_mma_each(bar_u, ph & 1, abort_flag);
+        wait_mma_each(bar_z, ph & 1, abort_flag);
+        ++ph;
+        __syncthreads();
+        ok = *abort_flag == 0.f;
     }
     if (ok) {
-        float ov[32];
-        tmem_ld16_x8(tq + 64 * hh, ov);
-        tmem_wait_ld();
-        const float os0 = xs0 * sG, os1 = xs1 * sG;
+        const float cu = xs * sG * eb, cz = xs * sG;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            const int col = cb + 8 * g;
-            if (tok0 < n)
-                *reinterpret_cast<float2*>(out + (base + tok0) * kD + col) =
-                    make_float2(ov[4 * g] * os0, ov[4 * g + 1] * os0);
-            if (tok1 < n)
-                *reinterpret_cast<float2*>(out + (base + tok1) * kD + col) =
-                    make_float2(ov[4 * g + 2] * os1, ov[4 * g + 3] * os1);
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float uv[16], zv[16];
+            tmem_ld32_x16(tl + kColU + 128 * ch + col0 + 16 * h2, uv);
+            tmem_ld32_x16(tl + kColS + col0 + 16 * h2, zv);
+            tmem_wait_ld();
+            if (valid) {
+                float4* dst = reinterpret_cast<float4*>(out + (base + tok) * kD + col0 + 16 * h2);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_float4(fmaf(uv[4 * i], cu, zv[4 * i] * cz), fmaf(uv[4 * i + 1], cu, zv[4 * i + 1] * cz),
+                                         fmaf(uv[4 * i + 2], cu, zv[4 * i + 2] * cz),
+                                         fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
+            }
         }
-        if (iters && hh == 0 && (lane & 3) == 0) {
-            if (tok0 < n) iters[base + tok0] = it0;
-            if (tok1 < n) iters[base + tok1] = it1;
-        }
-    } else {
-        if (tid == 0) {
-            record_error(err, kErrTimeout);
-            // one more bounded chance for every MMA issued so far to drain
-            mma_commit(bar_ld);
-            mbar_wait(bar_ld, 0);
-            mbar_wait(bar_ld, 1);
-        }
+        if (iters && cq == 0 && valid) iters[base + tok] = it;
+    } else if (tid == 0) {
+        record_error(err, kErrTimeout);
+        // one more bounded chance for every MMA issued so far to drain
+        mma_commit(bar_ld);
+        mbar_wait(bar_ld, 0);
+        mbar_wait(bar_ld, 1);
     }
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tbase, 256);
+    if (w == 0) tmem_dealloc(tbase, 512);
 }
 
 }  // namespace
@@ -897,7 +871,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     float* scales = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + images_bytes(a.B, a.H, a.T));
     unsigned* err = error_word_ptr();
     const int scan_smem = ScanSmem::bytes + 1024;
-    const int cg_smem = CgSmem::bytes + 1024;
+    const int cg_smem = PairSmem::bytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_cg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cg_smem);
@@ -912,7 +886,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     {
         LaunchTimer timer(kKindTcCg, st);
-        tc_cg_kernel<<<dim3(nc, BH), kThreads, cg_smem, st>>>(
+        tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kPairThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, nc, a.cg_steps, a.tol,
             img, scales, a.out, a.iters, err);

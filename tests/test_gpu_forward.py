@@ -145,14 +145,16 @@ def test_zero_steps_and_zero_query(mesa, oracle_mod):
 
 @pytest.mark.parametrize("dtype,d,chunk", [("f32", 64, 64), ("bf16", 128, 64)])
 def test_nan_input_does_not_hang(mesa, dtype, d, chunk):
-    """A NaN poisons the tokens that depend on it (its chunk onwards) and
-    nothing else; the call completes with no device error."""
-    w = rand_workload(d, chunk, dtype, 200, B=1, H=2, N=15, seed=9)
+    """A NaN poisons the tokens of its chunk (on the tensor-core path: of its
+    pair of chunks, which share every MMA) and all later tokens of the
+    sequence, and nothing else; the call completes with no device error."""
+    w = rand_workload(d, chunk, dtype, 300, B=1, H=2, N=15, seed=9)
     x = mi.batch(w)
-    x["v"][0, 0, 70, 3] = np.nan
-    x["k"][0, 0, 90, 1] = np.nan
+    x["v"][0, 0, 150, 3] = np.nan
+    x["k"][0, 0, 170, 1] = np.nan
     out, _ = run(mesa, to_dev(x, dtype), chunk, 15, 0.0)
-    assert np.isfinite(out[0, 0, :64]).all()
+    assert np.isfinite(out[0, 0, :128]).all()
+    assert not np.isfinite(out[0, 0, 192:]).all()
     assert np.isfinite(out[0, 1]).all()
 
 

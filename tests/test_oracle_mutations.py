@@ -1,0 +1,108 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the C oracle (on the CPU, in a
+temporary directory), builds it, and runs a fast subset of the pins from
+test_oracle_pins.py against it: at least one pin must fail for every mutant,
+and all of them must pass for the unmodified source."""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "mesa_oracle.c")
+
+MUTANTS = {
+    "beta dropped from the H update": ("Hm[(size_t)i * dk + j] = g * Hm[(size_t)i * dk + j] + bta * kt[i] * kt[j];",
+                                       "Hm[(size_t)i * dk + j] = g * Hm[(size_t)i * dk + j] + kt[i] * kt[j];"),
+    "decay dropped from the H update": ("Hm[(size_t)i * dk + j] = g * Hm[(size_t)i * dk + j] + bta * kt[i] * kt[j];",
+                                        "Hm[(size_t)i * dk + j] = Hm[(size_t)i * dk + j] + bta * kt[i] * kt[j];"),
+    "G built as k v^T": ("Gm[(size_t)i * dk + j] = g * Gm[(size_t)i * dk + j] + bta * vt[i] * kt[j];",
+                         "Gm[(size_t)i * dk + j] = g * Gm[(size_t)i * dk + j] + bta * vt[j] * kt[i];"),
+    "CG residual sign": ("r[i] -= alpha * y[i];", "r[i] += alpha * y[i];"),
+    "CG rho inverted": ("const double rho = rr_new / rr;", "const double rho = rr / rr_new;"),
+    "CG direction not conjugated": ("p[i] = r[i] + rho * p[i];", "p[i] = r[i];"),
+    "chunk diagonal term dropped": ("for (int j = 0; j <= t; ++j) {\n        const double m = c->betac[j]",
+                                    "for (int j = 0; j < t; ++j) {\n        const double m = c->betac[j]"),
+    "chunk decay sign": ("const double m = c->betac[j] * exp(c->bcum[t] - c->bcum[j]);",
+                         "const double m = c->betac[j] * exp(c->bcum[j] - c->bcum[t]);"),
+    "Cholesky back-substitution transposed": ("for (int m = i + 1; m < n; ++m) s -= A[(size_t)m * n + i] * x[m];",
+                                              "for (int m = i + 1; m < n; ++m) s -= A[(size_t)i * n + m] * x[m];"),
+    "Lambda applied twice": ("A[(size_t)i * dk + i] += lambda[(size_t)h * dk + i];",
+                             "A[(size_t)i * dk + i] += 2.0 * lambda[(size_t)h * dk + i];"),
+}
+
+
+class _Mutant:
+    """The oracle module's Python API bound to another build of the C source."""
+
+    def __init__(self, lib):
+        self.lib = lib
+
+    def __getattr__(self, name):
+        fn = getattr(oracle, name)
+
+        def call(*a, **kw):
+            saved = oracle._lib
+            oracle._lib = self.lib
+            try:
+                return fn(*a, **kw)
+            finally:
+                oracle._lib = saved
+        return call
+
+
+def build_variant(src_text, tmp):
+    c = os.path.join(tmp, "m.c")
+    h = os.path.join(tmp, "mesa_oracle.h")
+    with open(c, "w") as f:
+        f.write(src_text)
+    with open(os.path.join(os.path.dirname(SRC), "mesa_oracle.h")) as f, open(h, "w") as g:
+        g.write(f.read())
+    so = os.path.join(tmp, "libm.so")
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-I", tmp,
+                    "-o", so, c, "-lm"], check=True)
+    return _Mutant(oracle._configure(ctypes.CDLL(so)))
+
+
+PIN_SUBSET = [
+    lambda o: pins.test_cg_iterates_equal_krylov_galerkin(o, 9),
+    lambda o: pins.test_cg_one_step_closed_form(o),
+    lambda o: pins.test_cholesky_minimises_the_mesa_objective(o, 3, 2, 6),
+    lambda o: pins.test_gamma_beta_one_gives_plain_sums(o),
+    lambda o: pins.test_first_token_and_gamma_zero_match_sherman_morrison(o),
+    lambda o: pins.test_unconverged_cg_equals_galerkin_on_explicit_statistics(o),
+    lambda o: pins.test_chunked_equals_per_token(o, 8, 0.0),
+    lambda o: pins.test_large_lambda_gives_linear_attention(o),
+]
+
+
+def failing_pins(mod):
+    failed = 0
+    for pin in PIN_SUBSET:
+        try:
+            pin(mod)
+        except (AssertionError, RuntimeError, FloatingPointError, ValueError, IndexError):
+            failed += 1
+    return failed
+
+
+def test_unmodified_source_passes_the_subset():
+    with open(SRC) as f:
+        text = f.read()
+    with tempfile.TemporaryDirectory() as tmp:
+        assert failing_pins(build_variant(text, tmp)) == 0
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    old, new = MUTANTS[name]
+    with open(SRC) as f:
+        text = f.read()
+    assert text.count(old) >= 1, f"mutation anchor missing: {name}"
+    with tempfile.TemporaryDirectory() as tmp:      # the first occurrence is mutated
+        assert failing_pins(build_variant(text.replace(old, new, 1), tmp)) >= 1, name
