@@ -70,12 +70,14 @@ __device__ __forceinline__ float pow2_sqrt_scale(float rr) {
 
 // Inclusive log-cumsum of gamma over a 64-token chunk by warp 0 (padded
 // tokens count as gamma = 1).
-__device__ __forceinline__ void chunk_gates(const float* __restrict__ gamma, size_t base, int n, float* b) {
-    if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
+// b[t] for t < 64: in-chunk inclusive cumulative sum of log gamma over the
+// chunk's first n positions, held constant past n. One warp; g points at the
+// chunk's gamma (global or shared memory).
+__device__ __forceinline__ void warp_gate_cumsum(const float* g, int n, float* b) {
+    const int lane = threadIdx.x & 31;
     const int t0 = 2 * lane, t1 = 2 * lane + 1;
-    const float l0 = (t0 < n) ? logf(gamma[base + t0]) : 0.f;
-    const float l1 = (t1 < n) ? logf(gamma[base + t1]) : 0.f;
+    const float l0 = (t0 < n) ? logf(g[t0]) : 0.f;
+    const float l1 = (t1 < n) ? logf(g[t1]) : 0.f;
     const float pair = l0 + l1;
     float incl = pair;
 #pragma unroll
@@ -118,7 +120,8 @@ struct ScanSmem {
     static constexpr int oAlo = 81920;
     static constexpr int oB = 98304;              // MN-major [64 j][64 l] fp16, 8 KB
     static constexpr int oGate = 106496;          // b[64], w[64], amax[64], kmax[64]
-    static constexpr int oRed = oGate + 1024;     // 16 floats
+    static constexpr int oGraw = oGate + 1024;    // 2 x {gamma[64], beta[64]} prefetched with the rows
+    static constexpr int oRed = oGraw + 1024;     // 16 floats
     static constexpr int oBar = oRed + 64;        // raw[2], mma
     static constexpr int oSlot = oBar + 32;
     static constexpr int bytes = oSlot + 16;
@@ -142,6 +145,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     float* sw = sb + kC;
     float* amax = sw + kC;
     float* kmax = amax + kC;
+    float* graw = reinterpret_cast<float*>(smem + ScanSmem::oGraw);
     float* red = reinterpret_cast<float*>(smem + ScanSmem::oRed);
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(smem + ScanSmem::oBar);
     uint64_t* bar_mma = bar_raw + 2;
@@ -156,14 +160,22 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     const float* init = m ? G_in : H_in;
     float* fin = m ? G_out : H_out;
     const size_t seq = (size_t)bh * T;
+    // gamma/beta of a chunk travel with its rows when the chunk is full and its
+    // first element is 16-byte aligned (T % 4 == 0); otherwise warp 0 reads them.
+    const bool gates_bulk = (T % 4) == 0 && ((reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(beta)) & 15) == 0;
 
-    auto prefetch = [&](int cc) {                 // raw rows of chunk cc -> buffer cc & 1 (thread 0)
+    auto prefetch = [&](int cc) {                 // rows (and gates) of chunk cc -> buffer cc & 1 (thread 0)
         const int nn = min(kC, T - cc * kC);
         const uint32_t bytes = (uint32_t)nn * kD * 2;
         const int buf = cc & 1;
-        mbar_arrive_expect_tx(bar_raw + buf, m ? 2 * bytes : bytes);
+        const bool gb = gates_bulk && nn == kC;
+        mbar_arrive_expect_tx(bar_raw + buf, (m ? 2 * bytes : bytes) + (gb ? 512u : 0u));
         bulk_g2s(rawK + buf * 16384, k + (seq + (size_t)cc * kC) * kD, bytes, bar_raw + buf);
         if (m) bulk_g2s(rawA + buf * 16384, A + (seq + (size_t)cc * kC) * kD, bytes, bar_raw + buf);
+        if (gb) {
+            bulk_g2s(graw + buf * 128, gamma + seq + (size_t)cc * kC, 256, bar_raw + buf);
+            bulk_g2s(graw + buf * 128 + 64, beta + seq + (size_t)cc * kC, 256, bar_raw + buf);
+        }
     };
 
     if (tid == 0) {
@@ -217,11 +229,12 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     uint32_t mma_phase = 0;
     bool ok = true;
     for (int c = 0; c <= nc; ++c) {
-        // ---- emit the state before chunk c (fp16 image block + scale), or the final state ----
-        if (c < nc) {
+        // ---- emit the state before chunk c (fp16 image block + scale) when c starts a
+        //      128-token block of the solve, or the final state ----
+        if (c < nc && (c & 1) == 0) {
             const float s = pow2_ceil_at_least_one(bound);
             const float inv = 1.f / s;
-            const size_t ci = ((size_t)bh * nc + c) * 2 + m;
+            const size_t ci = ((size_t)bh * ((nc + 1) >> 1) + (c >> 1)) * 2 + m;
             if (tid == 0 && nb == 0) scales[ci] = s;
             uint8_t* dst = reinterpret_cast<uint8_t*>(img + ci * kImgHalves) + nb * 16384 + row * 128;
 #pragma unroll
@@ -233,7 +246,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
                 o.w = pack_half2(S[8 * g + 6] * inv, S[8 * g + 7] * inv);
                 *reinterpret_cast<uint4*>(dst + ((((lcol >> 3) + g) ^ (row & 7)) << 4)) = o;
             }
-        } else {
+        } else if (c == nc) {
             if (fin) {
                 float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
 #pragma unroll
@@ -248,15 +261,23 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         const size_t base = seq + t0;
         const int buf = c & 1;
         if (tid == 0 && !mbar_wait(bar_raw + buf, (c >> 1) & 1)) red[15] = 1.f;
-        chunk_gates(gamma, base, n, sb);
+        if (w == 0) {
+            __syncwarp();
+            const bool gb = gates_bulk && n == kC;
+            const float* gsrc = gb ? graw + buf * 128 : gamma + base;
+            const float* bsrc = gb ? graw + buf * 128 + 64 : beta + base;
+            warp_gate_cumsum(gsrc, n, sb);
+            __syncwarp();
+            const float bl = sb[kC - 1];                               // b at the chunk's last position
+            sw[lane] = (lane < n) ? bsrc[lane] * expf(bl - sb[lane]) : 0.f;
+            sw[lane + 32] = (lane + 32 < n) ? bsrc[lane + 32] * expf(bl - sb[lane + 32]) : 0.f;
+        }
         __syncthreads();
         if (red[15] != 0.f) {
             ok = false;
             break;
         }
         const float blast = sb[kC - 1];
-        if (tid < kC) sw[tid] = (tid < n) ? beta[base + tid] * expf(blast - sb[tid]) : 0.f;
-        __syncthreads();
 
         // ---- operand images: A = w_j a_j (hi/lo) [j][i], B = k_j block [j][l]; row maxima ----
         const uint8_t* ra = rawA + buf * 16384;
@@ -376,53 +397,63 @@ __device__ __forceinline__ void wait_mma_each(uint64_t* bar, uint32_t parity, fl
 }
 
 // =====================================================================
-// Fused CG iterations + read-out, a pair of chunks per CTA
+// Fused CG iterations + read-out, 128 tokens per CTA
 // =====================================================================
-// Two consecutive chunks A, B of one sequence (128 tokens) share every MMA:
-// tokens are the M = 128 dimension, so each product runs at the full M = 128
-// rate and the per-iteration round trip (MMA -> TMEM -> registers ->
-// reduction -> operand image) is paid once per 128 tokens.
-//   S = P K^T        (N = 128: only the two diagonal 64 x 64 blocks are used)
-//   U = P [H_A; H_B]^T (N = 256: token rows of A read columns 0..127, of B 128..255)
-//   Z = W K          (W block-diagonal, K = 128 keys)
-//   y_t = s_t sH (e^{b_t} U_t + Z_t) + lambda p_t
+// CTA blk takes tokens t0 .. t0+127 of one sequence (t0 = 128 blk, i.e. the
+// even chunk c = 2 blk and the chunk after it) and the state H_c before them.
+// With b_t the log-cumsum of gamma from t0 over all 128 tokens and
+// M_tj = beta_j e^{b_t-b_j} (t0 <= j <= t),
+//     H_t = e^{b_t} H_c + sum_j M_tj k_j k_j^T
+// for every token of the block. This is the chunkwise form of two 64-token
+// chunks with the second chunk's state H_{c+1} expanded into its definition,
+// so one chunk-start state serves 128 tokens and every product has M = N = 128:
+//   S = P K^T,  W = M o S (lower triangular),  U = P H_c^T,  Z = W K,
+//   y_t = s_t sH (e^{b_t} U_t + Z_t) + lambda p_t.
 // Thread layout: 16 warps; warp w holds the 32 tokens of TMEM lane quadrant
 // w % 4 (lane = token) and the 32 columns 32 * (w / 4) .. + 31 of each.
-constexpr int kPairThreads = 512;
+// TMEM columns: U [0,128), S / Z / y [128,256), x [256,384), r [384,512);
+// p stays in registers.
+constexpr int kBlk = 2 * kC;                      // tokens per CTA
+constexpr int kBlkThreads = 512;
 
-struct PairSmem {
-    static constexpr int oH = 0;                  // H images, per K block [A | B] (64 KB); later G
-    static constexpr int oK = 65536;              // key image [128 j][128 k] (32 KB); later values
-    static constexpr int oP = 98304;              // P-hat image [128 t][128 k] (32 KB); later X-hat
-    static constexpr int oW = 131072;             // masked scores [128 t][128 j] (32 KB), block-diagonal
-    static constexpr int kMS = 66;                // padded mask row stride (conflict-free float2 rows)
-    static constexpr int oM = 163840;             // decay mask / sH, fp32 [128 t][64 j], stride kMS
-    static constexpr int oLam = oM + 128 * kMS * 4;   // lambda [128]
+struct BlkSmem {
+    static constexpr int oH = 0;                  // state image [128 i][128 k] (32 KB); later G
+    static constexpr int oK = 32768;              // key image [128 j][128 k] (32 KB); later values
+    static constexpr int oP = 65536;              // P-hat image [128 t][128 k] (32 KB); later X-hat
+    static constexpr int oW = 98304;              // masked scores [128 t][128 j] (32 KB)
+    static constexpr int kMS = 130;               // mask row stride (conflict-free float2 rows)
+    static constexpr int oM = 131072;             // decay mask / sH, fp32 [128 t][128 j], stride kMS
+    static constexpr int oLam = oM + kBlk * kMS * 4;   // lambda [128]
     static constexpr int oEb = oLam + 512;        // e^{b_t} [128]
     static constexpr int oB = oEb + 512;          // b_t [128]
-    static constexpr int oRed = oB + 512;         // [4 column quarters][128 tokens] float4
+    static constexpr int oBeta = oB + 512;        // beta_j [128]
+    static constexpr int oRed = oBeta + 512;      // [4 column quarters][128 tokens] float4
     static constexpr int oMisc = oRed + 8192;     // 32 floats
     static constexpr int oBar = oMisc + 128;      // mbarriers: ld, s, u, z
     static constexpr int oSlot = oBar + 64;
     static constexpr int bytes = oSlot + 16;
 };
 
-// Log-cumsum of gamma over one chunk, by one warp (lane = threadIdx.x & 31).
-__device__ __forceinline__ void warp_chunk_gates(const float* __restrict__ gamma, size_t base, int n, float* b) {
+// b[t], t < 128: cumulative sum of log gamma over positions 0..t of the first
+// n positions, held constant past n. One warp, four positions per lane.
+__device__ __forceinline__ void warp_gate_cumsum128(const float* g, int n, float* b) {
     const int lane = threadIdx.x & 31;
-    const int t0 = 2 * lane, t1 = 2 * lane + 1;
-    const float l0 = (t0 < n) ? logf(gamma[base + t0]) : 0.f;
-    const float l1 = (t1 < n) ? logf(gamma[base + t1]) : 0.f;
-    const float pair = l0 + l1;
-    float incl = pair;
+    float l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) l[i] = (4 * lane + i < n) ? logf(g[4 * lane + i]) : 0.f;
+    const float quad = (l[0] + l[1]) + (l[2] + l[3]);
+    float incl = quad;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const float o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
     }
-    const float excl = incl - pair;
-    b[t0] = excl + l0;
-    b[t1] = excl + l0 + l1;
+    float acc = incl - quad;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc += l[i];
+        b[4 * lane + i] = acc;
+    }
 }
 
 // Sums 4 per-token partials over the 4 column quarters (one barrier).
@@ -453,45 +484,57 @@ __device__ __forceinline__ void store_row32(uint8_t* img, int tok, int col0, con
     }
 }
 
-__global__ void __launch_bounds__(kPairThreads, 1)
+// Eight K = 16 steps of one fp16 product into TMEM address d. A is a K-major
+// SW128 image (64-element K blocks a_kb bytes apart); B is K-major (b_k16 = 32)
+// or MN-major (b_lbo = MN block stride, b_k16 = 2048), its K blocks b_kb apart.
+// Kept out of line so that the descriptors live only in the issuing thread.
+__device__ __noinline__ void issue_k128(uint32_t d, uint32_t a, uint32_t b, uint32_t b_lbo, uint32_t a_kb,
+                                        uint32_t b_kb, uint32_t b_k16, uint32_t idesc) {
+    const uint64_t da = sdesc(a, 16, 1024), db = sdesc(b, b_lbo, 1024);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t oa = ((ks >> 2) * a_kb + (ks & 3) * 32) >> 4;
+        const uint32_t ob = ((ks >> 2) * b_kb + (ks & 3) * b_k16) >> 4;
+        mma_f16(d, da + oa, db + ob, idesc, ks > 0 ? 1u : 0u);
+    }
+}
+
+__global__ void __launch_bounds__(kBlkThreads, 1)
 tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
              const __nv_bfloat16* __restrict__ v, const float* __restrict__ gamma,
-             const float* __restrict__ beta, const float* __restrict__ lambda, int H, int T, int nc,
+             const float* __restrict__ beta, const float* __restrict__ lambda, int H, int T, int np,
              int cg_steps, float tol, const __half* __restrict__ img, const float* __restrict__ scales,
              float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* Hs = smem + PairSmem::oH;
-    uint8_t* Ks = smem + PairSmem::oK;
-    uint8_t* Ps = smem + PairSmem::oP;
-    uint8_t* Ws = smem + PairSmem::oW;
-    float* Mk = reinterpret_cast<float*>(smem + PairSmem::oM);
-    float* slam = reinterpret_cast<float*>(smem + PairSmem::oLam);
-    float* seb = reinterpret_cast<float*>(smem + PairSmem::oEb);
-    float* sbc = reinterpret_cast<float*>(smem + PairSmem::oB);
-    float4* red = reinterpret_cast<float4*>(smem + PairSmem::oRed);
-    float* misc = reinterpret_cast<float*>(smem + PairSmem::oMisc);
+    uint8_t* Hs = smem + BlkSmem::oH;
+    uint8_t* Ks = smem + BlkSmem::oK;
+    uint8_t* Ps = smem + BlkSmem::oP;
+    uint8_t* Ws = smem + BlkSmem::oW;
+    float* Mk = reinterpret_cast<float*>(smem + BlkSmem::oM);
+    float* slam = reinterpret_cast<float*>(smem + BlkSmem::oLam);
+    float* seb = reinterpret_cast<float*>(smem + BlkSmem::oEb);
+    float* sbc = reinterpret_cast<float*>(smem + BlkSmem::oB);
+    float* sbeta = reinterpret_cast<float*>(smem + BlkSmem::oBeta);
+    float4* red = reinterpret_cast<float4*>(smem + BlkSmem::oRed);
+    float* misc = reinterpret_cast<float*>(smem + BlkSmem::oMisc);
     float* abort_flag = misc + 31;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + PairSmem::oBar);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + BlkSmem::oBar);
     uint64_t* bar_s = bar_ld + 1;
     uint64_t* bar_u = bar_ld + 2;
     uint64_t* bar_z = bar_ld + 3;
-    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + PairSmem::oSlot);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + BlkSmem::oSlot);
 
-    const int pr = blockIdx.x, bh = blockIdx.y, head = bh % H;
-    const int cA = 2 * pr;
-    const bool hasB = cA + 1 < nc;
-    const int t0 = cA * kC;
-    const int nA = min(kC, T - t0);
-    const int nB = hasB ? min(kC, T - t0 - kC) : 0;
+    const int blk = blockIdx.x, bh = blockIdx.y, head = bh % H;
+    const int t0 = blk * kBlk;
+    const int n = min(kBlk, T - t0);
     const size_t base = (size_t)bh * T + t0;       // token tok of the CTA is base + tok
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int q4 = w & 3, cq = w >> 2;
     const int tok = 32 * q4 + lane;                  // 0..127 = TMEM lane
-    const int ch = tok >> 6;                          // 0: chunk A, 1: chunk B
-    const bool valid = (tok & 63) < (ch ? nB : nA);
+    const bool valid = tok < n;
     const int col0 = 32 * cq;                         // this thread's 32 columns
-    const size_t ciA = (size_t)bh * nc + cA, ciB = hasB ? ciA + 1 : ciA;
+    const size_t ci = (size_t)bh * np + blk;          // state image of the block
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
@@ -507,73 +550,68 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     tc_fence_after();
     const uint32_t tbase = *slot;
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);     // this warp's lane quadrant
-    // TMEM columns: U [0,256), S / Z / y [256,384), x [384,512)
-    constexpr uint32_t kColU = 0, kColS = 256, kColX = 384;
+    constexpr uint32_t kColU = 0, kColS = 128, kColX = 256, kColR = 384;
 
-    // bulk loads of the two chunk-start H images: per K block, rows of A then rows of B
-    auto load_state_images = [&](int which) {   // which: 0 = H, 1 = G
-        mbar_arrive_expect_tx(bar_ld, 4 * 16384);
-        const uint8_t* a = reinterpret_cast<const uint8_t*>(img + (ciA * 2 + which) * kImgHalves);
-        const uint8_t* b = reinterpret_cast<const uint8_t*>(img + (ciB * 2 + which) * kImgHalves);
-        bulk_g2s(Hs, a, 16384, bar_ld);
-        bulk_g2s(Hs + 16384, b, 16384, bar_ld);
-        bulk_g2s(Hs + 32768, a + 16384, 16384, bar_ld);
-        bulk_g2s(Hs + 49152, b + 16384, 16384, bar_ld);
+    auto load_state_image = [&](int which) {   // which: 0 = H, 1 = G (thread 0)
+        mbar_arrive_expect_tx(bar_ld, kImgBytes);
+        bulk_g2s(Hs, img + (ci * 2 + which) * kImgHalves, kImgBytes, bar_ld);
     };
-    if (tid == 0) load_state_images(0);
-    const float sH = scales[(ch ? ciB : ciA) * 2 + 0], sG = scales[(ch ? ciB : ciA) * 2 + 1];
+    if (tid == 0) load_state_image(0);
+    const float sH = scales[ci * 2 + 0];
 
-    // gates (warp 0: chunk A, warp 1: chunk B), lambda, key image, zeroed score image
-    if (w < 2) warp_chunk_gates(gamma, base + kC * w, w ? nB : nA, sbc + kC * w);
-    if (tid < kD) slam[tid] = lambda[(size_t)head * kD + tid];
+    // gates, beta, lambda, key image, zeroed score image
+    if (w == 0) warp_gate_cumsum128(gamma + base, n, sbc);
+    if (tid < kBlk) sbeta[tid] = (tid < n) ? beta[base + tid] : 0.f;
+    else if (tid < kBlk + kD) slam[tid - kBlk] = lambda[(size_t)head * kD + tid - kBlk];
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
-        const int cid = tid + kPairThreads * rep;       // 2048 16-byte chunks
+        const int cid = tid + kBlkThreads * rep;       // 2048 16-byte chunks
         const int j = cid >> 4, cc = cid & 15;
-        const bool ok = (j & 63) < ((j >> 6) ? nB : nA);
         uint4 rk = make_uint4(0, 0, 0, 0);
-        if (ok) rk = *reinterpret_cast<const uint4*>(k + (base + j) * kD + 8 * cc);
+        if (j < n) rk = *reinterpret_cast<const uint4*>(k + (base + j) * kD + 8 * cc);
         *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
             bf16x8_to_f16x8(rk, 1.f);
         reinterpret_cast<uint4*>(Ws)[cid] = make_uint4(0, 0, 0, 0);
     }
-    // CG state: x = 0 (TMEM), r = p = q; this thread: token tok, columns col0..col0+31
-    float2 r[16], p[16];
+    // CG state: x = 0 and r = q in TMEM, p = q in registers; this thread: token tok, columns col0..col0+31
+    float2 p[16];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         uint4 raw = make_uint4(0, 0, 0, 0);
         if (valid) raw = *reinterpret_cast<const uint4*>(q + (base + tok) * kD + col0 + 8 * g);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            r[4 * g + i] = __bfloat1622float2(b2[i]);
-            p[4 * g + i] = r[4 * g + i];
-        }
+        for (int i = 0; i < 4; ++i) p[4 * g + i] = __bfloat1622float2(b2[i]);
     }
-    {
-        float z[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0.f;
-        tmem_st32_x16(tl + kColX + col0, z);
-        tmem_st32_x16(tl + kColX + col0 + 16, z);
+    for (int h2 = 0; h2 < 4; ++h2) {
+        float z[8], rv[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            z[2 * i] = 0.f;
+            z[2 * i + 1] = 0.f;
+            rv[2 * i] = p[4 * h2 + i].x;
+            rv[2 * i + 1] = p[4 * h2 + i].y;
+        }
+        tmem_st32_x8(tl + kColX + col0 + 8 * h2, z);
+        tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
     }
-    __syncthreads();                                   // gates visible
-    if (tid < 128) seb[tid] = expf(sbc[tid]);
+    __syncthreads();                                   // gates and beta visible
+    if (tid < kBlk) seb[tid] = expf(sbc[tid]);
     {
-        for (int e = tid; e < 128 * kC; e += kPairThreads) {
-            const int tt = e >> 6, jl = e & 63, c = tt >> 6, tlc = tt & 63;
-            const int n = c ? nB : nA;
-            const float s_h = scales[(c ? ciB : ciA) * 2 + 0];
-            Mk[tt * PairSmem::kMS + jl] = (jl <= tlc && tlc < n)
-                        ? beta[base + kC * c + jl] * expf(sbc[tt] - sbc[kC * c + jl]) / s_h
-                        : 0.f;
+        const float inv_sH = 1.f / sH;                 // power of two: exact
+        for (int e = tid; e < kBlk * kBlk; e += kBlkThreads) {
+            const int tt = e >> 7, j = e & 127;
+            float m = 0.f;
+            if (j <= tt && tt < n) m = sbeta[j] * expf(sbc[tt] - sbc[j]) * inv_sH;
+            Mk[tt * BlkSmem::kMS + j] = m;
         }
     }
     float rr;
     {
         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a = __ffma2_rn(r[i], r[i], a);
+        for (int i = 0; i < 16; ++i) a = __ffma2_rn(p[i], p[i], a);
         rr = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;   // barrier publishes seb, Mk
     }
     tmem_wait_st();
@@ -584,38 +622,22 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     float s = pow2_sqrt_scale(rr), is = 1.f / s;
     store_row32(Ps, tok, col0, p, is);
 
-    constexpr uint32_t kIdS = idesc_f16(128, 128, false, false);
-    constexpr uint32_t kIdU = idesc_f16(128, 256, false, false);
-    constexpr uint32_t kIdZ = idesc_f16(128, 128, false, true);
-    auto issue_S = [&]() {      // S = P K^T -> columns [256, 384)
-        const uint64_t dA = sdesc(smem_addr(Ps), 16, 1024), dB = sdesc(smem_addr(Ks), 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t o = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase + kColS, dA + o, dB + o, kIdS, ks > 0 ? 1u : 0u);
-        }
+    constexpr uint32_t kIdKK = idesc_f16(128, 128, false, false);     // A and B K-major
+    constexpr uint32_t kIdKM = idesc_f16(128, 128, false, true);      // B MN-major
+    auto issue_S = [&]() {      // S = P K^T -> columns [128, 256)
+        issue_k128(tbase + kColS, smem_addr(Ps), smem_addr(Ks), 16, 16384, 16384, 32, kIdKK);
     };
-    auto issue_U = [&]() {      // U = P [H_A; H_B]^T -> columns [0, 256)
-        const uint64_t dA = sdesc(smem_addr(Ps), 16, 1024), dB = sdesc(smem_addr(Hs), 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t oa = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
-            const uint32_t ob = ((ks >> 2) * 32768 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase + kColU, dA + oa, dB + ob, kIdU, ks > 0 ? 1u : 0u);
-        }
+    auto issue_U = [&]() {      // U = P H^T -> columns [0, 128)
+        issue_k128(tbase + kColU, smem_addr(Ps), smem_addr(Hs), 16, 16384, 16384, 32, kIdKK);
     };
-    auto issue_Z = [&]() {      // Z = W K -> columns [256, 384)
-        const uint64_t dA = sdesc(smem_addr(Ws), 16, 1024), dB = sdesc(smem_addr(Ks), 16384, 1024);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t oa = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
-            mma_f16(tbase + kColS, dA + oa, dB + ((ks * 2048) >> 4), kIdZ, ks > 0 ? 1u : 0u);
-        }
+    auto issue_Z = [&]() {      // Z = W K -> columns [128, 256)
+        issue_k128(tbase + kColS, smem_addr(Ws), smem_addr(Ks), 16384, 16384, 8192, 2048, kIdKM);
     };
-    // S (TMEM) -> decay-masked, scaled scores -> the diagonal block of the score image
+    // S (TMEM) -> decay-masked, scaled scores -> score image. The quarter of
+    // tokens 0..63 against keys 64..127 lies above the diagonal: it stays zero.
     auto masked_scores = [&](float extra) {
-        if ((cq >> 1) != ch) return;                   // off-diagonal quarter: block stays zero
-        const float* mrow = Mk + tok * PairSmem::kMS + (col0 & 63);
+        if (q4 < 2 && cq >= 2) return;                 // warp-uniform
+        const float* mrow = Mk + tok * BlkSmem::kMS + col0;
         float2 wv[16];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -668,21 +690,23 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             float2 a = make_float2(0.f, 0.f), b = a, cc = a, e = a;
 #pragma unroll
             for (int h2 = 0; h2 < 4; ++h2) {
-                float uv[8], zv[8];
-                tmem_ld32_x8(tl + kColU + 128 * ch + col0 + 8 * h2, uv);
+                float uv[8], zv[8], rv[8];
+                tmem_ld32_x8(tl + kColU + col0 + 8 * h2, uv);
                 tmem_ld32_x8(tl + kColS + col0 + 8 * h2, zv);
+                tmem_ld32_x8(tl + kColR + col0 + 8 * h2, rv);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int pi = 4 * h2 + i;
                     const float2 lm = *reinterpret_cast<const float2*>(slam + col0 + 2 * pi);
+                    const float2 rp = make_float2(rv[2 * i], rv[2 * i + 1]);
                     float2 y = __ffma2_rn(make_float2(uv[2 * i], uv[2 * i + 1]), make_float2(c_u, c_u),
                                           __fmul2_rn(lm, p[pi]));
                     y = __ffma2_rn(make_float2(zv[2 * i], zv[2 * i + 1]), make_float2(c_z, c_z), y);
                     a = __ffma2_rn(p[pi], y, a);
-                    b = __ffma2_rn(r[pi], y, b);
+                    b = __ffma2_rn(rp, y, b);
                     cc = __ffma2_rn(y, y, cc);
-                    e = __ffma2_rn(r[pi], r[pi], e);
+                    e = __ffma2_rn(rp, rp, e);
                     zv[2 * i] = y.x;
                     zv[2 * i + 1] = y.y;
                 }
@@ -700,9 +724,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         const float2 pa = make_float2(al, al), na = make_float2(-al, -al), rh = make_float2(rho, rho);
 #pragma unroll
         for (int h2 = 0; h2 < 4; ++h2) {               // x += alpha p; r -= alpha y; p = r + rho p
-            float xv[8], yv[8];
+            float xv[8], yv[8], rv[8];
             tmem_ld32_x8(tl + kColX + col0 + 8 * h2, xv);
             tmem_ld32_x8(tl + kColS + col0 + 8 * h2, yv);
+            tmem_ld32_x8(tl + kColR + col0 + 8 * h2, rv);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -711,11 +736,15 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
                 xv[2 * i] = x.x;
                 xv[2 * i + 1] = x.y;
                 if (act) {
-                    r[pi] = __ffma2_rn(na, make_float2(yv[2 * i], yv[2 * i + 1]), r[pi]);
-                    p[pi] = __ffma2_rn(rh, p[pi], r[pi]);
+                    const float2 r = __ffma2_rn(na, make_float2(yv[2 * i], yv[2 * i + 1]),
+                                                make_float2(rv[2 * i], rv[2 * i + 1]));
+                    p[pi] = __ffma2_rn(rh, p[pi], r);
+                    rv[2 * i] = r.x;
+                    rv[2 * i + 1] = r.y;
                 }
             }
             tmem_st32_x8(tl + kColX + col0 + 8 * h2, xv);
+            tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
         }
         if (act) {
             rr = rn;
@@ -729,26 +758,33 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 
     // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern ----
     __syncthreads();                                   // last reduction's readers are done with red[]
-    float2 xr[16];
+    float xs;
     {
-        float xv[16];
+        float2 xr[16];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
+            float xv[16];
             tmem_ld32_x16(tl + kColX + col0 + 16 * h2, xv);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 8; ++i) xr[8 * h2 + i] = make_float2(xv[2 * i], xv[2 * i + 1]);
         }
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
+        const float xx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;
+        xs = xx > 0.f ? sqrtf(xx) : 1.f;
+        store_row32(Ps, tok, col0, xr, 1.f / xs);
     }
+    // values of the block (kept in registers until the key image is free) and max |v|
     uint4 vraw[4];
     float vmax = 0.f;
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
-        const int cid = tid + kPairThreads * rep;
+        const int cid = tid + kBlkThreads * rep;
         const int j = cid >> 4, cc = cid & 15;
-        const bool ok = (j & 63) < ((j >> 6) ? nB : nA);
         vraw[rep] = make_uint4(0, 0, 0, 0);
-        if (ok) vraw[rep] = *reinterpret_cast<const uint4*>(v + (base + j) * kD + 8 * cc);
+        if (j < n) vraw[rep] = *reinterpret_cast<const uint4*>(v + (base + j) * kD + 8 * cc);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[rep]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -759,27 +795,19 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
     if (lane == 0) misc[w] = vmax;
-    float xs;
-    {
-        float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
-        const float xx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;   // publishes misc
-        xs = xx > 0.f ? sqrtf(xx) : 1.f;
-    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();                                   // publishes X-hat and misc
+    tc_fence_after();
     float vm = misc[0];
 #pragma unroll
     for (int i = 1; i < 16; ++i) vm = fmaxf(vm, misc[i]);
     const float sV = pow2_ceil_at_least_one(vm);
-    store_row32(Ps, tok, col0, xr, 1.f / xs);
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    const float sG = scales[ci * 2 + 1];
     bool ok = *abort_flag == 0.f;
     if (ok) {
         if (tid == 0) {
-            load_state_images(1);              // every MMA that read the H images is done
+            load_state_image(1);               // every MMA that read the H image is done
             issue_S();                         // S' = X-hat K^T
             mma_commit(bar_s);
         }
@@ -788,7 +816,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         const float inv_sV = 1.f / sV;
 #pragma unroll
         for (int rep = 0; rep < 4; ++rep) {    // the key image is dead: values take its place
-            const int cid = tid + kPairThreads * rep;
+            const int cid = tid + kBlkThreads * rep;
             const int j = cid >> 4, cc = cid & 15;
             *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
                 bf16x8_to_f16x8(vraw[rep], inv_sV);
@@ -806,7 +834,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
                 mma_commit(bar_u);
                 mma_commit(bar_z);
             } else {
-                issue_U();                     // U' = X-hat [G_A; G_B]^T
+                issue_U();                     // U' = X-hat G^T
                 mma_commit(bar_u);
                 issue_Z();                     // Z' = W' V
                 mma_commit(bar_z);
@@ -823,7 +851,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
             float uv[16], zv[16];
-            tmem_ld32_x16(tl + kColU + 128 * ch + col0 + 16 * h2, uv);
+            tmem_ld32_x16(tl + kColU + col0 + 16 * h2, uv);
             tmem_ld32_x16(tl + kColS + col0 + 16 * h2, zv);
             tmem_wait_ld();
             if (valid) {
@@ -854,14 +882,15 @@ bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype) {
     return dtype == MESA_BF16 && dk == kD && dv == kD && chunk == kC;
 }
 
+// One H and one G image (and their scales) per 128-token block.
 static size_t images_bytes(int B, int H, int T) {
-    const size_t nc = (size_t)((T + kC - 1) / kC);
-    return (size_t)B * H * nc * 2 * kImgBytes;
+    const size_t np = (size_t)((T + kBlk - 1) / kBlk);
+    return (size_t)B * H * np * 2 * kImgBytes;
 }
 
 size_t tc_workspace_bytes(int B, int H, int T) {
-    const size_t nc = (size_t)((T + kC - 1) / kC);
-    return images_bytes(B, H, T) + ((size_t)B * H * nc * 2 * sizeof(float) + 255) / 256 * 256;
+    const size_t np = (size_t)((T + kBlk - 1) / kBlk);
+    return images_bytes(B, H, T) + ((size_t)B * H * np * 2 * sizeof(float) + 255) / 256 * 256;
 }
 
 cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
@@ -871,7 +900,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     float* scales = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + images_bytes(a.B, a.H, a.T));
     unsigned* err = error_word_ptr();
     const int scan_smem = ScanSmem::bytes + 1024;
-    const int cg_smem = PairSmem::bytes + 1024;
+    const int cg_smem = BlkSmem::bytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_cg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cg_smem);
@@ -886,9 +915,9 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     {
         LaunchTimer timer(kKindTcCg, st);
-        tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kPairThreads, cg_smem, st>>>(
+        tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-            static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, nc, a.cg_steps, a.tol,
+            static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
             img, scales, a.out, a.iters, err);
     }
     return cudaGetLastError();
