@@ -421,15 +421,16 @@ struct BlkSmem {
     static constexpr int oK = 32768;              // key image [128 j][128 k] (32 KB); later values
     static constexpr int oP = 65536;              // P-hat image [128 t][128 k] (32 KB); later X-hat
     static constexpr int oW = 98304;              // masked scores [128 t][128 j] (32 KB)
-    static constexpr int kMS = 130;               // mask row stride (conflict-free float2 rows)
-    static constexpr int oM = 131072;             // decay mask / sH, fp32 [128 t][128 j], stride kMS
-    static constexpr int oLam = oM + kBlk * kMS * 4;   // lambda [128]
+    static constexpr int oG = 131072;             // value-state image [128 i][128 k] (32 KB), fetched at start
+    static constexpr int kMS = 136;               // mask row stride in halves (conflict-free 16-byte rows)
+    static constexpr int oM = 163840;             // decay mask / sH, fp16 [128 t][128 j], stride kMS
+    static constexpr int oLam = oM + kBlk * kMS * 2;   // lambda [128]
     static constexpr int oEb = oLam + 512;        // e^{b_t} [128]
     static constexpr int oB = oEb + 512;          // b_t [128]
     static constexpr int oBeta = oB + 512;        // beta_j [128]
     static constexpr int oRed = oBeta + 512;      // [4 column quarters][128 tokens] float4
     static constexpr int oMisc = oRed + 8192;     // 32 floats
-    static constexpr int oBar = oMisc + 128;      // mbarriers: ld, s, u, z
+    static constexpr int oBar = oMisc + 128;      // mbarriers: ld (H), s, u, z, g (G), in (rows), v (values)
     static constexpr int oSlot = oBar + 64;
     static constexpr int bytes = oSlot + 16;
 };
@@ -487,8 +488,7 @@ __device__ __forceinline__ void store_row32(uint8_t* img, int tok, int col0, con
 // Eight K = 16 steps of one fp16 product into TMEM address d. A is a K-major
 // SW128 image (64-element K blocks a_kb bytes apart); B is K-major (b_k16 = 32)
 // or MN-major (b_lbo = MN block stride, b_k16 = 2048), its K blocks b_kb apart.
-// Kept out of line so that the descriptors live only in the issuing thread.
-__device__ __noinline__ void issue_k128(uint32_t d, uint32_t a, uint32_t b, uint32_t b_lbo, uint32_t a_kb,
+__device__ __forceinline__ void issue_k128(uint32_t d, uint32_t a, uint32_t b, uint32_t b_lbo, uint32_t a_kb,
                                         uint32_t b_kb, uint32_t b_k16, uint32_t idesc) {
     const uint64_t da = sdesc(a, 16, 1024), db = sdesc(b, b_lbo, 1024);
 #pragma unroll
@@ -511,7 +511,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     uint8_t* Ks = smem + BlkSmem::oK;
     uint8_t* Ps = smem + BlkSmem::oP;
     uint8_t* Ws = smem + BlkSmem::oW;
-    float* Mk = reinterpret_cast<float*>(smem + BlkSmem::oM);
+    uint8_t* Gs = smem + BlkSmem::oG;
+    __half* Mk = reinterpret_cast<__half*>(smem + BlkSmem::oM);
     float* slam = reinterpret_cast<float*>(smem + BlkSmem::oLam);
     float* seb = reinterpret_cast<float*>(smem + BlkSmem::oEb);
     float* sbc = reinterpret_cast<float*>(smem + BlkSmem::oB);
@@ -523,6 +524,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     uint64_t* bar_s = bar_ld + 1;
     uint64_t* bar_u = bar_ld + 2;
     uint64_t* bar_z = bar_ld + 3;
+    uint64_t* bar_g = bar_ld + 4;
+    uint64_t* bar_in = bar_ld + 5;
+    uint64_t* bar_v = bar_ld + 6;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + BlkSmem::oSlot);
 
     const int blk = blockIdx.x, bh = blockIdx.y, head = bh % H;
@@ -541,6 +545,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         mbar_init(bar_s, 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_z, 1);
+        mbar_init(bar_g, 1);
+        mbar_init(bar_in, 1);
+        mbar_init(bar_v, 1);
         fence_mbar_init();
         *abort_flag = 0.f;
     }
@@ -552,33 +559,50 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);     // this warp's lane quadrant
     constexpr uint32_t kColU = 0, kColS = 128, kColX = 256, kColR = 384;
 
-    auto load_state_image = [&](int which) {   // which: 0 = H, 1 = G (thread 0)
+    // One round of bulk copies brings everything the setup reads: both state
+    // images, the raw key rows (staged in the P-hat buffer), the raw query rows
+    // (staged in the score buffer) and, for a full aligned block, gamma and beta
+    // (staged in the reduction buffer).
+    const uint32_t row_bytes = (uint32_t)n * kD * 2;
+    const bool gates_bulk = n == kBlk && ((reinterpret_cast<uintptr_t>(gamma + base) |
+                                            reinterpret_cast<uintptr_t>(beta + base)) & 15) == 0;
+    float* gstage = reinterpret_cast<float*>(red);
+    if (tid == 0) {
         mbar_arrive_expect_tx(bar_ld, kImgBytes);
-        bulk_g2s(Hs, img + (ci * 2 + which) * kImgHalves, kImgBytes, bar_ld);
-    };
-    if (tid == 0) load_state_image(0);
+        bulk_g2s(Hs, img + (ci * 2 + 0) * kImgHalves, kImgBytes, bar_ld);
+        mbar_arrive_expect_tx(bar_g, kImgBytes);
+        bulk_g2s(Gs, img + (ci * 2 + 1) * kImgHalves, kImgBytes, bar_g);
+        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u));
+        bulk_g2s(Ps, k + base * kD, row_bytes, bar_in);
+        bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
+        if (gates_bulk) {
+            bulk_g2s(gstage, gamma + base, kBlk * 4, bar_in);
+            bulk_g2s(gstage + kBlk, beta + base, kBlk * 4, bar_in);
+        }
+    }
     const float sH = scales[ci * 2 + 0];
+    if (tid >= kBlk && tid < kBlk + kD) slam[tid - kBlk] = lambda[(size_t)head * kD + tid - kBlk];
+    if (tid == 0 && !mbar_wait(bar_in, 0)) *abort_flag = 1.f;
+    __syncthreads();
 
-    // gates, beta, lambda, key image, zeroed score image
-    if (w == 0) warp_gate_cumsum128(gamma + base, n, sbc);
-    if (tid < kBlk) sbeta[tid] = (tid < n) ? beta[base + tid] : 0.f;
-    else if (tid < kBlk + kD) slam[tid - kBlk] = lambda[(size_t)head * kD + tid - kBlk];
+    // gates, beta, key image (from the staged rows)
+    if (w == 0) warp_gate_cumsum128(gates_bulk ? gstage : gamma + base, n, sbc);
+    if (tid < kBlk) sbeta[tid] = (tid < n) ? (gates_bulk ? gstage[kBlk + tid] : beta[base + tid]) : 0.f;
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
         const int cid = tid + kBlkThreads * rep;       // 2048 16-byte chunks
         const int j = cid >> 4, cc = cid & 15;
         uint4 rk = make_uint4(0, 0, 0, 0);
-        if (j < n) rk = *reinterpret_cast<const uint4*>(k + (base + j) * kD + 8 * cc);
+        if (j < n) rk = *reinterpret_cast<const uint4*>(Ps + j * 256 + cc * 16);
         *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
             bf16x8_to_f16x8(rk, 1.f);
-        reinterpret_cast<uint4*>(Ws)[cid] = make_uint4(0, 0, 0, 0);
     }
     // CG state: x = 0 and r = q in TMEM, p = q in registers; this thread: token tok, columns col0..col0+31
     float2 p[16];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         uint4 raw = make_uint4(0, 0, 0, 0);
-        if (valid) raw = *reinterpret_cast<const uint4*>(q + (base + tok) * kD + col0 + 8 * g);
+        if (valid) raw = *reinterpret_cast<const uint4*>(Ws + tok * 256 + (col0 + 8 * g) * 2);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
         for (int i = 0; i < 4; ++i) p[4 * g + i] = __bfloat1622float2(b2[i]);
@@ -596,15 +620,23 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tmem_st32_x8(tl + kColX + col0 + 8 * h2, z);
         tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
     }
-    __syncthreads();                                   // gates and beta visible
+    __syncthreads();                                   // gates and beta visible, staged rows consumed
     if (tid < kBlk) seb[tid] = expf(sbc[tid]);
+#pragma unroll
+    for (int rep = 0; rep < 4; ++rep) reinterpret_cast<uint4*>(Ws)[tid + kBlkThreads * rep] = make_uint4(0, 0, 0, 0);
     {
+        // M_tj / sH for j <= t, as fp16 pairs. The exponent b_t - b_j is <= 0; the
+        // fast exponential's few-ulp error is far below the fp16 rounding that follows.
         const float inv_sH = 1.f / sH;                 // power of two: exact
-        for (int e = tid; e < kBlk * kBlk; e += kBlkThreads) {
-            const int tt = e >> 7, j = e & 127;
-            float m = 0.f;
-            if (j <= tt && tt < n) m = sbeta[j] * expf(sbc[tt] - sbc[j]) * inv_sH;
-            Mk[tt * BlkSmem::kMS + j] = m;
+        for (int e = tid; e < kBlk * kBlk / 2; e += kBlkThreads) {
+            const int tt = e >> 6, j = 2 * (e & 63);
+            float m0 = 0.f, m1 = 0.f;
+            if (tt < n) {
+                const float bt = sbc[tt];
+                if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * inv_sH;
+                if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * inv_sH;
+            }
+            *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
         }
     }
     float rr;
@@ -637,7 +669,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     // tokens 0..63 against keys 64..127 lies above the diagonal: it stays zero.
     auto masked_scores = [&](float extra) {
         if (q4 < 2 && cq >= 2) return;                 // warp-uniform
-        const float* mrow = Mk + tok * BlkSmem::kMS + col0;
+        const __half* mrow = Mk + tok * BlkSmem::kMS + col0;
         float2 wv[16];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -645,9 +677,15 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             tmem_ld32_x16(tl + kColS + col0 + 16 * h2, sv);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float2 m = *reinterpret_cast<const float2*>(mrow + 16 * h2 + 2 * i);
-                wv[8 * h2 + i] = __fmul2_rn(m, make_float2(sv[2 * i] * extra, sv[2 * i + 1] * extra));
+            for (int g = 0; g < 2; ++g) {
+                const uint4 m8 = *reinterpret_cast<const uint4*>(mrow + 16 * h2 + 8 * g);
+                const __half2* m2 = reinterpret_cast<const __half2*>(&m8);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = 4 * g + i;
+                    wv[8 * h2 + c] = __fmul2_rn(__half22float2(m2[i]),
+                                                make_float2(sv[2 * c] * extra, sv[2 * c + 1] * extra));
+                }
             }
         }
         store_row32(Ws, tok, col0, wv, 1.f);
@@ -718,10 +756,15 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         d = quarter_sum(d, red, cq, tok);
         if (act && !cg_curvature_ok(d.x)) act = false;
         if (act) rr = d.w;                             // true |r|^2 of the current residual
-        const float al = act ? rr / d.x : 0.f;
+        // alpha and rho feed recurrences that CG corrects: the fast division suffices
+        const float al = act ? __fdividef(rr, d.x) : 0.f;
         const float rn = fmaxf(fmaf(al, fmaf(al, d.z, -2.f * d.y), rr), 0.f);
-        const float rho = act ? rn / rr : 0.f;
+        const float rho = act ? __fdividef(rn, rr) : 0.f;
         const float2 pa = make_float2(al, al), na = make_float2(-al, -al), rh = make_float2(rho, rho);
+        // the next direction's image is written round by round (its scale is known here)
+        const float s_new = act ? pow2_sqrt_scale(rn) : s;
+        const float is_new = 1.f / s_new;
+        uint8_t* prow = Ps + (col0 >> 6) * 16384 + tok * 128;
 #pragma unroll
         for (int h2 = 0; h2 < 4; ++h2) {               // x += alpha p; r -= alpha y; p = r + rho p
             float xv[8], yv[8], rv[8];
@@ -745,18 +788,29 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             }
             tmem_st32_x8(tl + kColX + col0 + 8 * h2, xv);
             tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
+            {
+                const float2 f = make_float2(is_new, is_new);
+                const float2 a0 = __fmul2_rn(p[4 * h2], f), a1 = __fmul2_rn(p[4 * h2 + 1], f);
+                const float2 a2 = __fmul2_rn(p[4 * h2 + 2], f), a3 = __fmul2_rn(p[4 * h2 + 3], f);
+                *reinterpret_cast<uint4*>(prow + (((((col0 & 63) >> 3) + h2) ^ (tok & 7)) << 4)) =
+                    make_uint4(pack_half2(a0.x, a0.y), pack_half2(a1.x, a1.y), pack_half2(a2.x, a2.y),
+                               pack_half2(a3.x, a3.y));
+            }
         }
         if (act) {
             rr = rn;
             ++it;
-            s = pow2_sqrt_scale(rr);
-            is = 1.f / s;
         }
+        s = s_new;
+        is = is_new;
         tmem_wait_st();
-        store_row32(Ps, tok, col0, p, is);
     }
 
     // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern ----
+    if (tid == 0) {            // raw value rows into the dead H buffer, while x is normalised
+        mbar_arrive_expect_tx(bar_v, row_bytes);
+        bulk_g2s(Hs, v + base * kD, row_bytes, bar_v);
+    }
     __syncthreads();                                   // last reduction's readers are done with red[]
     float xs;
     {
@@ -777,6 +831,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         store_row32(Ps, tok, col0, xr, 1.f / xs);
     }
     // values of the block (kept in registers until the key image is free) and max |v|
+    if (!mbar_wait(bar_v, 0)) *abort_flag = 1.f;
     uint4 vraw[4];
     float vmax = 0.f;
 #pragma unroll
@@ -784,7 +839,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         const int cid = tid + kBlkThreads * rep;
         const int j = cid >> 4, cc = cid & 15;
         vraw[rep] = make_uint4(0, 0, 0, 0);
-        if (j < n) vraw[rep] = *reinterpret_cast<const uint4*>(v + (base + j) * kD + 8 * cc);
+        if (j < n) vraw[rep] = *reinterpret_cast<const uint4*>(Hs + j * 256 + cc * 16);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[rep]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -807,7 +862,6 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     bool ok = *abort_flag == 0.f;
     if (ok) {
         if (tid == 0) {
-            load_state_image(1);               // every MMA that read the H image is done
             issue_S();                         // S' = X-hat K^T
             mma_commit(bar_s);
         }
@@ -829,12 +883,12 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     }
     if (ok) {
         if (tid == 0) {
-            if (!mbar_wait(bar_ld, 1)) {
+            if (!mbar_wait(bar_g, 0)) {
                 *abort_flag = 1.f;
                 mma_commit(bar_u);
                 mma_commit(bar_z);
             } else {
-                issue_U();                     // U' = X-hat G^T
+                issue_k128(tbase + kColU, smem_addr(Ps), smem_addr(Gs), 16, 16384, 16384, 32, kIdKK);   // U' = X-hat G^T
                 mma_commit(bar_u);
                 issue_Z();                     // Z' = W' V
                 mma_commit(bar_z);
@@ -870,6 +924,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         mma_commit(bar_ld);
         mbar_wait(bar_ld, 0);
         mbar_wait(bar_ld, 1);
+        mbar_wait(bar_g, 0);
     }
     tc_fence_before();
     __syncthreads();
