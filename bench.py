@@ -52,8 +52,8 @@ def load_peaks():
 # of one launch / tokens of that launch). Reported only while the kernel
 # source still hashes to the captured version; otherwise the field is null.
 MEASURED_TRAFFIC = {
-    "tc_cg": {"src_sha16": "6cb7cfa309f72f83", "bytes_per_token": (471.978752e6 + 117.958912e6) / 262144},
-    "tc_scan": {"src_sha16": "6cb7cfa309f72f83", "bytes_per_token": (136.758016e6 + 213.465856e6) / 262144},
+    "tc_cg": {"src_sha16": "e471cec71b584f3a", "bytes_per_token": (338.001920e6 + 107.907072e6) / 262144},
+    "tc_scan": {"src_sha16": "e471cec71b584f3a", "bytes_per_token": (136.506368e6 + 93.002752e6) / 262144},
 }
 
 

@@ -25,18 +25,21 @@
 //     the fp32 running states carry ~22-bit products.
 //
 // Kernels:
-//   tc_scan_kernel  grid (2, B*H): CTA (m, bh) walks the chunks of sequence bh
-//                   for m = 0 (H) or 1 (G). Per chunk one M=128,N=128,K=128
-//                   MMA forms the weighted outer-product sum in TMEM; the
-//                   running fp32 state lives in registers (thread: one row,
-//                   64 columns) and each chunk-start state is written as a
-//                   swizzled fp16 image ready to be a shared-memory operand.
-//   tc_cg_kernel    grid (chunks, B*H), 2 CTAs per SM: one CTA runs every CG
-//                   iteration of one chunk and the read-out. Tokens are the
-//                   MMA M dimension (M = 64), so each token's CG vectors sit
-//                   in the registers of 8 threads and every dot product is a
-//                   thread-local sum plus a 4-lane shuffle and one shared-
-//                   memory exchange. x lives in TMEM.
+//   tc_scan_kernel  grid (4, B*H): CTA (m, nb, bh) walks the chunks of sequence
+//                   bh for m = 0 (H) or 1 (G), column block nb. Per chunk an
+//                   M=128, N=64 MMA over the chunk's 64 tokens, issued for the
+//                   hi and the lo fp16 parts (8 K steps), forms the weighted
+//                   outer-product sum in TMEM; the running fp32 state lives in
+//                   registers and the
+//                   state before every even chunk (the start of a 128-token
+//                   block) is written as a swizzled fp16 image that the solve
+//                   loads with one bulk copy.
+//   tc_cg_kernel    grid (ceil(T/128), B*H), one CTA per SM: one CTA runs every
+//                   CG iteration of a 128-token block and the read-out. Tokens
+//                   are the MMA M dimension (M = 128, lane = token); x and r
+//                   live in TMEM, p in registers (thread: one token, 32
+//                   columns); every dot product is a thread-local sum plus one
+//                   shared-memory exchange across the four column quarters.
 #include "mesa_common.cuh"
 #include "mesa_internal.h"
 #include "tc_common.cuh"
