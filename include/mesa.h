@@ -158,12 +158,19 @@ size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int
 
 /*
  * The same forward with every tensor in HOST memory (page-locked memory is
- * recommended for overlap; pageable memory works but is slower). The call
- * enqueues one host-to-device copy per input, the forward, and one
- * device-to-host copy per requested output on `stream`, then synchronises
- * the stream before returning, so the host outputs are valid on MESA_OK.
- * No host alignment is required. `workspace` is DEVICE memory of at least
- * mesa_forward_host_workspace_size() bytes, 256-byte aligned.
+ * needed for the copies to overlap; pageable memory works but is slower).
+ * The batch is split into up to 8 slices of whole batch rows b (one slice
+ * when the inputs are under 16 MiB). Slice by slice, the inputs are copied to
+ * the device on a library copy-in stream, the forward runs on one of two
+ * library compute streams once they have landed, and the outputs are copied
+ * back on a library copy-out stream, so both copy directions overlap the
+ * kernels. The library streams start after the work already enqueued on
+ * `stream`, `stream` waits for the last copy, and the call synchronises
+ * `stream` before returning, so the host outputs are valid on MESA_OK.
+ * Calls from several host threads are serialised by a library lock (the
+ * library streams are shared per device). No host alignment is required.
+ * `workspace` is DEVICE memory of at least mesa_forward_host_workspace_size()
+ * bytes, 256-byte aligned.
  */
 mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
                               const float* gamma, const float* beta, const float* lambda,

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
 #include <vector>
 
 #include "mesa_common.cuh"
@@ -120,6 +121,47 @@ unsigned* error_word_ptr() {
 
 using namespace mesa;
 
+namespace mesa {
+namespace {
+
+// Streams and events of the host-buffer pipeline, created once per device and
+// kept for the life of the process. The pipeline splits the batch into slices
+// of whole batch rows b (every (b, h) sequence is independent): slice i's
+// inputs go up on the copy-in stream, its forward runs on compute stream i % 2
+// once they have landed, and its outputs come down on the copy-out stream once
+// it is done, so the two copy directions and the kernels overlap.
+constexpr int kMaxSlices = 8;
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr, comp[2] = {nullptr, nullptr};
+    cudaEvent_t start = nullptr, end = nullptr, landed[kMaxSlices] = {}, done[kMaxSlices] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mutex;
+
+HostPipe* host_pipe() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    HostPipe& hp = g_pipe[dev];
+    if (hp.ready) return &hp;
+    const unsigned sf = cudaStreamNonBlocking, ef = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&hp.in, sf) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, sf) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.comp[0], sf) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.comp[1], sf) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.end, ef) == cudaSuccess;
+    for (int i = 0; ok && i < kMaxSlices; ++i)
+        ok = cudaEventCreateWithFlags(&hp.landed[i], ef) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.done[i], ef) == cudaSuccess;
+    if (!ok) return nullptr;
+    hp.ready = true;
+    return &hp;
+}
+
+}  // namespace
+}  // namespace mesa
+
 extern "C" {
 
 int mesa_version(void) { return 10000; }
@@ -175,13 +217,16 @@ size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int
     if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
     const size_t tok = (size_t)B * H * T;
     const size_t es = elem_size(dtype);
-    size_t n = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256);
+    // forward scratch: one region per compute stream of the pipeline (each sized
+    // for a slice), never more than two slices' worth of the whole batch, plus padding
+    size_t n = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256) + 2 * 256;
     n += round_up(tok * dk * es, 256) * 2 + round_up(tok * dv * es, 256);      // q, k, v
     n += round_up(tok * 4, 256) * 2 + round_up((size_t)H * dk * 4, 256);      // gamma, beta, lambda
     n += round_up(tok * dv * 4, 256) + round_up(tok * 4, 256);                // out, iters
     n += (round_up((size_t)B * H * dk * dk * 4, 256) + round_up((size_t)B * H * dv * dk * 4, 256)) * 2;
     return n;
 }
+
 
 mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
                               const float* gamma, const float* beta, const float* lambda,
@@ -203,50 +248,90 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
 
     const size_t tok = (size_t)B * H * T;
     const size_t es = elem_size(dtype);
+    // slices: whole batch rows; one slice for small or empty problems
+    const size_t in_bytes = tok * (2 * dk + dv) * es + tok * 8;
+    const int nS = (T == 0 || in_bytes < ((size_t)16 << 20)) ? 1 : (B < kMaxSlices ? B : kMaxSlices);
+    const int Bs = (B + nS - 1) / nS;
+    const int nslices = (B + Bs - 1) / Bs;
+
     char* w = static_cast<char*>(workspace);
-    const size_t fws = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256);
-    char* cur = w + fws;
+    const size_t fws_slice = round_up(workspace_bytes(Bs, H, T, dk, dv, chunk, dtype), 256);
+    const size_t fws_total = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256) + 2 * 256;
+    const int ncomp = (nslices > 1 && 2 * fws_slice <= fws_total) ? 2 : 1;   // compute streams
+    char* fws[2] = {w, ncomp == 2 ? w + fws_slice : w};
+    char* cur = w + fws_total;
     auto carve = [&](size_t bytes) { char* p = cur; cur += round_up(bytes, 256); return p; };
-    void* dq = carve(tok * dk * es);
-    void* dk_ = carve(tok * dk * es);
-    void* dv_ = carve(tok * dv * es);
+    char* dq = carve(tok * dk * es);
+    char* dk_ = carve(tok * dk * es);
+    char* dv_ = carve(tok * dv * es);
     float* dg = reinterpret_cast<float*>(carve(tok * 4));
     float* db = reinterpret_cast<float*>(carve(tok * 4));
     float* dl = reinterpret_cast<float*>(carve((size_t)H * dk * 4));
     float* dout = reinterpret_cast<float*>(carve(tok * dv * 4));
     int32_t* dit = reinterpret_cast<int32_t*>(carve(tok * 4));
-    const size_t sb = (size_t)B * H * dk * dk * 4, gb = (size_t)B * H * dv * dk * 4;
-    float* dHi = reinterpret_cast<float*>(carve(sb));
-    float* dGi = reinterpret_cast<float*>(carve(gb));
-    float* dHo = reinterpret_cast<float*>(carve(sb));
-    float* dGo = reinterpret_cast<float*>(carve(gb));
+    const size_t hs = (size_t)dk * dk, gs = (size_t)dv * dk;     // floats per sequence
+    float* dHi = reinterpret_cast<float*>(carve((size_t)B * H * hs * 4));
+    float* dGi = reinterpret_cast<float*>(carve((size_t)B * H * gs * 4));
+    float* dHo = reinterpret_cast<float*>(carve((size_t)B * H * hs * 4));
+    float* dGo = reinterpret_cast<float*>(carve((size_t)B * H * gs * 4));
 
-    auto h2d = [&](void* dst, const void* src, size_t bytes) {
-        return bytes == 0 || cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    HostPipe* hp = host_pipe();
+    if (!hp) return MESA_ERR_CUDA;
+    auto cp = [](void* dst, const void* src, size_t bytes, cudaMemcpyKind kind, cudaStream_t sm) {
+        return bytes == 0 || cudaMemcpyAsync(dst, src, bytes, kind, sm) == cudaSuccess;
     };
-    auto d2h = [&](void* dst, const void* src, size_t bytes) {
-        return bytes == 0 || cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
-    };
-    bool ok = true;
-    if (T > 0) {
-        ok = ok && h2d(dq, q, tok * dk * es) && h2d(dk_, k, tok * dk * es) && h2d(dv_, v, tok * dv * es);
-        ok = ok && h2d(dg, gamma, tok * 4) && h2d(db, beta, tok * 4);
+    const cudaMemcpyKind H2D = cudaMemcpyHostToDevice, D2H = cudaMemcpyDeviceToHost;
+    bool ok = cudaEventRecord(hp->start, st) == cudaSuccess;       // after the caller's earlier work
+    for (cudaStream_t sm : {hp->in, hp->comp[0], hp->comp[1], hp->out})
+        ok = ok && cudaStreamWaitEvent(sm, hp->start, 0) == cudaSuccess;
+    ok = ok && cp(dl, lambda, (size_t)H * dk * 4, H2D, hp->in);
+    for (int i = 0; ok && i < nslices; ++i) {
+        const int b0 = i * Bs, nb = (B - b0 < Bs) ? B - b0 : Bs;
+        const size_t s0 = (size_t)b0 * H, ns = (size_t)nb * H;      // sequences
+        const size_t t0 = s0 * T, nt = ns * T;                        // tokens
+        const char* hq = static_cast<const char*>(q);
+        const char* hk = static_cast<const char*>(k);
+        const char* hv = static_cast<const char*>(v);
+        if (T > 0) {
+            ok = ok && cp(dq + t0 * dk * es, hq + t0 * dk * es, nt * dk * es, H2D, hp->in);
+            ok = ok && cp(dk_ + t0 * dk * es, hk + t0 * dk * es, nt * dk * es, H2D, hp->in);
+            ok = ok && cp(dv_ + t0 * dv * es, hv + t0 * dv * es, nt * dv * es, H2D, hp->in);
+            ok = ok && cp(dg + t0, gamma + t0, nt * 4, H2D, hp->in) && cp(db + t0, beta + t0, nt * 4, H2D, hp->in);
+        }
+        if (H_in) ok = ok && cp(dHi + s0 * hs, H_in + s0 * hs, ns * hs * 4, H2D, hp->in);
+        if (G_in) ok = ok && cp(dGi + s0 * gs, G_in + s0 * gs, ns * gs * 4, H2D, hp->in);
+        ok = ok && cudaEventRecord(hp->landed[i], hp->in) == cudaSuccess;
     }
-    ok = ok && h2d(dl, lambda, (size_t)H * dk * 4);
-    if (H_in) ok = ok && h2d(dHi, H_in, sb);
-    if (G_in) ok = ok && h2d(dGi, G_in, gb);
-    if (!ok) return MESA_ERR_CUDA;
-    ForwardArgs a{dq, dk_, dv_, dg, db, dl, B, H, T, dk, dv, chunk, dtype, cg_steps, tol,
-                  dout, iters_out ? dit : nullptr, H_in ? dHi : nullptr, G_in ? dGi : nullptr,
-                  H_out ? dHo : nullptr, G_out ? dGo : nullptr, w, fws};
-    s = launch_forward(a, st);
-    if (s != MESA_OK) return s;
-    if (T > 0) ok = ok && d2h(out, dout, tok * dv * 4);
-    if (T > 0 && iters_out) ok = ok && d2h(iters_out, dit, tok * 4);
-    if (H_out) ok = ok && d2h(H_out, dHo, sb);
-    if (G_out) ok = ok && d2h(G_out, dGo, gb);
-    if (!ok) return MESA_ERR_CUDA;
-    return cudaStreamSynchronize(st) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+    for (int i = 0; ok && i < nslices; ++i) {
+        const int b0 = i * Bs, nb = (B - b0 < Bs) ? B - b0 : Bs;
+        const size_t s0 = (size_t)b0 * H, t0 = s0 * T;
+        cudaStream_t cs = hp->comp[i % ncomp];
+        ok = cudaStreamWaitEvent(cs, hp->landed[i], 0) == cudaSuccess;
+        if (!ok) break;
+        ForwardArgs a{dq + t0 * dk * es, dk_ + t0 * dk * es, dv_ + t0 * dv * es, dg + t0, db + t0, dl,
+                      nb, H, T, dk, dv, chunk, dtype, cg_steps, tol,
+                      dout + t0 * dv, iters_out ? dit + t0 : nullptr,
+                      H_in ? dHi + s0 * hs : nullptr, G_in ? dGi + s0 * gs : nullptr,
+                      H_out ? dHo + s0 * hs : nullptr, G_out ? dGo + s0 * gs : nullptr,
+                      fws[i % ncomp], fws_slice};
+        s = launch_forward(a, cs);
+        if (s != MESA_OK) return s;
+        ok = cudaEventRecord(hp->done[i], cs) == cudaSuccess;
+    }
+    for (int i = 0; ok && i < nslices; ++i) {
+        const int b0 = i * Bs, nb = (B - b0 < Bs) ? B - b0 : Bs;
+        const size_t s0 = (size_t)b0 * H, ns = (size_t)nb * H, t0 = s0 * T, nt = ns * T;
+        ok = cudaStreamWaitEvent(hp->out, hp->done[i], 0) == cudaSuccess;
+        if (T > 0) ok = ok && cp(out + t0 * dv, dout + t0 * dv, nt * dv * 4, D2H, hp->out);
+        if (T > 0 && iters_out) ok = ok && cp(iters_out + t0, dit + t0, nt * 4, D2H, hp->out);
+        if (H_out) ok = ok && cp(H_out + s0 * hs, dHo + s0 * hs, ns * hs * 4, D2H, hp->out);
+        if (G_out) ok = ok && cp(G_out + s0 * gs, dGo + s0 * gs, ns * gs * 4, D2H, hp->out);
+    }
+    // the caller's stream resumes after the last copy; the call returns once it has landed
+    ok = ok && cudaEventRecord(hp->end, hp->out) == cudaSuccess && cudaStreamWaitEvent(st, hp->end, 0) == cudaSuccess;
+    const bool synced = cudaStreamSynchronize(st) == cudaSuccess;
+    return ok && synced ? MESA_OK : MESA_ERR_CUDA;
 }
 
 mesa_status mesa_step(const float* q, const float* k, const float* v,

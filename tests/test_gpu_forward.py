@@ -176,6 +176,36 @@ def test_host_buffer_variant(mesa, oracle_mod):
     assert np.allclose(Hout.numpy(), Hf, rtol=1e-4, atol=1e-5)
 
 
+@pytest.mark.parametrize("dtype,chunk,B,T", [("bf16", 64, 11, 1536), ("f32", 32, 3, 2100)])
+def test_host_pipeline_matches_device(mesa, dtype, chunk, B, T):
+    """Inputs above 16 MiB go through the sliced copy/compute pipeline (uneven
+    last slice for B = 11). Every sequence is independent, so the host-buffer
+    call must reproduce the device-buffer call bit for bit, initial and final
+    states included."""
+    w = rand_workload(128, chunk, dtype, T, B=B, H=4, N=15, seed=33)
+    dev = mi.device_batch(w, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(5)
+    Hin = torch.randn((B, 4, 128, 128), generator=g, device="cuda") * 0.01
+    Hin = Hin @ Hin.transpose(-1, -2)                  # symmetric positive semi-definite
+    Gin = torch.randn((B, 4, 128, 128), generator=g, device="cuda") * 0.01
+    out_d, it_d, Ho_d, Go_d = mesa.forward(dev["q"], dev["k"], dev["v"], dev["gamma"], dev["beta"], dev["lam"],
+                                           chunk=chunk, cg_steps=15, return_iters=True, H_in=Hin, G_in=Gin,
+                                           return_state=True)
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    h = {n: dev[n].cpu().pin_memory() for n in ("q", "k", "v", "gamma", "beta", "lam")}
+    out = torch.empty((B, 4, T, 128)).pin_memory()
+    iters = torch.empty((B, 4, T), dtype=torch.int32).pin_memory()
+    Hout = torch.empty((B, 4, 128, 128)).pin_memory()
+    Gout = torch.empty((B, 4, 128, 128)).pin_memory()
+    mesa.forward_host(h["q"], h["k"], h["v"], h["gamma"], h["beta"], h["lam"], chunk=chunk, cg_steps=15, out=out,
+                      iters=iters, H_in=Hin.cpu(), G_in=Gin.cpu(), H_out=Hout, G_out=Gout)
+    assert mesa.get_error() == 0
+    assert torch.equal(out, out_d.cpu())
+    assert torch.equal(iters, it_d.cpu())
+    assert torch.equal(Hout, Ho_d.cpu()) and torch.equal(Gout, Go_d.cpu())
+
+
 FULL = ["bf16_T2048", "bf16_T8192", "bf16_T8192_tol"]
 
 
