@@ -121,6 +121,18 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 #define MESA_R4(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3])
 
+// 16 lanes x 16 columns (thread t: lanes t/4 and t/4+8 of the base, columns
+// 2(t%4), 2(t%4)+1 of each 8-column group; v[4g..4g+1] row t/4, v[4g+2..4g+3]
+// row t/4+8).
+__device__ __forceinline__ void tmem_ld16_x2(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : MESA_R4(0), MESA_R4(4)
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_ld16_x4(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
@@ -151,6 +163,12 @@ __device__ __forceinline__ void tmem_st16_x8(uint32_t taddr, const float (&v)[32
         "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
         MESA_W4(0), MESA_W4(4), MESA_W4(8), MESA_W4(12), MESA_W4(16), MESA_W4(20), MESA_W4(24), MESA_W4(28)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16_x2(uint32_t taddr, const float (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 MESA_W4(0), MESA_W4(4)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16_x4(uint32_t taddr, const float (&v)[16]) {

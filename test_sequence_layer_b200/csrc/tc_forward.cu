@@ -540,6 +540,11 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     const int q4 = w & 3, cq = w >> 2;
     const int tok = 32 * q4 + lane;                  // 0..127 = TMEM lane
     const bool valid = tok < n;
+    // The MMA-issuing thread: tcgen05.mma stalls its thread while the tensor
+    // pipe is full, so the issuer is the first thread of warp 8 (tokens 0..31,
+    // columns 64..95), whose block of masked scores lies above the diagonal and
+    // is never computed: it issues S and U while the other warps mask scores.
+    constexpr int kIssuer = 256;
     const int col0 = 32 * cq;                         // this thread's 32 columns
     const size_t ci = (size_t)bh * np + blk;          // state image of the block
 
@@ -703,7 +708,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         const int any = __syncthreads_or(act ? 1 : 0);
         tc_fence_after();
         if (!any || *abort_flag != 0.f) break;
-        if (tid == 0) {
+        if (tid == kIssuer) {
             issue_S();
             mma_commit(bar_s);
             issue_U();
@@ -716,7 +721,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         __syncthreads();
         tc_fence_after();
         if (*abort_flag != 0.f) break;
-        if (tid == 0) {
+        if (tid == kIssuer) {
             issue_Z();
             mma_commit(bar_z);
         }
@@ -864,7 +869,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     const float sG = scales[ci * 2 + 1];
     bool ok = *abort_flag == 0.f;
     if (ok) {
-        if (tid == 0) {
+        if (tid == kIssuer) {
             issue_S();                         // S' = X-hat K^T
             mma_commit(bar_s);
         }
@@ -885,7 +890,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         ok = *abort_flag == 0.f;
     }
     if (ok) {
-        if (tid == 0) {
+        if (tid == kIssuer) {
             if (!mbar_wait(bar_g, 0)) {
                 *abort_flag = 1.f;
                 mma_commit(bar_u);
@@ -921,7 +926,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             }
         }
         if (iters && cq == 0 && valid) iters[base + tok] = it;
-    } else if (tid == 0) {
+    } else if (tid == kIssuer) {
         record_error(err, kErrTimeout);
         // one more bounded chance for every MMA issued so far to drain
         mma_commit(bar_ld);
