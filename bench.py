@@ -47,30 +47,34 @@ def load_peaks():
     return d
 
 
-# DRAM bytes moved per token by each kernel, from one ncu capture
-# (profiles/tc_kernels_bf16_T2048.md: dram__bytes_read.sum + dram__bytes_write.sum
-# of one launch / tokens of that launch). Reported only while the kernel
-# source still hashes to the captured version; otherwise the field is null.
+# DRAM bytes moved per token (per head for the decode step) by each kernel, from
+# one ncu capture (profiles/tc_kernels_bf16_T2048.md, profiles/decode_step_4096heads.md:
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch / units of that launch).
+# Reported only while the kernel source still hashes to the captured version;
+# otherwise the field is null.
 MEASURED_TRAFFIC = {
-    "tc_cg": {"src_sha16": "e471cec71b584f3a", "bytes_per_token": (338.001920e6 + 107.907072e6) / 262144},
-    "tc_scan": {"src_sha16": "e471cec71b584f3a", "bytes_per_token": (136.506368e6 + 93.002752e6) / 262144},
+    "tc_cg": {"src_sha16": "c9bf4937f22b6188", "bytes_per_token": (337.729280e6 + 108.120320e6) / 262144},
+    "tc_scan": {"src_sha16": "c9bf4937f22b6188", "bytes_per_token": (136.442624e6 + 92.728576e6) / 262144},
+    "decode_step": {"src_sha16": "4d0417ce028476ac", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
 }
 
 
-def kernel_source_sha16():
+def kernel_source_sha16(files=("tc_forward.cu", "tc_common.cuh")):
     import hashlib
     h = hashlib.sha256()
-    for f in ("tc_forward.cu", "tc_common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "test_sequence_layer_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel, tokens):
+def measured_traffic(kernel, units):
+    """Measured DRAM bytes of one launch processing `units` tokens (heads for
+    the decode step), or None when the source changed since the capture."""
     rec = MEASURED_TRAFFIC.get(kernel)
-    if rec is None or rec["src_sha16"] != kernel_source_sha16():
+    if rec is None or rec["src_sha16"] != kernel_source_sha16(rec.get("files", ("tc_forward.cu", "tc_common.cuh"))):
         return None
-    return rec["bytes_per_token"] * tokens
+    return rec["bytes_per_token"] * units
 
 
 def flops_per_token_iter(d, C):
@@ -210,7 +214,21 @@ def run_decode(args, w, world, rank, local):
     Gs = torch.empty((B, H, d, d), device=dev)
     dec = {n: [] for n in ("q", "k", "v", "gamma", "beta")}
     slab = 32
-    for b0 in range(0, B, slab):
+    if args.decode_state == "random":
+        # Seeded stand-in for a prefilled state (rank-32 sums of the same gated
+        # outer products), for profiling the step kernel without the 13 GB prefill.
+        g = torch.Generator(device=dev).manual_seed(77 + rank)
+        for b0 in range(0, B, slab):
+            kr = torch.nn.functional.normalize(torch.randn((slab, H, 32, d), generator=g, device=dev), dim=-1)
+            vr = torch.randn((slab, H, 32, d), generator=g, device=dev)
+            br = torch.sigmoid(torch.randn((slab, H, 32, 1), generator=g, device=dev))
+            Hs[b0:b0 + slab] = (kr * br).transpose(-1, -2) @ kr
+            Gs[b0:b0 + slab] = (vr * br).transpose(-1, -2) @ kr
+            x = mi.device_batch(w, dev, T=steps_total, B=slab, seed_offset=1000 * rank + b0)
+            for n in dec:
+                dec[n].append(x[n].float())
+            del x
+    for b0 in (range(0, B, slab) if args.decode_state == "prefill" else ()):
         x = mi.device_batch(w, dev, T=w.T + steps_total, B=slab, seed_offset=1000 * rank + b0)
         _, Hp, Gp = mesa.forward(*(x[n][:, :, :w.T].contiguous() for n in ("q", "k", "v", "gamma", "beta")),
                                  x["lam"], chunk=w.chunk, cg_steps=w.cg_steps, return_state=True)
@@ -269,9 +287,11 @@ def run_decode(args, w, world, rank, local):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "sequences": B, "H": H, "d": d, "prefill_tokens": w.T,
-                   "cg_steps": w.cg_steps, "l2": "state larger than L2 (%.2f GB)" % (2 * Hs.numel() * 4 / 1e9)},
+                   "cg_steps": w.cg_steps, "state": args.decode_state,
+                   "l2": "state larger than L2 (%.2f GB)" % (2 * Hs.numel() * 4 / 1e9)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "decode_step",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic("decode_step", heads),
+                     "kernel": "decode_step",
                      "avg_ms": avg_ms, "peak_kind": f"{peaks['_source']} HBM copy bandwidth"},
         "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
         "gpu_launches": sum(v[0] for v in kernels.values()),
@@ -289,6 +309,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode-state", default="prefill", choices=["prefill", "random"],
+                    help="decode: state from a mesa_forward prefill (default) or a seeded random stand-in")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference" or os.environ.get("MESA_BENCH_ALLOW_SHORT"), \
         "at least 3 warm-up steps"
