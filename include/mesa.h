@@ -229,6 +229,22 @@ int mesa_timing_read(const char** names, int* launches, double* total_ms, int ma
 /* Library version: major*10000 + minor*100 + patch. */
 int mesa_version(void);
 
+#ifdef MESA_DEBUG
+/*
+ * Debug builds only (libmesa_b200_debug.so, compiled with -DMESA_DEBUG):
+ * fault injection for the failure-detection tests; the pages have no
+ * counterpart. The next `launches` launches of the tensor-core solve kernel
+ * (bf16, d = 128, chunk 64) leave out the completion signal of their first
+ * Z product. Every thread's bounded wait on it (about one second of clock
+ * cycles) then runs out; the kernel records a timeout in the error word,
+ * lets every issued MMA and copy drain (bounded again), frees its tensor
+ * memory and returns, leaving the context usable. The forward's outputs are
+ * then undefined and mesa_get_error() returns MESA_ERR_DEVICE_TIMEOUT.
+ * Returns MESA_ERR_INVALID_ARG for launches < 0.
+ */
+mesa_status mesa_debug_skip_commit(int launches);
+#endif
+
 #ifdef __cplusplus
 }
 #endif

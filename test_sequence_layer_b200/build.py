@@ -1,6 +1,8 @@
-"""Builds libmesa_b200.so in-tree with nvcc for sm_100a.
+"""Builds libmesa_b200.so in-tree with nvcc for sm_100a, and its MESA_DEBUG
+variant libmesa_b200_debug.so (the same library plus the fault-injection
+entry point mesa_debug_skip_commit, used by the failure-detection tests).
 
-Usage: python -m test_sequence_layer_b200.build [--force] [--verbose-ptxas]
+Usage: python -m test_sequence_layer_b200.build [--force] [--verbose-ptxas] [--debug]
 """
 from __future__ import annotations
 
@@ -14,6 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmesa_b200.so")
+DEBUG_LIB = os.path.join(HERE, "libmesa_b200_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -27,28 +30,30 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib) -> bool:
+    if not os.path.exists(lib):
         return True
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, *(["-DMESA_DEBUG"] if debug else []), "-I", INCLUDE, "-I", CSRC, "-o", tmp,
+           *sources()]
     if ptxas_verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <nvtx3/nvToolsExt.h>
 #include <vector>
 
 #include "mesa_common.cuh"
@@ -90,7 +91,10 @@ cudaEvent_t take_event() {
 
 }  // namespace
 
+// Every launch is also an NVTX range named after its kernel kind, so that
+// Nsight tools show the library's kernels by name on the host timeline.
 LaunchTimer::LaunchTimer(int kind, cudaStream_t st) : slot_(-1), st_(st) {
+    nvtxRangePushA(kKindNames[kind]);
     if (!g_timing_on || g_recs.size() >= kMaxRecs) return;
     TimingRec r{kind, take_event(), take_event()};
     if (!r.start || !r.stop || cudaEventRecord(r.start, st) != cudaSuccess) {
@@ -104,6 +108,7 @@ LaunchTimer::LaunchTimer(int kind, cudaStream_t st) : slot_(-1), st_(st) {
 
 LaunchTimer::~LaunchTimer() {
     if (slot_ >= 0) cudaEventRecord(g_recs[slot_].stop, st_);
+    nvtxRangePop();
 }
 
 unsigned* error_word_ptr() {
@@ -385,6 +390,13 @@ int mesa_timing_read(const char** names, int* launches, double* total_ms, int ma
     }
     return n;
 }
+
+#ifdef MESA_DEBUG
+mesa_status mesa_debug_skip_commit(int launches) {
+    if (launches < 0) return MESA_ERR_INVALID_ARG;
+    return tc_debug_skip_commit(launches) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+#endif
 
 mesa_status mesa_get_error(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MESA_ERR_CUDA;

@@ -58,6 +58,11 @@ cudaError_t forward_simt(const ForwardArgs& a, cudaStream_t st);
 bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype);
 size_t tc_workspace_bytes(int B, int H, int T);
 cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st);
+#ifdef MESA_DEBUG
+// The next `launches` launches of the tensor-core solve kernel leave out the
+// completion signal of their first Z product (fault injection, debug builds).
+cudaError_t tc_debug_skip_commit(int launches);
+#endif
 
 // Decode step (decode.cu).
 struct StepArgs {

@@ -47,6 +47,14 @@
 namespace mesa {
 namespace {
 
+#ifdef MESA_DEBUG
+// Debug builds only: when set, the solve kernel leaves out the completion
+// signal of its first Z product, so every thread's bounded wait on it runs
+// out, the kernel records a timeout in the error word and returns.
+__device__ int g_debug_skip_commit = 0;
+int g_debug_skip_launches = 0;
+#endif
+
 using namespace tc;
 
 constexpr int kD = 128;          // dk = dv
@@ -723,6 +731,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         if (*abort_flag != 0.f) break;
         if (tid == kIssuer) {
             issue_Z();
+#ifdef MESA_DEBUG
+            if (!(step == 0 && g_debug_skip_commit))   // fault injection: nothing signals Z of step 0
+#endif
             mma_commit(bar_z);
         }
         wait_mma_each(bar_u, ph & 1, abort_flag);
@@ -976,6 +987,15 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+#ifdef MESA_DEBUG
+    static const int kOne = 1, kZero = 0;
+    const bool inject = g_debug_skip_launches > 0;
+    if (inject) {
+        --g_debug_skip_launches;
+        e = cudaMemcpyToSymbolAsync(g_debug_skip_commit, &kOne, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return e;
+    }
+#endif
     {
         LaunchTimer timer(kKindTcCg, st);
         tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
@@ -983,7 +1003,21 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
             img, scales, a.out, a.iters, err);
     }
+#ifdef MESA_DEBUG
+    if (inject) {
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return cudaMemcpyToSymbolAsync(g_debug_skip_commit, &kZero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    }
+#endif
     return cudaGetLastError();
 }
+
+#ifdef MESA_DEBUG
+cudaError_t tc_debug_skip_commit(int launches) {
+    g_debug_skip_launches = launches;
+    return cudaSuccess;
+}
+#endif
 
 }  // namespace mesa

@@ -17,12 +17,16 @@ def lib():
     return mesa._load()
 
 
-def declared_functions():
+def declared_functions(debug=False):
+    """Entry points declared in include/*.h; the MESA_DEBUG blocks only for
+    the debug build."""
     names = set()
     for fn in os.listdir(os.path.join(ROOT, "include")):
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            if not debug:
+                src = re.sub(r"#ifdef MESA_DEBUG.*?#endif", "", src, flags=re.S)
             names |= set(re.findall(r"\b(mesa_\w+)\s*\(", src))
     return sorted(names)
 
@@ -31,8 +35,21 @@ def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
     assert {"mesa_forward", "mesa_step", "mesa_forward_workspace_size", "mesa_get_error",
             "mesa_status_string", "mesa_forward_host"} <= set(names)
+    assert "mesa_debug_skip_commit" not in names
     for n in names:
         assert hasattr(lib, n), n
+    assert not hasattr(lib, "mesa_debug_skip_commit")          # fault injection lives in the debug build only
+
+
+def test_debug_build_exports_the_injection_entry():
+    from test_sequence_layer_b200 import build as b
+    dlib = ctypes.CDLL(b.build(debug=True))
+    names = declared_functions(debug=True)
+    assert "mesa_debug_skip_commit" in names
+    for n in names:
+        assert hasattr(dlib, n), n
+    dlib.mesa_debug_skip_commit.argtypes = [ctypes.c_int]
+    assert dlib.mesa_debug_skip_commit(-1) == 1                 # MESA_ERR_INVALID_ARG, no device call
 
 
 def test_status_strings(lib):
