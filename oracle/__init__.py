@@ -53,8 +53,9 @@ def _configure(lib):
     lib.oracle_forward_chunked.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, i, d, D, D, D, I32, D, D]
     lib.oracle_step.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, i, d, D, I32]
     lib.oracle_cg_dense.argtypes = [i, D, D, i, d, D, I32]
+    lib.oracle_preprocess.argtypes = [D, D, i, i, i, i, i, D]
     for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
-              lib.oracle_step, lib.oracle_cg_dense):
+              lib.oracle_step, lib.oracle_cg_dense, lib.oracle_preprocess):
         f.restype = ctypes.c_int
     return lib
 
@@ -63,19 +64,7 @@ def _load():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(_LIB_PATH)
-        D = ctypes.POINTER(ctypes.c_double)
-        I32 = ctypes.POINTER(ctypes.c_int32)
-        i, d = ctypes.c_int, ctypes.c_double
-        lib.oracle_forward_cg.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, I32, D, D]
-        lib.oracle_forward_cholesky.argtypes = [D, D, D, D, D, D, i, i, i, i, i, D, D, D, D, D]
-        lib.oracle_forward_chunked.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, i, d, D, D, D, I32, D, D]
-        lib.oracle_step.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, i, d, D, I32]
-        lib.oracle_cg_dense.argtypes = [i, D, D, i, d, D, I32]
-        for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
-                  lib.oracle_step, lib.oracle_cg_dense):
-            f.restype = ctypes.c_int
-        _lib = lib
+        _lib = _configure(ctypes.CDLL(_LIB_PATH))
     return _lib
 
 
@@ -178,3 +167,15 @@ def cg_dense(A, b, cg_steps, tol=0.0):
     rc = _load().oracle_cg_dense(n, _ptr(A), _ptr(b), int(cg_steps), float(tol), _ptr(x), _ptr(it))
     _check(rc, "oracle_cg_dense")
     return x, int(it[0])
+
+
+def preprocess(x, conv):
+    """Causal depthwise convolution over time, then per-token L2 normalisation.
+    x: [B,H,T,d]; conv: [H,W,d] (w = lag). Returns y [B,H,T,d]."""
+    x, conv = _f64(x), _f64(conv)
+    B, H, T, dd = x.shape
+    W = conv.shape[1]
+    y = np.zeros((B, H, T, dd))
+    rc = _load().oracle_preprocess(_ptr(x), _ptr(conv), B, H, T, dd, W, _ptr(y))
+    _check(rc, "oracle_preprocess")
+    return y

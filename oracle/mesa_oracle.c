@@ -366,6 +366,36 @@ int oracle_forward_chunked(const double* q, const double* k, const double* v,
 /* One decode step: O(1) per token on explicit state                          */
 /* ------------------------------------------------------------------------ */
 
+/* ------------------------------------------------------------------------ */
+/* Input preprocessing (MesaNet page, Architecture, "Preprocessing"): a causal */
+/* depthwise convolution over time, then L2 normalisation per token.          */
+/* ------------------------------------------------------------------------ */
+
+int oracle_preprocess(const double* x, const double* conv, int B, int H, int T, int d, int W, double* y) {
+    if (bad_dims(B, H, T, d, d) || W < 1 || !x || !conv || !y) return -1;
+    const int BH = B * H;
+#pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < BH; ++bh) {
+        const int h = bh % H;
+        const double* xs = x + (size_t)bh * T * d;
+        double* ys = y + (size_t)bh * T * d;
+        for (int t = 0; t < T; ++t) {
+            double nn = 0.0;
+            for (int i = 0; i < d; ++i) {
+                double u = 0.0;
+                for (int w = 0; w < W && w <= t; ++w)
+                    u += conv[((size_t)h * W + w) * d + i] * xs[(size_t)(t - w) * d + i];
+                ys[(size_t)t * d + i] = u;
+                nn += u * u;
+            }
+            const double nrm = sqrt(nn);
+            const double inv = 1.0 / (nrm > 1e-6 ? nrm : 1e-6);
+            for (int i = 0; i < d; ++i) ys[(size_t)t * d + i] *= inv;
+        }
+    }
+    return 0;
+}
+
 int oracle_step(const double* q, const double* k, const double* v,
                 const double* gamma, const double* beta, const double* lambda,
                 int B, int H, int dk, int dv, double* Hstate, double* Gstate,

@@ -55,6 +55,15 @@ int oracle_step(const double* q, const double* k, const double* v,
                 int B, int H, int dk, int dv, double* Hstate, double* Gstate,
                 int cg_steps, double tol, double* out, int32_t* iters);
 
+/* Input preprocessing of queries or keys (MesaNet page, Architecture,
+ * "Preprocessing": keys and queries are normalised, with a short-window
+ * convolution before the Mesa layer). Read as: a causal depthwise convolution
+ * over time, then L2 normalisation of every token:
+ *   u_t[i] = sum_{w=0..W-1} conv[h][w][i] * x[b][h][t-w][i]   (x = 0 before t = 0)
+ *   y_t    = u_t / max(|u_t|_2, 1e-6)
+ * x, y [B, H, T, d]; conv [H, W, d] (w = lag in tokens). */
+int oracle_preprocess(const double* x, const double* conv, int B, int H, int T, int d, int W, double* y);
+
 /* Dense CG on one SPD system A x = b (A n-by-n row-major), same rule as above.
  * Exposed so tests can pin the CG rule on its own. */
 int oracle_cg_dense(int n, const double* A, const double* b, int cg_steps, double tol,

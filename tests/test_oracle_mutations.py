@@ -34,6 +34,13 @@ MUTANTS = {
                                               "for (int m = i + 1; m < n; ++m) s -= A[(size_t)i * n + m] * x[m];"),
     "Lambda applied twice": ("A[(size_t)i * dk + i] += lambda[(size_t)h * dk + i];",
                              "A[(size_t)i * dk + i] += 2.0 * lambda[(size_t)h * dk + i];"),
+    "preprocessing convolution looks ahead": (
+        "for (int w = 0; w < W && w <= t; ++w)\n                    u += conv[((size_t)h * W + w) * d + i] * xs[(size_t)(t - w) * d + i];",
+        "for (int w = 0; w < W && t + w < T; ++w)\n                    u += conv[((size_t)h * W + w) * d + i] * xs[(size_t)(t + w) * d + i];"),
+    "preprocessing weights read with the lag reversed": (
+        "u += conv[((size_t)h * W + w) * d + i] * xs[(size_t)(t - w) * d + i];",
+        "u += conv[((size_t)h * W + (W - 1 - w)) * d + i] * xs[(size_t)(t - w) * d + i];"),
+    "preprocessing norm left out": ("const double inv = 1.0 / (nrm > 1e-6 ? nrm : 1e-6);", "const double inv = 1.0;"),
 }
 
 
@@ -78,6 +85,8 @@ PIN_SUBSET = [
     lambda o: pins.test_unconverged_cg_equals_galerkin_on_explicit_statistics(o),
     lambda o: pins.test_chunked_equals_per_token(o, 8, 0.0),
     lambda o: pins.test_large_lambda_gives_linear_attention(o),
+    lambda o: pins.test_preprocess_matches_numpy_convolution(o),
+    lambda o: pins.test_preprocess_causal_and_scale_invariant(o),
 ]
 
 

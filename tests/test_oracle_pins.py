@@ -331,3 +331,54 @@ def test_empty_sequence(oracle_mod):
     out, it, Hf, Gf = oracle_mod.forward_cg(z, z, z, np.zeros((1, 1, 0)), np.zeros((1, 1, 0)),
                                             np.ones((1, 4)), 3)
     assert out.shape == (1, 1, 0, 4) and np.all(Hf == 0) and np.all(Gf == 0)
+
+
+# ---------------------------------------------------------------------------
+# Input preprocessing (MesaNet page, Architecture, "Preprocessing"): causal
+# depthwise convolution over time, then L2 normalisation per token.
+# ---------------------------------------------------------------------------
+
+def test_preprocess_matches_numpy_convolution(oracle_mod):
+    rng = np.random.default_rng(11)
+    B, H, T, d, W = 2, 3, 19, 8, 4
+    x = rng.standard_normal((B, H, T, d))
+    conv = rng.standard_normal((H, W, d))
+    y = oracle_mod.preprocess(x, conv)
+    for b in range(B):
+        for h in range(H):
+            u = np.stack([np.convolve(x[b, h, :, i], conv[h, :, i])[:T] for i in range(d)], axis=1)
+            ref = u / np.maximum(np.linalg.norm(u, axis=1, keepdims=True), 1e-6)
+            assert np.allclose(y[b, h], ref, rtol=0, atol=1e-13)
+
+
+def test_preprocess_window_one_is_normalisation(oracle_mod):
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((1, 2, 7, 16))
+    y = oracle_mod.preprocess(x, np.ones((2, 1, 16)))
+    assert np.allclose(np.linalg.norm(y, axis=-1), 1.0, atol=1e-14)
+    cos = (y * x).sum(-1) / np.linalg.norm(x, axis=-1)
+    assert np.allclose(cos, 1.0, atol=1e-14)
+
+
+def test_preprocess_delta_filter_shifts(oracle_mod):
+    rng = np.random.default_rng(13)
+    T, d, s = 9, 8, 2
+    x = rng.standard_normal((1, 1, T, d))
+    conv = np.zeros((1, 4, d))
+    conv[0, s] = 1.0
+    y = oracle_mod.preprocess(x, conv)
+    assert np.all(y[0, 0, :s] == 0.0)                          # nothing before the sequence start
+    ref = x[0, 0, :T - s] / np.linalg.norm(x[0, 0, :T - s], axis=-1, keepdims=True)
+    assert np.allclose(y[0, 0, s:], ref, atol=1e-14)
+
+
+def test_preprocess_causal_and_scale_invariant(oracle_mod):
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((1, 2, 12, 8))
+    conv = rng.standard_normal((2, 3, 8))
+    y = oracle_mod.preprocess(x, conv)
+    x2 = x.copy()
+    x2[:, :, 7:] = rng.standard_normal(x2[:, :, 7:].shape)     # change the future
+    assert np.array_equal(oracle_mod.preprocess(x2, conv)[:, :, :7], y[:, :, :7])
+    assert np.allclose(oracle_mod.preprocess(3.5 * x, conv), y, atol=1e-14)
+    assert np.allclose(oracle_mod.preprocess(-x, conv), -y, atol=1e-14)
