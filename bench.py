@@ -199,6 +199,7 @@ def run_reference(args, w, rank):
 
 METRIC = "Mesa-layer fwd tokens/s (B*H*T) at T=8192,d=128,15 CG steps; % tensor peak"
 DECODE_METRIC = "Mesa decode tokens/s (sequences x heads per mesa_step), d=128, 15 CG steps; % HBM peak"
+PRE_METRIC = "Mesa input preprocessing tokens/s (q and k: causal depthwise conv, window 4, + L2 norm); % HBM peak"
 
 
 def run_decode(args, w, world, rank, local):
@@ -304,6 +305,81 @@ def run_decode(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_preprocess(args, w, world, rank, local):
+    """mesa_preprocess alone on the workload's shape: causal depthwise
+    convolution (window 4) and per-token L2 normalisation of q and k."""
+    import torch
+    import torch.distributed as dist
+    from test_sequence_layer_b200 import build as mbuild, mesa
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    B, H, T, d, W = w.B, w.H, w.T, w.dk, 4
+    g = torch.Generator(device=dev).manual_seed(5 + rank)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q_raw = torch.randn((B, H, T, d), generator=g, device=dev).to(dt)
+    k_raw = torch.randn((B, H, T, d), generator=g, device=dev).to(dt)
+    cq = torch.randn((H, W, d), generator=g, device=dev) / 2
+    ck = torch.randn((H, W, d), generator=g, device=dev) / 2
+    q_out, k_out = torch.empty_like(q_raw), torch.empty_like(k_raw)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mesa.preprocess(q_raw, k_raw, cq, ck, q_out=q_out, k_out=k_out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    mesa.timing_enable(False)
+    kernels = mesa.timing_read()
+    clk = clocks.stop()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    tokens = B * H * T
+    launches, kms = kernels["preprocess"]
+    avg_ms = kms / launches
+    bytes_per_launch = 2 * 2 * tokens * d * q_raw.element_size()      # q and k, read and written
+    peaks = load_peaks()
+    achieved = bytes_per_launch / (avg_ms / 1e3) / 1e9
+    line = {
+        "metric": PRE_METRIC, "value": whole_job_rate(tokens, world, ms / args.steps), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-in/f32/bf16-out" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name + "+preprocess", "B": B, "H": H, "T": T, "d": d, "window": W,
+                   "l2": "inputs larger than L2 (%.2f GB per step)" % (2 * q_raw.numel() * q_raw.element_size() / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic("preprocess", tokens),
+                     "kernel": "preprocess", "avg_ms": avg_ms,
+                     "peak_kind": f"{peaks['_source']} HBM copy bandwidth"},
+        "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
+        "gpu_launches": sum(v[0] for v in kernels.values()),
+        "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -313,6 +389,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--preprocess", action="store_true",
+                    help="time mesa_preprocess (q/k convolution + normalisation) on the workload's shape")
     ap.add_argument("--decode-state", default="prefill", choices=["prefill", "random"],
                     help="decode: state from a mesa_forward prefill (default) or a seeded random stand-in")
     args = ap.parse_args()
@@ -326,6 +404,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, rank)
+        return
+    if args.preprocess:
+        run_preprocess(args, w, world, rank, local)
         return
     if w.decode_steps > 0:
         run_decode(args, w, world, rank, local)

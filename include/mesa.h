@@ -150,6 +150,27 @@ mesa_status mesa_forward_noalloc(const void* q, const void* k, const void* v,
                                  float* H_out, float* G_out, void* stream);
 
 /*
+ * Input preprocessing of queries and keys, the layer's own input path
+ * ("MesaNet" page, Technical summary > Architecture > "Preprocessing": keys
+ * and queries are normalised, with a short-window convolution before the
+ * Mesa layer; read as the convolution first, then the normalisation, so that
+ * the layer receives unit-norm keys and queries). For every (b, h, t) and
+ * channel i, separately for q and k with their own weights:
+ *     u_t[i] = sum_{w=0..W-1} conv[h][w][i] * x_{t-w}[i]   (x = 0 before t = 0)
+ *     y_t    = u_t / max(|u_t|_2, 1e-6)
+ * q_raw, k_raw, q_out, k_out: [B,H,T,d] in `dtype` (MESA_BF16 rounds the
+ * outputs to bf16, nearest-even; the arithmetic is fp32). conv_q, conv_k:
+ * [H,W,d] fp32, w = lag in tokens (w = 0 multiplies the current token).
+ * 1 <= W <= 4; d in {16, 32, 64, 128}; B*H <= 65535. The outputs are ready
+ * to pass to mesa_forward as q and k. Outputs must not overlap the inputs or
+ * each other (MESA_ERR_INVALID_ARG). Pointers are DEVICE pointers, 16-byte
+ * aligned (conv 4-byte aligned). Asynchronous on `stream`; T = 0 is a no-op.
+ */
+mesa_status mesa_preprocess(const void* q_raw, const void* k_raw, const float* conv_q, const float* conv_k,
+                            int B, int H, int T, int d, int W, mesa_dtype dtype, void* q_out, void* k_out,
+                            void* stream);
+
+/*
  * Bytes of device workspace mesa_forward_host needs: the mesa_forward
  * workspace plus device staging for every tensor argument.
  */

@@ -68,7 +68,8 @@ mesa_status launch_forward(const ForwardArgs& a, cudaStream_t st) {
 }
 
 // ---- kernel timing records ----
-const char* const kKindNames[kKindCount] = {"simt_scan", "simt_cg", "decode_step", "tc_scan", "tc_cg"};
+const char* const kKindNames[kKindCount] = {"simt_scan", "simt_cg", "decode_step", "tc_scan", "tc_cg",
+                                             "preprocess"};
 struct TimingRec {
     int kind;
     cudaEvent_t start, stop;
@@ -358,6 +359,32 @@ mesa_status mesa_step(const float* q, const float* k, const float* v,
     if (Hstate == Gstate) return MESA_ERR_INVALID_ARG;
     StepArgs a{q, k, v, gamma, beta, lambda, B, H, dk, dv, Hstate, Gstate, cg_steps, tol, out, iters_out};
     return step_launch(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+mesa_status mesa_preprocess(const void* q_raw, const void* k_raw, const float* conv_q, const float* conv_k,
+                            int B, int H, int T, int d, int W, mesa_dtype dtype, void* q_out, void* k_out,
+                            void* stream) {
+    if (B < 1 || H < 1 || T < 0 || W < 1 || W > 4) return MESA_ERR_INVALID_ARG;
+    if (dtype != MESA_F32 && dtype != MESA_BF16) return MESA_ERR_INVALID_ARG;
+    if (!supported_width(d)) return MESA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 65535) return MESA_ERR_UNSUPPORTED;                 // grid.y limit
+    if (T == 0) return MESA_OK;
+    if (!q_raw || !k_raw || !conv_q || !conv_k || !q_out || !k_out) return MESA_ERR_INVALID_ARG;
+    for (const void* p : {q_raw, k_raw, (const void*)q_out, (const void*)k_out})
+        if (!aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    if (!aligned(conv_q, 4) || !aligned(conv_k, 4)) return MESA_ERR_INVALID_ARG;
+    // outputs must not overlap the inputs: rows are read by the warp after their own
+    const size_t bytes = (size_t)B * H * T * d * elem_size(dtype);
+    auto overlap = [bytes](const void* a, const void* b) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        return x < y + bytes && y < x + bytes;
+    };
+    if (overlap(q_out, q_raw) || overlap(q_out, k_raw) || overlap(k_out, q_raw) || overlap(k_out, k_raw) ||
+        overlap(q_out, k_out))
+        return MESA_ERR_INVALID_ARG;
+    PreArgs a{q_raw, k_raw, conv_q, conv_k, B, H, T, d, W, dtype, q_out, k_out};
+    return preprocess_launch(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
 }
 
 mesa_status mesa_timing_enable(int on) {

@@ -35,7 +35,7 @@ struct ForwardArgs {
 unsigned* error_word_ptr();
 
 // Kernel kinds for the optional timing records (mesa_timing_enable).
-enum KernelKind : int { kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindCount };
+enum KernelKind : int { kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindPre, kKindCount };
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
 class LaunchTimer {
@@ -81,5 +81,18 @@ struct StepArgs {
     int32_t* iters;
 };
 cudaError_t step_launch(const StepArgs& a, cudaStream_t st);
+
+// Input preprocessing (preprocess.cu).
+struct PreArgs {
+    const void* xq;
+    const void* xk;
+    const float* conv_q;
+    const float* conv_k;
+    int B, H, T, d, W;
+    mesa_dtype dtype;
+    void* yq;
+    void* yk;
+};
+cudaError_t preprocess_launch(const PreArgs& a, cudaStream_t st);
 
 }  // namespace mesa

@@ -61,6 +61,8 @@ def _load():
     lib.mesa_timing_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(I),
                                      ctypes.POINTER(ctypes.c_double), I]
     lib.mesa_timing_read.restype = I
+    lib.mesa_preprocess.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.mesa_preprocess.restype = I
     _lib = lib
     return lib
 
@@ -158,6 +160,27 @@ def forward_host(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, o
                                _ptr(workspace), ws_bytes, _stream(stream, device))
     _check(rc, "mesa_forward_host")
     return out
+
+
+def preprocess(q_raw, k_raw, conv_q, conv_k, *, q_out=None, k_out=None, stream=None):
+    """mesa_preprocess: causal depthwise convolution over time (conv [H,W,d],
+    w = lag), then per-token L2 normalisation, for q and k. q_raw, k_raw:
+    [B,H,T,d] float32 or bfloat16 CUDA tensors. Returns (q, k) in the same
+    dtype, ready for forward()."""
+    lib = _load()
+    B, H, T, d = q_raw.shape
+    W = conv_q.shape[1]
+    assert k_raw.shape == q_raw.shape and k_raw.dtype == q_raw.dtype
+    assert conv_q.shape == (H, W, d) and conv_k.shape == (H, W, d)
+    assert conv_q.dtype == torch.float32 and conv_k.dtype == torch.float32
+    for t in (q_raw, k_raw, conv_q, conv_k):
+        assert t.is_cuda and t.is_contiguous()
+    q_out = torch.empty_like(q_raw) if q_out is None else q_out
+    k_out = torch.empty_like(k_raw) if k_out is None else k_out
+    rc = lib.mesa_preprocess(_ptr(q_raw), _ptr(k_raw), _ptr(conv_q), _ptr(conv_k), B, H, T, d, W,
+                             _dtype_code(q_raw), _ptr(q_out), _ptr(k_out), _stream(stream, q_raw.device))
+    _check(rc, "mesa_preprocess")
+    return q_out, k_out
 
 
 def step(q, k, v, gamma, beta, lam, Hstate, Gstate, *, cg_steps=15, tol=0.0, out=None,

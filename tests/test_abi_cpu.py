@@ -133,3 +133,17 @@ def test_product_does_not_import_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "oracle" not in src.lower().replace("oracles", ""), fn
+
+
+def test_preprocess_argument_errors(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.mesa_preprocess.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, P]
+    a, b_, c, o1, o2 = (ctypes.c_void_p(0x10000 * i) for i in (1, 3, 5, 7, 9))
+    call = lambda W=4, d=128, T=8, dt=1, q=a, o=o1: lib.mesa_preprocess(q, b_, c, c, 1, 1, T, d, W, dt, o, o2, None)  # noqa: E731
+    assert call(W=0) == 1 and call(W=5) == 1                    # window out of range
+    assert call(d=48) == 2                                      # unsupported width
+    assert call(dt=7) == 1                                      # bad dtype
+    assert call(T=0, q=None) == 0                               # nothing to do, no pointer needed
+    assert call(q=None) == 1                                    # null input
+    assert call(q=ctypes.c_void_p(0x10008)) == 1                # misaligned
+    assert call(o=a) == 1                                       # output overlaps input
