@@ -48,13 +48,16 @@ def load_peaks():
 
 
 # DRAM bytes moved per token (per head for the decode step) by each kernel, from
-# one ncu capture (profiles/tc_kernels_bf16_T2048.md, profiles/decode_step_4096heads.md:
+# one ncu capture (profiles/tc_kernels_bf16_T2048.md, profiles/decode_step_4096heads.md,
+# profiles/preprocess_bf16_T8192.md:
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch / units of that launch).
 # Reported only while the kernel source still hashes to the captured version;
 # otherwise the field is null.
 MEASURED_TRAFFIC = {
     "tc_cg": {"src_sha16": "c37d4ab6e10641c0", "bytes_per_token": (337.729280e6 + 108.120320e6) / 262144},
     "tc_scan": {"src_sha16": "c37d4ab6e10641c0", "bytes_per_token": (136.442624e6 + 92.728576e6) / 262144},
+    "preprocess": {"src_sha16": "084d9e828774199c", "files": ("preprocess.cu",),
+                   "bytes_per_token": (537.019904e6 + 489.792512e6) / 1048576},
     "decode_step": {"src_sha16": "6f15ddc891a713b8", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
 }
 
