@@ -52,10 +52,11 @@ def _configure(lib):
     lib.oracle_forward_cholesky.argtypes = [D, D, D, D, D, D, i, i, i, i, i, D, D, D, D, D]
     lib.oracle_forward_chunked.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, i, d, D, D, D, I32, D, D]
     lib.oracle_step.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, i, d, D, I32]
-    lib.oracle_cg_dense.argtypes = [i, D, D, i, d, D, I32]
+    lib.oracle_step_warm.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, D, i, d, D, I32]
+    lib.oracle_cg_dense.argtypes = [i, D, D, D, i, d, D, I32]
     lib.oracle_preprocess.argtypes = [D, D, i, i, i, i, i, D]
     for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
-              lib.oracle_step, lib.oracle_cg_dense, lib.oracle_preprocess):
+              lib.oracle_step, lib.oracle_step_warm, lib.oracle_cg_dense, lib.oracle_preprocess):
         f.restype = ctypes.c_int
     return lib
 
@@ -141,30 +142,32 @@ def forward_chunked(q, k, v, gamma, beta, lam, chunk, cg_steps, tol=0.0, H0=None
     return out, iters, Hf, Gf
 
 
-def step(q, k, v, gamma, beta, lam, Hstate, Gstate, cg_steps, tol=0.0):
+def step(q, k, v, gamma, beta, lam, Hstate, Gstate, cg_steps, tol=0.0, x_state=None):
     """One decode step. q,k,v: [B,H,d]; gamma,beta: [B,H]. States are copied
-    (not modified). Returns (out, iters, H_new, G_new)."""
+    (not modified). x_state [B,H,dk] (optional): CG starts from it (warm start).
+    Returns (out, iters, H_new, G_new), plus x_new when x_state is given."""
     q, k, v, gamma, beta, lam = map(_f64, (q, k, v, gamma, beta, lam))
     Hs = _f64(Hstate).copy()
     Gs = _f64(Gstate).copy()
+    xs = None if x_state is None else _f64(x_state).copy()
     B, H, dk = q.shape
     dv = v.shape[-1]
     out = np.zeros((B, H, dv))
     iters = np.zeros((B, H), dtype=np.int32)
-    rc = _load().oracle_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
-                             B, H, dk, dv, _ptr(Hs), _ptr(Gs), int(cg_steps), float(tol),
-                             _ptr(out), _ptr(iters))
-    _check(rc, "oracle_step")
-    return out, iters, Hs, Gs
+    rc = _load().oracle_step_warm(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                  B, H, dk, dv, _ptr(Hs), _ptr(Gs), _ptr(xs), int(cg_steps), float(tol),
+                                  _ptr(out), _ptr(iters))
+    _check(rc, "oracle_step_warm")
+    return (out, iters, Hs, Gs) if xs is None else (out, iters, Hs, Gs, xs)
 
 
-def cg_dense(A, b, cg_steps, tol=0.0):
-    """CG on one dense SPD system. Returns (x, iters)."""
-    A, b = _f64(A), _f64(b)
+def cg_dense(A, b, cg_steps, tol=0.0, x0=None):
+    """CG on one dense SPD system, from x0 (default zero). Returns (x, iters)."""
+    A, b, x0 = _f64(A), _f64(b), _f64(x0)
     n = b.shape[0]
     x = np.zeros(n)
     it = np.zeros(1, dtype=np.int32)
-    rc = _load().oracle_cg_dense(n, _ptr(A), _ptr(b), int(cg_steps), float(tol), _ptr(x), _ptr(it))
+    rc = _load().oracle_cg_dense(n, _ptr(A), _ptr(b), _ptr(x0), int(cg_steps), float(tol), _ptr(x), _ptr(it))
     _check(rc, "oracle_cg_dense")
     return x, int(it[0])
 

@@ -67,15 +67,24 @@ static double dot(int n, const double* a, const double* b) {
     return s;
 }
 
-/* Solves A x = b by CG, A given only through mv. work: 3n doubles. */
-static int cg_generic(int n, matvec_fn mv, const void* ctx, const double* b,
-                      int cg_steps, double tol, double* x, double* work) {
+/* Solves A x = b by CG, A given only through mv, starting from x0 (NULL:
+ * x0 = 0). The first residual is r0 = b - A x0 and the first direction
+ * p0 = r0; the stopping test compares |r_k| with tol |b| whatever the start.
+ * work: 3n doubles. */
+static int cg_generic_x0(int n, matvec_fn mv, const void* ctx, const double* b, const double* x0,
+                         int cg_steps, double tol, double* x, double* work) {
     double* r = work;
     double* p = work + n;
     double* y = work + 2 * n;
-    for (int i = 0; i < n; ++i) { x[i] = 0.0; r[i] = b[i]; p[i] = b[i]; }
+    if (x0) {
+        for (int i = 0; i < n; ++i) x[i] = x0[i];
+        mv(ctx, x, y);
+        for (int i = 0; i < n; ++i) { r[i] = b[i] - y[i]; p[i] = r[i]; }
+    } else {
+        for (int i = 0; i < n; ++i) { x[i] = 0.0; r[i] = b[i]; p[i] = b[i]; }
+    }
     double rr = dot(n, r, r);
-    const double bnorm = sqrt(rr);
+    const double bnorm = sqrt(dot(n, b, b));
     int it = 0;
     for (int kstep = 0; kstep < cg_steps; ++kstep) {
         if (tol > 0.0 && sqrt(rr) <= tol * bnorm) break;   /* stopping criterion */
@@ -93,6 +102,11 @@ static int cg_generic(int n, matvec_fn mv, const void* ctx, const double* b,
     return it;
 }
 
+static int cg_generic(int n, matvec_fn mv, const void* ctx, const double* b,
+                      int cg_steps, double tol, double* x, double* work) {
+    return cg_generic_x0(n, mv, ctx, b, NULL, cg_steps, tol, x, work);
+}
+
 /* Dense (H + Lambda) p: the matrix is formed explicitly. */
 typedef struct { int n; const double* A; } dense_ctx;
 
@@ -101,13 +115,13 @@ static void dense_mv(const void* vctx, const double* p, double* y) {
     for (int i = 0; i < c->n; ++i) y[i] = dot(c->n, c->A + (size_t)i * c->n, p);
 }
 
-int oracle_cg_dense(int n, const double* A, const double* b, int cg_steps, double tol,
+int oracle_cg_dense(int n, const double* A, const double* b, const double* x0, int cg_steps, double tol,
                     double* x, int32_t* iters) {
     if (n <= 0 || !A || !b || !x || cg_steps < 0) return -1;
     double* work = (double*)malloc(sizeof(double) * 3 * (size_t)n);
     if (!work) return -2;
     dense_ctx c = {n, A};
-    int it = cg_generic(n, dense_mv, &c, b, cg_steps, tol, x, work);
+    int it = cg_generic_x0(n, dense_mv, &c, b, x0, cg_steps, tol, x, work);
     if (iters) *iters = it;
     free(work);
     return 0;
@@ -400,6 +414,18 @@ int oracle_step(const double* q, const double* k, const double* v,
                 const double* gamma, const double* beta, const double* lambda,
                 int B, int H, int dk, int dv, double* Hstate, double* Gstate,
                 int cg_steps, double tol, double* out, int32_t* iters) {
+    return oracle_step_warm(q, k, v, gamma, beta, lambda, B, H, dk, dv, Hstate, Gstate, NULL, cg_steps, tol,
+                            out, iters);
+}
+
+/* One decode step whose CG starts from x_state (MesaNet page, Significance and
+ * claims: warm starts named as the way to cut the solver's cost). x_state
+ * [B, H, dk] holds the starting guess on entry and the solution on exit;
+ * NULL starts from zero. */
+int oracle_step_warm(const double* q, const double* k, const double* v,
+                     const double* gamma, const double* beta, const double* lambda,
+                     int B, int H, int dk, int dv, double* Hstate, double* Gstate, double* x_state,
+                     int cg_steps, double tol, double* out, int32_t* iters) {
     if (bad_dims(B, H, 1, dk, dv) || cg_steps < 0) return -1;
     if (!q || !k || !v || !gamma || !beta || !lambda || !Hstate || !Gstate || !out) return -1;
     const int BH = B * H;
@@ -421,9 +447,12 @@ int oracle_step(const double* q, const double* k, const double* v,
                 A[(size_t)i * dk + i] += lambda[(size_t)h * dk + i];
             }
             dense_ctx c = {dk, A};
-            int it = cg_generic(dk, dense_mv, &c, q + (size_t)bh * dk, cg_steps, tol, x, work);
+            int it = cg_generic_x0(dk, dense_mv, &c, q + (size_t)bh * dk, x_state ? x_state + (size_t)bh * dk : NULL,
+                                   cg_steps, tol, x, work);
             if (iters) iters[bh] = it;
             for (int i = 0; i < dv; ++i) out[(size_t)bh * dv + i] = dot(dk, Gm + (size_t)i * dk, x);
+            if (x_state)
+                for (int i = 0; i < dk; ++i) x_state[(size_t)bh * dk + i] = x[i];
         }
         free(A); free(x); free(work);
     }

@@ -64,9 +64,17 @@ int oracle_step(const double* q, const double* k, const double* v,
  * x, y [B, H, T, d]; conv [H, W, d] (w = lag in tokens). */
 int oracle_preprocess(const double* x, const double* conv, int B, int H, int T, int d, int W, double* y);
 
-/* Dense CG on one SPD system A x = b (A n-by-n row-major), same rule as above.
- * Exposed so tests can pin the CG rule on its own. */
-int oracle_cg_dense(int n, const double* A, const double* b, int cg_steps, double tol,
+/* One decode step whose CG starts from x_state ([B, H, dk]: the starting
+ * guess on entry, the solution on exit; NULL starts from zero, which is
+ * oracle_step). The stopping test stays |r_k| <= tol |q|. */
+int oracle_step_warm(const double* q, const double* k, const double* v,
+                     const double* gamma, const double* beta, const double* lambda,
+                     int B, int H, int dk, int dv, double* Hstate, double* Gstate, double* x_state,
+                     int cg_steps, double tol, double* out, int32_t* iters);
+
+/* Dense CG on one SPD system A x = b (A n-by-n row-major), same rule as above,
+ * from x0 (NULL: zero). Exposed so tests can pin the CG rule on its own. */
+int oracle_cg_dense(int n, const double* A, const double* b, const double* x0, int cg_steps, double tol,
                     double* x, int32_t* iters);
 
 #ifdef __cplusplus

@@ -40,6 +40,12 @@ MUTANTS = {
     "preprocessing weights read with the lag reversed": (
         "u += conv[((size_t)h * W + w) * d + i] * xs[(size_t)(t - w) * d + i];",
         "u += conv[((size_t)h * W + (W - 1 - w)) * d + i] * xs[(size_t)(t - w) * d + i];"),
+    "warm start residual sign": ("for (int i = 0; i < n; ++i) { r[i] = b[i] - y[i]; p[i] = r[i]; }",
+                                 "for (int i = 0; i < n; ++i) { r[i] = b[i] + y[i]; p[i] = r[i]; }"),
+    "warm start drops x0 from x": ("for (int i = 0; i < n; ++i) x[i] = x0[i];\n        mv(ctx, x, y);",
+                                   "for (int i = 0; i < n; ++i) x[i] = x0[i];\n        mv(ctx, x, y);\n        for (int i = 0; i < n; ++i) x[i] = 0.0;"),
+    "warm stopping test relative to the first residual": ("const double bnorm = sqrt(dot(n, b, b));",
+                                                          "const double bnorm = sqrt(rr);"),
     "preprocessing norm left out": ("const double inv = 1.0 / (nrm > 1e-6 ? nrm : 1e-6);", "const double inv = 1.0;"),
 }
 
@@ -87,6 +93,8 @@ PIN_SUBSET = [
     lambda o: pins.test_large_lambda_gives_linear_attention(o),
     lambda o: pins.test_preprocess_matches_numpy_convolution(o),
     lambda o: pins.test_preprocess_causal_and_scale_invariant(o),
+    lambda o: pins.test_warm_cg_equals_shifted_cold_cg(o),
+    lambda o: pins.test_warm_cg_from_the_solution_stops_at_once(o),
 ]
 
 

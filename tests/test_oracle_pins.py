@@ -382,3 +382,65 @@ def test_preprocess_causal_and_scale_invariant(oracle_mod):
     assert np.array_equal(oracle_mod.preprocess(x2, conv)[:, :, :7], y[:, :, :7])
     assert np.allclose(oracle_mod.preprocess(3.5 * x, conv), y, atol=1e-14)
     assert np.allclose(oracle_mod.preprocess(-x, conv), -y, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Warm-started CG (MesaNet page, Significance and claims: warm starts named as
+# the way to cut the solver's cost). CG from x0 on A x = b is, in exact
+# arithmetic, x0 plus CG from zero on the residual system A e = b - A x0.
+# ---------------------------------------------------------------------------
+
+def _spd(rng, n):
+    M = rng.standard_normal((n, n))
+    return M @ M.T / n + 0.5 * np.eye(n)
+
+
+def test_warm_cg_equals_shifted_cold_cg(oracle_mod):
+    rng = np.random.default_rng(21)
+    n = 12
+    A, b, x0 = _spd(rng, n), rng.standard_normal(n), rng.standard_normal(n)
+    r0 = b - A @ x0
+    for k in range(1, n + 1):
+        xw, itw = oracle_mod.cg_dense(A, b, k, 0.0, x0=x0)
+        xc, itc = oracle_mod.cg_dense(A, r0, k, 0.0)
+        assert itw == itc == k
+        assert np.allclose(xw, x0 + xc, rtol=0, atol=1e-10), k
+
+
+def test_warm_cg_one_step_closed_form(oracle_mod):
+    rng = np.random.default_rng(22)
+    n = 7
+    A, b, x0 = _spd(rng, n), rng.standard_normal(n), rng.standard_normal(n)
+    r0 = b - A @ x0
+    x1, it = oracle_mod.cg_dense(A, b, 1, 0.0, x0=x0)
+    assert it == 1
+    assert np.allclose(x1, x0 + (r0 @ r0) / (r0 @ A @ r0) * r0, rtol=0, atol=1e-13)
+
+
+def test_warm_cg_from_the_solution_stops_at_once(oracle_mod):
+    rng = np.random.default_rng(23)
+    n = 9
+    A, b = _spd(rng, n), rng.standard_normal(n)
+    xs = np.linalg.solve(A, b)
+    x, it = oracle_mod.cg_dense(A, b, 20, 1e-6, x0=xs)
+    assert it == 0 and np.array_equal(x, xs)
+    # the stopping test is relative to |b|, not to the first residual
+    x, it = oracle_mod.cg_dense(A, b, 20, 1e-3, x0=xs + 1e-6 * rng.standard_normal(n))
+    assert it == 0
+
+
+def test_warm_step_from_zero_is_the_cold_step(oracle_mod):
+    w = mi.Workload("t", 2, 3, 6, 8, 8, 2, "f32", 5, 0.0, False, 24)
+    x = mi.batch(w)
+    rng = np.random.default_rng(24)
+    Hs = rng.standard_normal((2, 3, 8, 8)) * 0.1
+    Hs = Hs @ np.swapaxes(Hs, -1, -2)
+    Gs = rng.standard_normal((2, 3, 8, 8))
+    args = (x["q"][:, :, 0], x["k"][:, :, 0], x["v"][:, :, 0], x["gamma"][:, :, 0], x["beta"][:, :, 0], x["lam"],
+            Hs, Gs, 5)
+    cold = oracle_mod.step(*args)
+    warm = oracle_mod.step(*args, x_state=np.zeros((2, 3, 8)))
+    for a, b_ in zip(cold, warm[:4]):
+        assert np.array_equal(a, b_)
+    # the returned x reproduces the output through the updated G
+    assert np.allclose(np.einsum("bhij,bhj->bhi", warm[3], warm[4]), warm[0], atol=1e-12)
