@@ -58,7 +58,7 @@ MEASURED_TRAFFIC = {
     "tc_scan": {"src_sha16": "c37d4ab6e10641c0", "bytes_per_token": (136.442624e6 + 92.728576e6) / 262144},
     "preprocess": {"src_sha16": "084d9e828774199c", "files": ("preprocess.cu",),
                    "bytes_per_token": (537.019904e6 + 489.792512e6) / 1048576},
-    "decode_step": {"src_sha16": "6f15ddc891a713b8", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
+    "decode_step": {"src_sha16": "2d83b99e92f2442f", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
 }
 
 
@@ -249,12 +249,23 @@ def run_decode(args, w, world, rank, local):
     # one contiguous [steps, B, H, ...] block per input, resident before timing
     tok = {n: dec[n].movedim(2, 0).contiguous() for n in dec}
     del dec
+    if args.query_walk > 0:
+        # correlated query stream (stand-in for consecutive queries of a language model):
+        # q_s = normalise(q_{s-1} + sigma * eps_s), eps seeded
+        gq = torch.Generator(device=dev).manual_seed(91 + rank)
+        qw = tok["q"]
+        for s_ in range(1, qw.shape[0]):
+            nxt = qw[s_ - 1] + args.query_walk * torch.randn(qw[s_].shape, generator=gq, device=dev)
+            qw[s_] = nxt / nxt.norm(dim=-1, keepdim=True)
+    tol = w.tol if args.tol is None else args.tol
+    xs = torch.zeros((B, H, d), device=dev) if args.warm_start else None
+    its = torch.zeros((steps_total, B, H), dtype=torch.int32, device=dev)
     lam = torch.from_numpy(mi.lambdas(w.seed, w.H, w.dk)).to(dev)
     out = torch.empty((B, H, d), device=dev)
     stream = torch.cuda.current_stream(dev)
     for s in range(args.warmup):
         mesa.step(tok["q"][s], tok["k"][s], tok["v"][s], tok["gamma"][s], tok["beta"][s], lam, Hs, Gs,
-                  cg_steps=w.cg_steps, out=out, stream=stream)
+                  cg_steps=w.cg_steps, tol=tol, out=out, iters=its[s], x_state=xs, stream=stream)
     torch.cuda.synchronize()
     assert mesa.get_error(stream) == 0
     clocks = ClockSampler(local)
@@ -269,7 +280,7 @@ def run_decode(args, w, world, rank, local):
     ev0.record(stream)
     for s in range(args.warmup, steps_total):
         mesa.step(tok["q"][s], tok["k"][s], tok["v"][s], tok["gamma"][s], tok["beta"][s], lam, Hs, Gs,
-                  cg_steps=w.cg_steps, out=out, stream=stream)
+                  cg_steps=w.cg_steps, tol=tol, out=out, iters=its[s], x_state=xs, stream=stream)
     ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -295,7 +306,9 @@ def run_decode(args, w, world, rank, local):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "sequences": B, "H": H, "d": d, "prefill_tokens": w.T,
-                   "cg_steps": w.cg_steps, "state": args.decode_state,
+                   "cg_steps": w.cg_steps, "tol": tol, "warm_start": bool(args.warm_start),
+                   "query_walk": args.query_walk,
+                   "mean_cg_iters": float(its[args.warmup:].float().mean().item()), "state": args.decode_state,
                    "l2": "state larger than L2 (%.2f GB)" % (2 * Hs.numel() * 4 / 1e9)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic("decode_step", heads),
@@ -394,6 +407,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--preprocess", action="store_true",
                     help="time mesa_preprocess (q/k convolution + normalisation) on the workload's shape")
+    ap.add_argument("--warm-start", action="store_true",
+                    help="decode: start each step's CG from the previous step's solution (mesa_step_warm)")
+    ap.add_argument("--tol", type=float, default=None, help="override the workload's CG tolerance")
+    ap.add_argument("--query-walk", type=float, default=0.0,
+                    help="decode: queries as a random walk on the sphere with this step size (correlated stream)")
     ap.add_argument("--decode-state", default="prefill", choices=["prefill", "random"],
                     help="decode: state from a mesa_forward prefill (default) or a seeded random stand-in")
     args = ap.parse_args()

@@ -225,6 +225,25 @@ mesa_status mesa_step(const float* q, const float* k, const float* v,
                       float* out, int32_t* iters_out, void* stream);
 
 /*
+ * mesa_step with a warm-started solve: the CG of each head starts from the
+ * guess in x_state instead of zero (the pages name warm starts as the way to
+ * cut the solver's cost: "MesaNet" page, Significance and claims). x_state
+ * [B,H,dk] fp32 DEVICE buffer, in/out: on entry the starting guess x0 (for
+ * example the previous step's solution; zeros make this call mesa_step), on
+ * exit this step's solution x. The CG rule is mesa_step's with r0 = q -
+ * (H + Lambda) x0 and p0 = r0; the stopping test stays |r_k| <= tol |q|, so a
+ * good guess stops after fewer updates (iters counts the updates applied).
+ * x_state may be NULL (cold start); it must not alias q or out. Other
+ * arguments, errors and the state update are those of mesa_step.
+ */
+mesa_status mesa_step_warm(const float* q, const float* k, const float* v,
+                           const float* gamma, const float* beta, const float* lambda,
+                           int B, int H, int dk, int dv,
+                           float* Hstate, float* Gstate, float* x_state,
+                           int cg_steps, float tol,
+                           float* out, int32_t* iters_out, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the calling device's error
  * word. Returns MESA_OK if no kernel recorded an error since the last call,
  * MESA_ERR_DEVICE_TIMEOUT if one gave up a bounded wait, MESA_ERR_CUDA if the

@@ -340,12 +340,12 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
     return ok && synced ? MESA_OK : MESA_ERR_CUDA;
 }
 
-mesa_status mesa_step(const float* q, const float* k, const float* v,
-                      const float* gamma, const float* beta, const float* lambda,
-                      int B, int H, int dk, int dv,
-                      float* Hstate, float* Gstate,
-                      int cg_steps, float tol,
-                      float* out, int32_t* iters_out, void* stream) {
+mesa_status mesa_step_warm(const float* q, const float* k, const float* v,
+                           const float* gamma, const float* beta, const float* lambda,
+                           int B, int H, int dk, int dv,
+                           float* Hstate, float* Gstate, float* x_state,
+                           int cg_steps, float tol,
+                           float* out, int32_t* iters_out, void* stream) {
     if (B < 1 || H < 1 || dk < 1 || dv < 1) return MESA_ERR_INVALID_ARG;
     if (cg_steps < 0 || cg_steps > 1024 || isnan(tol)) return MESA_ERR_INVALID_ARG;
     if (!supported_width(dk) || dk != dv) return MESA_ERR_UNSUPPORTED;
@@ -356,9 +356,21 @@ mesa_status mesa_step(const float* q, const float* k, const float* v,
         if (!aligned(p, 16)) return MESA_ERR_INVALID_ARG;
     if (!aligned(gamma, 4) || !aligned(beta, 4) || !aligned(lambda, 4)) return MESA_ERR_INVALID_ARG;
     if (iters_out && !aligned(iters_out, 4)) return MESA_ERR_INVALID_ARG;
+    if (x_state && !aligned(x_state, 4)) return MESA_ERR_INVALID_ARG;
     if (Hstate == Gstate) return MESA_ERR_INVALID_ARG;
-    StepArgs a{q, k, v, gamma, beta, lambda, B, H, dk, dv, Hstate, Gstate, cg_steps, tol, out, iters_out};
+    if (x_state && ((const void*)x_state == (const void*)q || x_state == out)) return MESA_ERR_INVALID_ARG;
+    StepArgs a{q, k, v, gamma, beta, lambda, B, H, dk, dv, Hstate, Gstate, cg_steps, tol, out, iters_out, x_state};
     return step_launch(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+mesa_status mesa_step(const float* q, const float* k, const float* v,
+                      const float* gamma, const float* beta, const float* lambda,
+                      int B, int H, int dk, int dv,
+                      float* Hstate, float* Gstate,
+                      int cg_steps, float tol,
+                      float* out, int32_t* iters_out, void* stream) {
+    return mesa_step_warm(q, k, v, gamma, beta, lambda, B, H, dk, dv, Hstate, Gstate, nullptr, cg_steps, tol,
+                          out, iters_out, stream);
 }
 
 mesa_status mesa_preprocess(const void* q_raw, const void* k_raw, const float* conv_q, const float* conv_k,

@@ -17,7 +17,12 @@
 //     l*CPL .. l*CPL+CPL-1), so every CG matvec runs from registers;
 //   * each matvec reduces its per-lane partial row sums with a butterfly
 //     transpose-reduction (R rows over 32 lanes in R-1+log2(32/R)... shuffles)
-//     instead of R full warp reductions.
+//     instead of R full warp reductions; the block sums use a double-buffered
+//     scratch, one barrier each;
+//   * with x_state the CG starts from the caller's guess (warm start; the
+//     pages name warm starts as the way to cut the solver's cost, MesaNet
+//     page, Significance and claims): r0 = q - (H + Lambda) x0, and the
+//     solution is written back to x_state.
 #include "mesa_common.cuh"
 #include "mesa_internal.h"
 
@@ -58,16 +63,20 @@ __device__ __forceinline__ int row_of_lane(int lane) {
 }
 
 // Block-wide sum; exactly one lane per row contributes (contrib == true).
-__device__ __forceinline__ float block_sum(float v, bool contrib, float* red, int warp, int lane) {
+// red holds two kWarps-slot buffers used alternately (par flips per call):
+// the barrier of the call in between orders a buffer's readers before its
+// next writers, so each call needs one barrier.
+__device__ __forceinline__ float block_sum(float v, bool contrib, float* red, int& par, int warp, int lane) {
     float s = contrib ? v : 0.f;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    __syncthreads();  // previous readers of red are done
-    if (lane == 0) red[warp] = s;
+    float* rb = red + par * kWarps;
+    if (lane == 0) rb[warp] = s;
     __syncthreads();
     float tot = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) tot += red[w];
+    for (int w = 0; w < kWarps; ++w) tot += rb[w];
+    par ^= 1;
     return tot;
 }
 
@@ -76,7 +85,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 step_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
             const float* __restrict__ gamma, const float* __restrict__ beta,
             const float* __restrict__ lambda, int H, float* __restrict__ Hs, float* __restrict__ Gs,
-            int cg_steps, float tol, float* __restrict__ out, int32_t* __restrict__ iters) {
+            int cg_steps, float tol, float* __restrict__ out, int32_t* __restrict__ iters,
+            float* __restrict__ xs) {
     constexpr int RPW = D / kWarps;                  // rows per warp
     constexpr int CPL = D >= 32 ? D / 32 : 1;        // columns per lane
     constexpr int DUP = 32 / RPW;                    // lanes sharing one row after the reduction
@@ -87,7 +97,7 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
     float* sk = sG + D * D;       // D
     float* sv = sk + D;           // D
     float* sp = sv + D;           // D (CG direction, later x)
-    float* red = sp + D;          // kWarps
+    float* red = sp + D;          // 2 x kWarps
 
     const int bh = blockIdx.x, h = bh % H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -151,12 +161,10 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
     const int ri = warp + kWarps * row_of_lane<RPW>(lane);
     const bool contrib = (lane & (DUP - 1)) == 0;
     const float lam_i = lambda[(size_t)h * D + ri];
-    float xi = 0.f, r_i = sp[ri], pi = r_i;
-    float rr = block_sum(r_i * r_i, contrib, red, warp, lane);
-    const float qn = sqrtf(rr);
-    int it = 0;
-    for (int s = 0; s < cg_steps; ++s) {
-        if (!cg_may_continue(rr, qn, tol)) break;   // block-uniform
+    int par = 0;
+    // (H + Lambda) applied to the vector in sp, for row ri (sp must be
+    // published by a barrier before the call)
+    auto matvec_row = [&](float own) {
         float pc[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; ++c) pc[c] = col_ok ? sp[col0 + c] : 0.f;
@@ -168,13 +176,33 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
             for (int c = 0; c < CPL; ++c) acc = fmaf(Hr[m][c], pc[c], acc);
             part[m] = acc;
         }
-        const float yi = fmaf(lam_i, pi, butterfly_reduce<RPW>(part, lane));
-        const float pAp = block_sum(pi * yi, contrib, red, warp, lane);
+        return fmaf(lam_i, own, butterfly_reduce<RPW>(part, lane));
+    };
+    const float q_i = sp[ri];
+    float xi = 0.f, r_i = q_i;
+    const float qq = block_sum(q_i * q_i, contrib, red, par, warp, lane);   // its barrier ends the reads of q
+    const float qn = sqrtf(qq);
+    float rr = qq;
+    if (xs) {                                           // r0 = q - (H + Lambda) x0
+        xi = xs[(size_t)bh * D + ri];
+        if (contrib) sp[ri] = xi;
+        __syncthreads();
+        r_i = q_i - matvec_row(xi);
+        rr = block_sum(r_i * r_i, contrib, red, par, warp, lane);          // its barrier ends the reads of x0
+        if (contrib) sp[ri] = r_i;                      // p0 = r0
+        __syncthreads();
+    }
+    float pi = r_i;
+    int it = 0;
+    for (int s = 0; s < cg_steps; ++s) {
+        if (!cg_may_continue(rr, qn, tol)) break;   // block-uniform
+        const float yi = matvec_row(pi);
+        const float pAp = block_sum(pi * yi, contrib, red, par, warp, lane);
         if (!cg_curvature_ok(pAp)) break;
         const float alpha = rr / pAp;
         xi = fmaf(alpha, pi, xi);
         r_i = fmaf(-alpha, yi, r_i);
-        const float rr_new = block_sum(r_i * r_i, contrib, red, warp, lane);
+        const float rr_new = block_sum(r_i * r_i, contrib, red, par, warp, lane);
         pi = fmaf(rr_new / rr, pi, r_i);
         rr = rr_new;
         ++it;
@@ -216,18 +244,19 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
     const float oi = butterfly_reduce<RPW>(part, lane);
     if (contrib) out[(size_t)bh * D + ri] = oi;
     if (iters && tid == 0) iters[bh] = it;
+    if (xs && contrib) xs[(size_t)bh * D + ri] = xi;
 }
 
 template <int D>
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
-    const size_t smem = sizeof(float) * ((size_t)D * D + 3 * D + kWarps);
+    const size_t smem = sizeof(float) * ((size_t)D * D + 3 * D + 2 * kWarps);
     auto kern = step_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     {
         LaunchTimer timer(kKindStep, st);
         kern<<<a.B * a.H, kThreads, smem, st>>>(a.q, a.k, a.v, a.gamma, a.beta, a.lambda, a.H, a.Hs, a.Gs,
-                                                a.cg_steps, a.tol, a.out, a.iters);
+                                                a.cg_steps, a.tol, a.out, a.iters, a.xs);
     }
     return cudaGetLastError();
 }

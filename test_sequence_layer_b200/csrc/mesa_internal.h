@@ -79,6 +79,7 @@ struct StepArgs {
     float tol;
     float* out;
     int32_t* iters;
+    float* xs;           // optional warm start [B,H,dk], in/out
 };
 cudaError_t step_launch(const StepArgs& a, cudaStream_t st);
 

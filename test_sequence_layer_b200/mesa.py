@@ -50,6 +50,8 @@ def _load():
     lib.mesa_forward_host_workspace_size.restype = Z
     lib.mesa_step.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, I, F, P, P, P]
     lib.mesa_step.restype = I
+    lib.mesa_step_warm.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, P, I, F, P, P, P]
+    lib.mesa_step_warm.restype = I
     lib.mesa_get_error.argtypes = [P]
     lib.mesa_get_error.restype = I
     lib.mesa_status_string.argtypes = [I]
@@ -184,18 +186,20 @@ def preprocess(q_raw, k_raw, conv_q, conv_k, *, q_out=None, k_out=None, stream=N
 
 
 def step(q, k, v, gamma, beta, lam, Hstate, Gstate, *, cg_steps=15, tol=0.0, out=None,
-         iters=None, stream=None):
+         iters=None, x_state=None, stream=None):
     """One decode step; Hstate [B,H,dk,dk] and Gstate [B,H,dv,dk] (float32) are
-    updated in place. q, k: [B,H,dk]; v: [B,H,dv]; gamma, beta: [B,H]."""
+    updated in place. q, k: [B,H,dk]; v: [B,H,dv]; gamma, beta: [B,H].
+    x_state [B,H,dk] float32 (optional, in/out): the CG starts from it and it
+    receives the solution (mesa_step_warm)."""
     lib = _load()
     B, H, dk = q.shape
     dv = v.shape[-1]
     if out is None:
         out = torch.empty((B, H, dv), dtype=torch.float32, device=q.device)
-    rc = lib.mesa_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam), B, H, dk, dv,
-                       _ptr(Hstate), _ptr(Gstate), int(cg_steps), float(tol), _ptr(out), _ptr(iters),
-                       _stream(stream, q.device))
-    _check(rc, "mesa_step")
+    rc = lib.mesa_step_warm(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam), B, H, dk, dv,
+                            _ptr(Hstate), _ptr(Gstate), _ptr(x_state), int(cg_steps), float(tol), _ptr(out),
+                            _ptr(iters), _stream(stream, q.device))
+    _check(rc, "mesa_step_warm")
     return out
 
 

@@ -125,3 +125,58 @@ def test_full_size_decode_sampled(mesa, oracle_mod):
     ref = np.stack(refs, 1)
     # the prefill runs in bf16-input mode; the steps themselves are fp32
     assert rel_err(got, ref) <= 2e-3, err_report(got, ref)
+
+
+@pytest.mark.parametrize("d", [16, 64, 128])
+@pytest.mark.parametrize("tol", [0.0, 1e-3])
+def test_warm_steps_match_oracle(mesa, oracle_mod, d, tol):
+    """mesa_step_warm carrying x between steps (each solve starts from the
+    previous step's solution) against oracle_step_warm, step by step."""
+    w = mi.Workload("t", 2, 3, 24, d, d, 16, "f32", 15, tol, tol > 0, 61 + d)
+    x = mi.batch(w)
+    t0 = 8
+    N = 30 if tol > 0 else 4                     # few steps: the start matters for the result
+    _, _, Hs, Gs = oracle_mod.forward_cg(*(x[n][:, :, :t0] for n in ("q", "k", "v", "gamma", "beta")), x["lam"], N, tol)
+    Hg = torch.from_numpy(Hs).float().cuda()
+    Gg = torch.from_numpy(Gs).float().cuda()
+    xs_ref = np.zeros((2, 3, d))
+    xs = torch.zeros((2, 3, d), device="cuda")
+    lam = torch.from_numpy(x["lam"]).float().cuda()
+    iters = torch.empty((2, 3), dtype=torch.int32, device="cuda")
+    for t in range(t0, w.T):
+        step_in = [x[n][:, :, t] for n in ("q", "k", "v", "gamma", "beta")]
+        ref, it_ref, Hs, Gs, xs_ref = oracle_mod.step(*step_in, x["lam"], Hs, Gs, N, tol, x_state=xs_ref)
+        o = mesa.step(*(torch.from_numpy(np.ascontiguousarray(a)).float().cuda() for a in step_in), lam, Hg, Gg,
+                      cg_steps=N, tol=tol, iters=iters, x_state=xs)
+        torch.cuda.synchronize()
+        # with a tolerance an iteration count may differ by one, which moves the result by ~tol
+        bound = TOL_F32 if tol == 0 else 2e-2
+        assert rel_err(o.cpu().numpy(), ref) <= bound, (t, err_report(o.cpu().numpy(), ref))
+        assert rel_err(xs.cpu().numpy(), xs_ref) <= bound, t
+        if tol == 0:
+            assert np.all(iters.cpu().numpy() == N)
+        else:
+            assert np.abs(iters.cpu().numpy() - it_ref).max() <= 1
+    assert mesa.get_error() == 0
+
+
+def test_warm_step_from_zero_equals_cold_step(mesa):
+    """x_state = 0 gives exactly mesa_step, and x_state receives the solution."""
+    B, H, d = 4, 16, 128
+    g = torch.Generator(device="cuda").manual_seed(3)
+    kr = torch.nn.functional.normalize(torch.randn((B, H, 32, d), generator=g, device="cuda"), dim=-1)
+    Hs = kr.transpose(-1, -2) @ kr
+    Gs = torch.randn((B, H, 32, d), generator=g, device="cuda").transpose(-1, -2) @ kr
+    q = torch.nn.functional.normalize(torch.randn((B, H, d), generator=g, device="cuda"), dim=-1)
+    k = torch.nn.functional.normalize(torch.randn((B, H, d), generator=g, device="cuda"), dim=-1)
+    v = torch.randn((B, H, d), generator=g, device="cuda")
+    gam = torch.full((B, H), 0.9, device="cuda")
+    bet = torch.full((B, H), 0.5, device="cuda")
+    lam = torch.full((H, d), 0.3, device="cuda")
+    H1, G1, H2, G2 = Hs.clone(), Gs.clone(), Hs.clone(), Gs.clone()
+    o1 = mesa.step(q, k, v, gam, bet, lam, H1, G1, cg_steps=15)
+    xs = torch.zeros((B, H, d), device="cuda")
+    o2 = mesa.step(q, k, v, gam, bet, lam, H2, G2, cg_steps=15, x_state=xs)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(H1, H2) and torch.equal(G1, G2)
+    assert torch.allclose(torch.einsum("bhij,bhj->bhi", G2, xs), o2, rtol=1e-5, atol=1e-5)
