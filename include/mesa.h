@@ -180,8 +180,10 @@ size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int
 /*
  * The same forward with every tensor in HOST memory (page-locked memory is
  * needed for the copies to overlap; pageable memory works but is slower).
- * The batch is split into up to 8 slices of whole batch rows b (one slice
- * when the inputs are under 16 MiB). Slice by slice, the inputs are copied to
+ * The batch is split into slices of sequences (one slice when the inputs are
+ * under 16 MiB): with 16 or more batch rows, up to 32 groups of whole rows;
+ * with fewer, runs of heads inside one batch row (about 16 slices). Slice by
+ * slice, the inputs are copied to
  * the device on a library copy-in stream, the forward runs on one of two
  * library compute streams once they have landed, and the outputs are copied
  * back on a library copy-out stream, so both copy directions overlap the

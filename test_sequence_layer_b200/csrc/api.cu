@@ -132,11 +132,15 @@ namespace {
 
 // Streams and events of the host-buffer pipeline, created once per device and
 // kept for the life of the process. The pipeline splits the batch into slices
-// of whole batch rows b (every (b, h) sequence is independent): slice i's
-// inputs go up on the copy-in stream, its forward runs on compute stream i % 2
-// once they have landed, and its outputs come down on the copy-out stream once
-// it is done, so the two copy directions and the kernels overlap.
-constexpr int kMaxSlices = 8;
+// of sequences (every (b, h) sequence is independent): a slice is a run of
+// nh heads of one batch row b, so it is contiguous in every [B,H,...] tensor
+// and runs as a forward with B = 1, H = nh and lambda offset to its first
+// head. Slice i's inputs go up on the copy-in stream, its forward runs on
+// compute stream i % 2 once they have landed, and its outputs come down on the
+// copy-out stream once it is done, so the two copy directions and the kernels
+// overlap.
+constexpr int kMaxSlices = 32;
+constexpr int kTargetSlices = 16;
 struct HostPipe {
     bool ready = false;
     cudaStream_t in = nullptr, out = nullptr, comp[2] = {nullptr, nullptr};
@@ -254,14 +258,24 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
 
     const size_t tok = (size_t)B * H * T;
     const size_t es = elem_size(dtype);
-    // slices: whole batch rows; one slice for small or empty problems
+    // slices: with at least kTargetSlices batch rows, groups of whole rows (at
+    // most kMaxSlices slices); with fewer, runs of nh heads inside one row (nh
+    // halves while it divides evenly, to about kTargetSlices slices); one
+    // slice for small or empty problems
     const size_t in_bytes = tok * (2 * dk + dv) * es + tok * 8;
-    const int nS = (T == 0 || in_bytes < ((size_t)16 << 20)) ? 1 : (B < kMaxSlices ? B : kMaxSlices);
-    const int Bs = (B + nS - 1) / nS;
-    const int nslices = (B + Bs - 1) / Bs;
-
+    const bool split = T > 0 && in_bytes >= ((size_t)16 << 20);
+    int nslices = 1, Bs = B, Hs_ = H, per_row = 1;
+    if (split && B >= kTargetSlices) {
+        Bs = (B + kMaxSlices - 1) / kMaxSlices;
+        nslices = (B + Bs - 1) / Bs;
+    } else if (split) {
+        while (Hs_ % 2 == 0 && B * (H / Hs_) < kTargetSlices) Hs_ /= 2;
+        per_row = H / Hs_;
+        nslices = B * per_row;                         // < 2 kTargetSlices = kMaxSlices
+        Bs = 1;
+    }
     char* w = static_cast<char*>(workspace);
-    const size_t fws_slice = round_up(workspace_bytes(Bs, H, T, dk, dv, chunk, dtype), 256);
+    const size_t fws_slice = round_up(workspace_bytes(Bs, Hs_, T, dk, dv, chunk, dtype), 256);
     const size_t fws_total = round_up(workspace_bytes(B, H, T, dk, dv, chunk, dtype), 256) + 2 * 256;
     const int ncomp = (nslices > 1 && 2 * fws_slice <= fws_total) ? 2 : 1;   // compute streams
     char* fws[2] = {w, ncomp == 2 ? w + fws_slice : w};
@@ -292,9 +306,28 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
     for (cudaStream_t sm : {hp->in, hp->comp[0], hp->comp[1], hp->out})
         ok = ok && cudaStreamWaitEvent(sm, hp->start, 0) == cudaSuccess;
     ok = ok && cp(dl, lambda, (size_t)H * dk * 4, H2D, hp->in);
+    // slice i: sequences s0 .. s0+ns-1, run as a forward over nb batch rows of
+    // nhs heads starting at head h0 (lambda is offset to h0)
+    auto slice = [&](int i, size_t& s0, size_t& ns, int& h0, int& nb, int& nhs) {
+        if (per_row > 1) {
+            const int b = i / per_row;
+            h0 = (i % per_row) * Hs_;
+            nb = 1;
+            nhs = Hs_;
+            s0 = (size_t)b * H + h0;
+        } else {
+            const int b0 = i * Bs;
+            nb = (B - b0 < Bs) ? B - b0 : Bs;
+            h0 = 0;
+            nhs = H;
+            s0 = (size_t)b0 * H;
+        }
+        ns = (size_t)nb * nhs;
+    };
     for (int i = 0; ok && i < nslices; ++i) {
-        const int b0 = i * Bs, nb = (B - b0 < Bs) ? B - b0 : Bs;
-        const size_t s0 = (size_t)b0 * H, ns = (size_t)nb * H;      // sequences
+        size_t s0, ns;
+        int h0, nb, nhs;
+        slice(i, s0, ns, h0, nb, nhs);
         const size_t t0 = s0 * T, nt = ns * T;                        // tokens
         const char* hq = static_cast<const char*>(q);
         const char* hk = static_cast<const char*>(k);
@@ -310,13 +343,15 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
         ok = ok && cudaEventRecord(hp->landed[i], hp->in) == cudaSuccess;
     }
     for (int i = 0; ok && i < nslices; ++i) {
-        const int b0 = i * Bs, nb = (B - b0 < Bs) ? B - b0 : Bs;
-        const size_t s0 = (size_t)b0 * H, t0 = s0 * T;
+        size_t s0, ns;
+        int h0, nb, nhs;
+        slice(i, s0, ns, h0, nb, nhs);
+        const size_t t0 = s0 * T;
         cudaStream_t cs = hp->comp[i % ncomp];
         ok = cudaStreamWaitEvent(cs, hp->landed[i], 0) == cudaSuccess;
         if (!ok) break;
-        ForwardArgs a{dq + t0 * dk * es, dk_ + t0 * dk * es, dv_ + t0 * dv * es, dg + t0, db + t0, dl,
-                      nb, H, T, dk, dv, chunk, dtype, cg_steps, tol,
+        ForwardArgs a{dq + t0 * dk * es, dk_ + t0 * dk * es, dv_ + t0 * dv * es, dg + t0, db + t0, dl + (size_t)h0 * dk,
+                      nb, nhs, T, dk, dv, chunk, dtype, cg_steps, tol,
                       dout + t0 * dv, iters_out ? dit + t0 : nullptr,
                       H_in ? dHi + s0 * hs : nullptr, G_in ? dGi + s0 * gs : nullptr,
                       H_out ? dHo + s0 * hs : nullptr, G_out ? dGo + s0 * gs : nullptr,
@@ -326,8 +361,10 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
         ok = cudaEventRecord(hp->done[i], cs) == cudaSuccess;
     }
     for (int i = 0; ok && i < nslices; ++i) {
-        const int b0 = i * Bs, nb = (B - b0 < Bs) ? B - b0 : Bs;
-        const size_t s0 = (size_t)b0 * H, ns = (size_t)nb * H, t0 = s0 * T, nt = ns * T;
+        size_t s0, ns;
+        int h0, nb, nhs;
+        slice(i, s0, ns, h0, nb, nhs);
+        const size_t t0 = s0 * T, nt = ns * T;
         ok = cudaStreamWaitEvent(hp->out, hp->done[i], 0) == cudaSuccess;
         if (T > 0) ok = ok && cp(out + t0 * dv, dout + t0 * dv, nt * dv * 4, D2H, hp->out);
         if (T > 0 && iters_out) ok = ok && cp(iters_out + t0, dit + t0, nt * 4, D2H, hp->out);

@@ -176,10 +176,11 @@ def test_host_buffer_variant(mesa, oracle_mod):
     assert np.allclose(Hout.numpy(), Hf, rtol=1e-4, atol=1e-5)
 
 
-@pytest.mark.parametrize("dtype,chunk,B,T", [("bf16", 64, 11, 1536), ("f32", 32, 3, 2100)])
+@pytest.mark.parametrize("dtype,chunk,B,T", [("bf16", 64, 11, 1536), ("f32", 32, 3, 2100), ("bf16", 64, 17, 1024)])
 def test_host_pipeline_matches_device(mesa, dtype, chunk, B, T):
-    """Inputs above 16 MiB go through the sliced copy/compute pipeline (uneven
-    last slice for B = 11). Every sequence is independent, so the host-buffer
+    """Inputs above 16 MiB go through the sliced copy/compute pipeline: runs of
+    heads inside a batch row (B = 11, B = 3), groups of whole rows (B = 17).
+    Every sequence is independent, so the host-buffer
     call must reproduce the device-buffer call bit for bit, initial and final
     states included."""
     w = rand_workload(128, chunk, dtype, T, B=B, H=4, N=15, seed=33)
