@@ -22,6 +22,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -99,7 +100,8 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # raw samples of the timed region, kept beside the JSON line's summary
+        self.path = os.path.join(tempfile.gettempdir(), f"mesa_bench_clocks_rank{index}.csv")
 
     def start(self):
         try:
