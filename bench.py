@@ -55,15 +55,17 @@ def load_peaks():
 # Reported only while the kernel source still hashes to the captured version;
 # otherwise the field is null.
 MEASURED_TRAFFIC = {
-    "tc_cg": {"src_sha16": "c37d4ab6e10641c0", "bytes_per_token": (337.729280e6 + 108.120320e6) / 262144},
-    "tc_scan": {"src_sha16": "c37d4ab6e10641c0", "bytes_per_token": (136.442624e6 + 92.728576e6) / 262144},
+    "tc_cg": {"src_sha16": "c37d4ab6e10641c0", "files": ("tc_forward.cu", "tc_layout.cuh", "tc_common.cuh"),
+              "bytes_per_token": (337.729280e6 + 108.120320e6) / 262144},
+    "tc_scan": {"src_sha16": "c37d4ab6e10641c0", "files": ("tc_scan.cu", "tc_layout.cuh", "tc_common.cuh"),
+                "bytes_per_token": (136.442624e6 + 92.728576e6) / 262144},
     "preprocess": {"src_sha16": "084d9e828774199c", "files": ("preprocess.cu",),
                    "bytes_per_token": (537.019904e6 + 489.792512e6) / 1048576},
     "decode_step": {"src_sha16": "2d83b99e92f2442f", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
 }
 
 
-def kernel_source_sha16(files=("tc_forward.cu", "tc_common.cuh")):
+def kernel_source_sha16(files):
     """Hash of the release kernel source: MESA_DEBUG blocks (compiled only into
     the debug library) are left out."""
     import hashlib
@@ -80,7 +82,7 @@ def measured_traffic(kernel, units):
     """Measured DRAM bytes of one launch processing `units` tokens (heads for
     the decode step), or None when the source changed since the capture."""
     rec = MEASURED_TRAFFIC.get(kernel)
-    if rec is None or rec["src_sha16"] != kernel_source_sha16(rec.get("files", ("tc_forward.cu", "tc_common.cuh"))):
+    if rec is None or rec["src_sha16"] != kernel_source_sha16(rec["files"]):
         return None
     return rec["bytes_per_token"] * units
 

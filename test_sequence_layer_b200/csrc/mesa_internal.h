@@ -58,6 +58,9 @@ cudaError_t forward_simt(const ForwardArgs& a, cudaStream_t st);
 bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype);
 size_t tc_workspace_bytes(int B, int H, int T);
 cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st);
+// Chunk-state scan of the tensor-core forward: state images and scales into
+// img / scales (layout in tc_layout.cuh), final states into a.H_out / a.G_out.
+cudaError_t tc_scan_launch(const ForwardArgs& a, void* img, float* scales, unsigned* err, cudaStream_t st);
 #ifdef MESA_DEBUG
 // The next `launches` launches of the tensor-core solve kernel leave out the
 // completion signal of their first Z product (fault injection, debug builds).

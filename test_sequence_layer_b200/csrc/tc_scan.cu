@@ -1,0 +1,353 @@
+// tc_scan.cu -- tensor-core chunk-state scan of the Mesa layer for bf16
+// inputs, dk = dv = 128, chunk C = 64.
+//
+// Method: "MesaNet: Sequence Modeling by Locally Optimal Test-Time Training"
+// (gist.science), Technical summary > Method > Mesa layer and its
+// "Parallelisation" paragraph: the states carried from chunk to chunk obey
+//     H_{c+1} = e^{b_last} H_c + K^T diag(w) K,   G_{c+1} = e^{b_last} G_c + V^T diag(w) K,
+// with b_t the in-chunk log-cumsum of gamma and w_j = beta_j e^{b_last-b_j}.
+// The kernel walks the chunks of each sequence, keeps the running state in
+// fp32 registers and writes the state before every 128-token block of the
+// solve as a scaled fp16 image (format in tc_layout.cuh), plus the final state.
+//
+// Numerics: w_j a_j is split into an fp16 hi/lo pair, both multiplied by the
+// fp16 keys on the tensor cores with fp32 accumulation, so each chunk's sum
+// carries ~22-bit products into the fp32 running state.
+#include "mesa_internal.h"
+#include "tc_layout.cuh"
+
+namespace mesa {
+namespace {
+
+using namespace tc;
+
+// Inclusive log-cumsum of gamma over a 64-token chunk by warp 0 (padded
+// tokens count as gamma = 1).
+// b[t] for t < 64: in-chunk inclusive cumulative sum of log gamma over the
+// chunk's first n positions, held constant past n. One warp; g points at the
+// chunk's gamma (global or shared memory).
+__device__ __forceinline__ void warp_gate_cumsum(const float* g, int n, float* b) {
+    const int lane = threadIdx.x & 31;
+    const int t0 = 2 * lane, t1 = 2 * lane + 1;
+    const float l0 = (t0 < n) ? logf(g[t0]) : 0.f;
+    const float l1 = (t1 < n) ? logf(g[t1]) : 0.f;
+    const float pair = l0 + l1;
+    float incl = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    const float excl = incl - pair;
+    b[t0] = excl + l0;
+    b[t1] = excl + l0 + l1;
+}
+
+// =====================================================================
+// Chunk-state scan
+// =====================================================================
+// The fp16 image of a chunk-start state is scaled by s = 2^ceil(log2 max(Bnd,1))
+// where Bnd bounds every entry: Bnd_0 = max|S_in| and
+// Bnd_{c+1} = e^{b_last} Bnd_c + sum_j w_j |a_j|_inf |k_j|_inf (a = k for H,
+// a = v for G), since |(a_j k_j^T)_il| <= |a_j|_inf |k_j|_inf. Every warp of
+// the CTA evaluates the same scalar recurrence in the same order, so all
+// threads agree on the scale without communicating.
+constexpr int kScanThreads = 512;
+
+struct ScanSmem {
+    static constexpr int oRawA = 0;               // 2 x [64][128] bf16 rows of a (16 KB each)
+    static constexpr int oRawK = 32768;           // 2 x [64][128] bf16 rows of k
+    static constexpr int oAhi = 65536;            // MN-major [64 j][128 i] fp16, 16 KB
+    static constexpr int oAlo = 81920;
+    static constexpr int oB = 98304;              // MN-major [64 j][128 l] fp16, 16 KB
+    static constexpr int oGate = 114688;          // b[2][64], w[2][64], amax[64], kmax[64]
+    static constexpr int oGraw = oGate + 1536;    // 2 x {gamma[64], beta[64]} prefetched with the rows
+    static constexpr int oRed = oGraw + 1024;     // 32 floats; [31] is the abort flag
+    static constexpr int oBar = oRed + 128;       // raw[2], mma
+    static constexpr int oSlot = oBar + 32;
+    static constexpr int bytes = oSlot + 16;
+};
+
+// CTA (m, bh) walks the chunks of sequence bh for m = 0 (H, a = k) or m = 1
+// (G, a = v) and holds the whole 128 x 128 running state in registers: warp w
+// serves TMEM lane quadrant w % 4 (state rows 32 (w % 4) .. + 31, one per
+// thread) and the 32 columns 32 (w / 4) .. + 31. Per chunk, with
+// w_j = beta_j e^{b_last - b_j},
+//     S <- e^{b_last} S + sum_j (w_j a_j) k_j^T
+// where the sum is one M = 128, N = 128, K = 64 MMA over the chunk's tokens,
+// issued for the hi and the lo fp16 parts of w_j a_j. The gates of chunk c + 1
+// are formed by warp 1 while the MMA of chunk c runs.
+__global__ void __launch_bounds__(kScanThreads, 1)
+tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+               const float* __restrict__ gamma, const float* __restrict__ beta, int T, int nc,
+               const float* __restrict__ H_in, const float* __restrict__ G_in, __half* __restrict__ img,
+               float* __restrict__ scales, float* __restrict__ H_out, float* __restrict__ G_out,
+               unsigned* __restrict__ err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int m = blockIdx.x, bh = blockIdx.y;
+    uint8_t* rawK = smem + ScanSmem::oRawK;
+    uint8_t* rawA = m ? smem + ScanSmem::oRawA : rawK;     // for H the left factor is k itself
+    uint8_t* Ahi = smem + ScanSmem::oAhi;
+    uint8_t* Alo = smem + ScanSmem::oAlo;
+    uint8_t* Bk = smem + ScanSmem::oB;
+    float* sb = reinterpret_cast<float*>(smem + ScanSmem::oGate);      // [2][64]
+    float* sw = sb + 2 * kC;                                            // [2][64]
+    float* amax = sw + 2 * kC;
+    float* kmax = amax + kC;
+    float* graw = reinterpret_cast<float*>(smem + ScanSmem::oGraw);
+    float* red = reinterpret_cast<float*>(smem + ScanSmem::oRed);
+    uint64_t* bar_raw = reinterpret_cast<uint64_t*>(smem + ScanSmem::oBar);
+    uint64_t* bar_mma = bar_raw + 2;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + ScanSmem::oSlot);
+
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int q4 = w & 3;
+    const int row = 32 * q4 + lane;               // state row owned by this thread
+    const int col0 = 32 * (w >> 2);               // its 32 columns
+    const __nv_bfloat16* A = m ? v : k;
+    const float* init = m ? G_in : H_in;
+    float* fin = m ? G_out : H_out;
+    const size_t seq = (size_t)bh * T;
+    // gamma/beta of a chunk travel with its rows when the chunk is full and its
+    // first element is 16-byte aligned (T % 4 == 0); otherwise warp 1 reads them.
+    const bool gates_bulk = (T % 4) == 0 && ((reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(beta)) & 15) == 0;
+
+    int prefetched = 0;                           // chunks whose copies were issued (thread 0)
+    auto prefetch = [&](int cc) {                 // rows (and gates) of chunk cc -> buffer cc & 1 (thread 0)
+        const int nn = min(kC, T - cc * kC);
+        const uint32_t bytes = (uint32_t)nn * kD * 2;
+        const int buf = cc & 1;
+        const bool gb = gates_bulk && nn == kC;
+        mbar_arrive_expect_tx(bar_raw + buf, (m ? 2 * bytes : bytes) + (gb ? 512u : 0u));
+        bulk_g2s(rawK + buf * 16384, k + (seq + (size_t)cc * kC) * kD, bytes, bar_raw + buf);
+        if (m) bulk_g2s(rawA + buf * 16384, A + (seq + (size_t)cc * kC) * kD, bytes, bar_raw + buf);
+        if (gb) {
+            bulk_g2s(graw + buf * 128, gamma + seq + (size_t)cc * kC, 256, bar_raw + buf);
+            bulk_g2s(graw + buf * 128 + 64, beta + seq + (size_t)cc * kC, 256, bar_raw + buf);
+        }
+        prefetched = cc + 1;
+    };
+    // One warp: waits for chunk cc's copies, then b (log-cumsum of gamma) and
+    // w_j = beta_j e^{b_last - b_j} into gate buffer cc & 1.
+    auto chunk_gates = [&](int cc) {
+        const int buf = cc & 1;
+        if (!mbar_wait(bar_raw + buf, (cc >> 1) & 1)) red[31] = 1.f;
+        __syncwarp();
+        const int nn = min(kC, T - cc * kC);
+        const size_t base = seq + (size_t)cc * kC;
+        const bool gb = gates_bulk && nn == kC;
+        const float* gsrc = gb ? graw + buf * 128 : gamma + base;
+        const float* bsrc = gb ? graw + buf * 128 + 64 : beta + base;
+        float* b = sb + buf * kC;
+        float* wv = sw + buf * kC;
+        warp_gate_cumsum(gsrc, nn, b);
+        __syncwarp();
+        const float bl = b[kC - 1];                                // b at the chunk's last position
+        wv[lane] = (lane < nn) ? bsrc[lane] * expf(bl - b[lane]) : 0.f;
+        wv[lane + 32] = (lane + 32 < nn) ? bsrc[lane + 32] * expf(bl - b[lane + 32]) : 0.f;
+    };
+
+    if (tid == 0) {
+        mbar_init(bar_raw, 1);
+        mbar_init(bar_raw + 1, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        red[31] = 0.f;
+    }
+    if (w == 0) tmem_alloc(slot, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *slot;
+    if (tid == 0 && nc > 0) {
+        prefetch(0);
+        if (nc > 1) prefetch(1);
+    }
+
+    float S[32];
+    float bound = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) S[i] = 0.f;
+    if (init) {
+        const float4* src = reinterpret_cast<const float4*>(init + ((size_t)bh * kD + row) * kD + col0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 f = src[i];
+            S[4 * i] = f.x; S[4 * i + 1] = f.y; S[4 * i + 2] = f.z; S[4 * i + 3] = f.w;
+        }
+        // max |S_in| over the matrix: each thread's own 32 entries, then the CTA
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(S[i]));
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red[w] = mx;
+        __syncthreads();
+        bound = red[0];
+#pragma unroll
+        for (int i = 1; i < kScanThreads / 32; ++i) bound = fmaxf(bound, red[i]);
+    }
+    if (w == 1 && nc > 0) chunk_gates(0);
+    __syncthreads();                              // gates of chunk 0 (and the bound's partials) read
+    bool ok = red[31] == 0.f;
+
+    constexpr uint32_t kIdesc = idesc_f16(128, 128, true, true);
+    const uint64_t dAhi = sdesc(smem_addr(Ahi), 8192, 1024), dAlo = sdesc(smem_addr(Alo), 8192, 1024);
+    const uint64_t dB = sdesc(smem_addr(Bk), 8192, 1024);
+    uint32_t mma_phase = 0;
+    bool mma_out = false;                         // thread 0: a committed MMA not yet observed
+    int c = 0;
+    for (; ok; ++c) {
+        // ---- emit the state before chunk c (fp16 image + scale) when c starts a
+        //      128-token block of the solve, or the final state ----
+        if (c < nc && (c & 1) == 0) {
+            const float s = pow2_ceil_at_least_one(bound);
+            const float inv = 1.f / s;
+            const size_t ci = image_index(bh, (nc + 1) >> 1, c >> 1, m);
+            if (tid == 0) scales[ci] = s;
+            uint8_t* dst = reinterpret_cast<uint8_t*>(img + ci * kImgHalves) + (col0 >> 6) * 16384 + row * 128;
+            const int g0 = (col0 & 63) >> 3;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint4 o;
+                o.x = pack_half2(S[8 * g] * inv, S[8 * g + 1] * inv);
+                o.y = pack_half2(S[8 * g + 2] * inv, S[8 * g + 3] * inv);
+                o.z = pack_half2(S[8 * g + 4] * inv, S[8 * g + 5] * inv);
+                o.w = pack_half2(S[8 * g + 6] * inv, S[8 * g + 7] * inv);
+                *reinterpret_cast<uint4*>(dst + (((g0 + g) ^ (row & 7)) << 4)) = o;
+            }
+        } else if (c == nc) {
+            if (fin) {
+                float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+            }
+            break;
+        }
+        const int n = min(kC, T - c * kC);
+        const int buf = c & 1;
+        const float* swc = sw + buf * kC;
+        const float blast = sb[buf * kC + kC - 1];
+        // ---- operand images: A = w_j a_j (hi/lo) [j][i], B = k_j [j][l], both
+        //      MN-major SW128 in two 64-column blocks; row maxima of a and k ----
+        const uint8_t* ra = rawA + buf * 16384;
+        const uint8_t* rk = rawK + buf * 16384;
+#pragma unroll
+        for (int rep = 0; rep < 2; ++rep) {
+            const int cid = tid + kScanThreads * rep;      // 1024 16-byte chunks of the rows
+            const int j = cid >> 4, cc = cid & 15;
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (j < n) raw = *reinterpret_cast<const uint4*>(ra + j * 256 + cc * 16);
+            const float wj = swc[j];
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            uint4 hi, lo;
+            uint32_t* hw = reinterpret_cast<uint32_t*>(&hi);
+            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+            float mx = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(a2[i]);
+                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+                const float x0 = wj * f.x, x1 = wj * f.y;
+                const __half2 h2 = __floats2half2_rn(x0, x1);
+                const float2 hb = __half22float2(h2);
+                hw[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                lw[i] = pack_half2(x0 - hb.x, x1 - hb.y);
+            }
+            const uint32_t off = (uint32_t)((cc >> 3) * 8192 + j * 128 + (((cc & 7) ^ (j & 7)) << 4));
+            *reinterpret_cast<uint4*>(Ahi + off) = hi;
+            *reinterpret_cast<uint4*>(Alo + off) = lo;
+            // row max over the 16 threads (same half-warp) that hold row j
+#pragma unroll
+            for (int o2 = 8; o2 >= 1; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+            if (cc == 0) amax[j] = mx;
+            uint4 kr = raw;
+            if (m) {   // key rows: the B operand and the key row maxima for the value-state bound
+                kr = make_uint4(0, 0, 0, 0);
+                if (j < n) kr = *reinterpret_cast<const uint4*>(rk + j * 256 + cc * 16);
+                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+                float km = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(k2[i]);
+                    km = fmaxf(km, fmaxf(fabsf(f.x), fabsf(f.y)));
+                }
+#pragma unroll
+                for (int o2 = 8; o2 >= 1; o2 >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o2));
+                if (cc == 0) kmax[j] = km;
+            }
+            *reinterpret_cast<uint4*>(Bk + off) = bf16x8_to_f16x8(kr, 1.f);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();                          // images written; every thread's last TMEM read done
+        tc_fence_after();
+        if (tid == 0) {
+            if (c + 2 < nc) prefetch(c + 2);       // raw buffer `buf` is consumed
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t ko = ((ks & 3) * 2048) >> 4;
+                mma_f16(tbase, (ks < 4 ? dAhi : dAlo) + ko, dB + ko, kIdesc, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_mma);
+            mma_out = true;
+        }
+        if (w == 1 && c + 1 < nc) chunk_gates(c + 1);
+        // bound update: every warp reduces the same 64 terms in the same order,
+        // so every thread gets the same value
+        {
+            const float* km = m ? kmax : amax;
+            float add = swc[lane] * (amax[lane] * km[lane]) + swc[lane + 32] * (amax[lane + 32] * km[lane + 32]);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) add += __shfl_xor_sync(0xffffffffu, add, off);
+            bound = fmaf(expf(blast), bound, add);
+        }
+        if (tid == 0) {
+            if (mbar_wait(bar_mma, mma_phase & 1)) {
+                ++mma_phase;
+                mma_out = false;
+            } else {
+                red[31] = 1.f;
+            }
+        }
+        __syncthreads();                          // MMA done; gates of chunk c + 1 written
+        tc_fence_after();
+        if (red[31] != 0.f) {
+            ok = false;
+            break;
+        }
+        // ---- S <- e^{b_last} S + Delta ----
+        const float Gam = expf(blast);
+        float dv[32];
+        tmem_ld32_x32(tbase + ((uint32_t)(32 * q4) << 16) + col0, dv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) S[i] = fmaf(Gam, S[i], dv[i]);
+    }
+    if (!ok && tid == 0) {
+        record_error(err, kErrTimeout);
+        // one more bounded chance for the MMA and the row copies in flight to drain
+        if (mma_out) mbar_wait(bar_mma, mma_phase & 1);
+        for (int cc = c; cc < prefetched; ++cc) mbar_wait(bar_raw + (cc & 1), (cc >> 1) & 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tbase, 128);
+}
+
+}  // namespace
+
+cudaError_t tc_scan_launch(const ForwardArgs& a, void* img, float* scales, unsigned* err, cudaStream_t st) {
+    const int nc = (a.T + kC - 1) / kC;
+    const int smem = ScanSmem::bytes + 1024;
+    const cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    LaunchTimer timer(kKindTcScan, st);
+    tc_scan_kernel<<<dim3(2, a.B * a.H), kScanThreads, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.T, nc,
+        a.H_in, a.G_in, static_cast<__half*>(img), scales, a.H_out, a.G_out, err);
+    return cudaGetLastError();
+}
+
+}  // namespace mesa
