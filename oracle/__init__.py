@@ -55,8 +55,10 @@ def _configure(lib):
     lib.oracle_step_warm.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, D, i, d, D, I32]
     lib.oracle_cg_dense.argtypes = [i, D, D, D, i, d, D, I32]
     lib.oracle_preprocess.argtypes = [D, D, i, i, i, i, i, D]
+    lib.oracle_backward.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, D, D, D, D, I32, I32]
     for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
-              lib.oracle_step, lib.oracle_step_warm, lib.oracle_cg_dense, lib.oracle_preprocess):
+              lib.oracle_step, lib.oracle_step_warm, lib.oracle_cg_dense, lib.oracle_preprocess,
+              lib.oracle_backward):
         f.restype = ctypes.c_int
     return lib
 
@@ -182,3 +184,20 @@ def preprocess(x, conv):
     rc = _load().oracle_preprocess(_ptr(x), _ptr(conv), B, H, T, dd, W, _ptr(y))
     _check(rc, "oracle_preprocess")
     return y
+
+
+def backward(q, k, v, gamma, beta, lam, dout, cg_steps, tol=0.0):
+    """Gradients of L = sum(dout * o) through the layer (zero initial states),
+    by implicit differentiation with an adjoint CG solve under the same rule.
+    Returns a dict with dq, dk, dv, dgamma, dbeta, dlambda, iters_fwd, iters_adj."""
+    q, k, v, gamma, beta, lam, dout = map(_f64, (q, k, v, gamma, beta, lam, dout))
+    B, H, T, dk, dv = _shapes(q, v)
+    r = {"dq": np.zeros((B, H, T, dk)), "dk": np.zeros((B, H, T, dk)), "dv": np.zeros((B, H, T, dv)),
+         "dgamma": np.zeros((B, H, T)), "dbeta": np.zeros((B, H, T)), "dlambda": np.zeros((H, dk)),
+         "iters_fwd": np.zeros((B, H, T), dtype=np.int32), "iters_adj": np.zeros((B, H, T), dtype=np.int32)}
+    rc = _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                 B, H, T, dk, dv, int(cg_steps), float(tol), _ptr(dout),
+                                 _ptr(r["dq"]), _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dgamma"]), _ptr(r["dbeta"]),
+                                 _ptr(r["dlambda"]), _ptr(r["iters_fwd"]), _ptr(r["iters_adj"]))
+    _check(rc, "oracle_backward")
+    return r

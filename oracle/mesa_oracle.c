@@ -458,3 +458,140 @@ int oracle_step_warm(const double* q, const double* k, const double* v,
     }
     return err ? -2 : 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass: gradients of a scalar loss L through o_t = G_t x_t         */
+/* ------------------------------------------------------------------------ */
+/*
+ * The pages claim the layer trains in time linear in T but give no backward
+ * method. Reading taken here: implicit differentiation of the solution map
+ * x_t = (H_t + Lambda)^-1 q_t, the adjoint system solved by the same CG rule
+ * (same step count; the stopping test relative to its own right-hand side).
+ * Given do_t = dL/do_t (tokens t = 0..T-1, zero initial states):
+ *   dG_t = do_t x_t^T                     (o_t = G_t x_t)
+ *   u_t  = CG_N(H_t + Lambda, G_t^T do_t)  (adjoint; exactly A_t^-1 G_t^T do_t)
+ *   dq_t = u_t,   dH_t = -u_t x_t^T,   dlambda_i += -u_ti x_ti
+ * then back through the recurrences H_t = gamma_t H_{t-1} + beta_t k_t k_t^T
+ * and G_t = gamma_t G_{t-1} + beta_t v_t k_t^T with the running totals
+ *   Hbar_t = dH_t + gamma_{t+1} Hbar_{t+1},   Gbar_t = dG_t + gamma_{t+1} Gbar_{t+1}:
+ *   dbeta_t  = k_t^T Hbar_t k_t + v_t^T Gbar_t k_t
+ *   dk_t     = beta_t (Hbar_t + Hbar_t^T) k_t + beta_t Gbar_t^T v_t
+ *   dv_t     = beta_t Gbar_t k_t
+ *   dgamma_t = <Hbar_t, H_{t-1}> + <Gbar_t, G_{t-1}>      (Frobenius products)
+ * When CG has converged this is the exact gradient of the layer. The states
+ * H_t and G_t are kept for every t (memory (T+1)(dk^2 + dv dk) doubles per
+ * sequence).
+ */
+int oracle_backward(const double* q, const double* k, const double* v,
+                    const double* gamma, const double* beta, const double* lambda,
+                    int B, int H, int T, int dk, int dv, int cg_steps, double tol, const double* dout,
+                    double* dq, double* dk_out, double* dv_out, double* dgamma, double* dbeta,
+                    double* dlambda, int32_t* iters_fwd, int32_t* iters_adj) {
+    if (bad_dims(B, H, T, dk, dv) || cg_steps < 0 || !lambda || !dlambda) return -1;
+    if (T > 0 && (!q || !k || !v || !gamma || !beta || !dout || !dq || !dk_out || !dv_out || !dgamma || !dbeta))
+        return -1;
+    const int BH = B * H;
+    const size_t SH = (size_t)dk * dk, SG = (size_t)dv * dk;
+    double* part = (double*)calloc((size_t)(BH > 0 ? BH : 1) * dk, sizeof(double));   /* dlambda per sequence */
+    if (!part) return -2;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int bh = 0; bh < BH; ++bh) {
+        const int h = bh % H;
+        double* Hs = (double*)calloc((size_t)(T + 1) * SH, sizeof(double));    /* Hs[t] = state after t tokens */
+        double* Gs = (double*)calloc((size_t)(T + 1) * SG, sizeof(double));
+        double* X = (double*)malloc(sizeof(double) * ((size_t)T * dk + 1));
+        double* U = (double*)malloc(sizeof(double) * ((size_t)T * dk + 1));
+        double* A = (double*)malloc(sizeof(double) * SH);
+        double* g = (double*)malloc(sizeof(double) * (size_t)dk);
+        double* work = (double*)malloc(sizeof(double) * 3 * (size_t)dk);
+        double* Hbar = (double*)calloc(SH, sizeof(double));
+        double* Gbar = (double*)calloc(SG, sizeof(double));
+        if (!Hs || !Gs || !X || !U || !A || !g || !work || !Hbar || !Gbar) {
+            err |= 1;
+        } else {
+            /* forward in time: states, x_t and the adjoint u_t */
+            for (int t = 0; t < T; ++t) {
+                const size_t bt = (size_t)bh * T + t;
+                double* Hm = Hs + (size_t)(t + 1) * SH;
+                double* Gm = Gs + (size_t)(t + 1) * SG;
+                memcpy(Hm, Hs + (size_t)t * SH, sizeof(double) * SH);
+                memcpy(Gm, Gs + (size_t)t * SG, sizeof(double) * SG);
+                update_state(dk, dv, gamma[bt], beta[bt], k + bt * dk, v + bt * dv, Hm, Gm);
+                for (int i = 0; i < dk; ++i) {
+                    for (int j = 0; j < dk; ++j) A[(size_t)i * dk + j] = Hm[(size_t)i * dk + j];
+                    A[(size_t)i * dk + i] += lambda[(size_t)h * dk + i];
+                }
+                dense_ctx c = {dk, A};
+                double* xt = X + (size_t)t * dk;
+                double* ut = U + (size_t)t * dk;
+                const int itf = cg_generic(dk, dense_mv, &c, q + bt * dk, cg_steps, tol, xt, work);
+                /* right-hand side of the adjoint system: G_t^T do_t */
+                const double* dot_ = dout + bt * dv;
+                for (int j = 0; j < dk; ++j) {
+                    double s = 0.0;
+                    for (int i = 0; i < dv; ++i) s += Gm[(size_t)i * dk + j] * dot_[i];
+                    g[j] = s;
+                }
+                const int ita = cg_generic(dk, dense_mv, &c, g, cg_steps, tol, ut, work);
+                if (iters_fwd) iters_fwd[bt] = itf;
+                if (iters_adj) iters_adj[bt] = ita;
+                for (int i = 0; i < dk; ++i) {
+                    dq[bt * dk + i] = ut[i];
+                    part[(size_t)bh * dk + i] -= ut[i] * xt[i];
+                }
+            }
+            /* backward in time through the recurrences */
+            for (int t = T - 1; t >= 0; --t) {
+                const size_t bt = (size_t)bh * T + t;
+                const double* kt = k + bt * dk;
+                const double* vt = v + bt * dv;
+                const double* xt = X + (size_t)t * dk;
+                const double* ut = U + (size_t)t * dk;
+                const double* dot_ = dout + bt * dv;
+                const double gnext = (t + 1 < T) ? gamma[bt + 1] : 0.0;
+                for (size_t e = 0; e < SH; ++e) Hbar[e] *= gnext;
+                for (size_t e = 0; e < SG; ++e) Gbar[e] *= gnext;
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dk; ++j) Hbar[(size_t)i * dk + j] -= ut[i] * xt[j];
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j) Gbar[(size_t)i * dk + j] += dot_[i] * xt[j];
+                const double bta = beta[bt];
+                double db = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dk; ++j) db += kt[i] * Hbar[(size_t)i * dk + j] * kt[j];
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j) db += vt[i] * Gbar[(size_t)i * dk + j] * kt[j];
+                dbeta[bt] = db;
+                for (int i = 0; i < dk; ++i) {
+                    double s = 0.0;
+                    for (int j = 0; j < dk; ++j) s += (Hbar[(size_t)i * dk + j] + Hbar[(size_t)j * dk + i]) * kt[j];
+                    for (int l = 0; l < dv; ++l) s += Gbar[(size_t)l * dk + i] * vt[l];
+                    dk_out[bt * dk + i] = bta * s;
+                }
+                for (int l = 0; l < dv; ++l) {
+                    double s = 0.0;
+                    for (int j = 0; j < dk; ++j) s += Gbar[(size_t)l * dk + j] * kt[j];
+                    dv_out[bt * dv + l] = bta * s;
+                }
+                const double* Hprev = Hs + (size_t)t * SH;
+                const double* Gprev = Gs + (size_t)t * SG;
+                double dg = 0.0;
+                for (size_t e = 0; e < SH; ++e) dg += Hbar[e] * Hprev[e];
+                for (size_t e = 0; e < SG; ++e) dg += Gbar[e] * Gprev[e];
+                dgamma[bt] = dg;
+            }
+        }
+        free(Hs); free(Gs); free(X); free(U); free(A); free(g); free(work); free(Hbar); free(Gbar);
+    }
+    if (!err) {   /* dlambda[h] = sum over the batch, in batch order */
+        for (int h = 0; h < H; ++h)
+            for (int i = 0; i < dk; ++i) {
+                double s = 0.0;
+                for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * dk + i];
+                dlambda[(size_t)h * dk + i] = s;
+            }
+    }
+    free(part);
+    return err ? -2 : 0;
+}

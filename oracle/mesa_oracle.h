@@ -77,6 +77,18 @@ int oracle_step_warm(const double* q, const double* k, const double* v,
 int oracle_cg_dense(int n, const double* A, const double* b, const double* x0, int cg_steps, double tol,
                     double* x, int32_t* iters);
 
+/* Backward pass (reading: implicit differentiation of x_t = (H_t+Lambda)^-1 q_t,
+ * adjoint u_t = CG_N(H_t + Lambda, G_t^T do_t) under the same CG rule) for
+ * zero initial states. dout [B,H,T,dv] is dL/do. Outputs: dq, dk [B,H,T,dk];
+ * dv [B,H,T,dv]; dgamma, dbeta [B,H,T]; dlambda [H,dk] (summed over the
+ * batch); iters_fwd / iters_adj [B,H,T] (NULL allowed): CG updates of the
+ * forward and the adjoint solve. */
+int oracle_backward(const double* q, const double* k, const double* v,
+                    const double* gamma, const double* beta, const double* lambda,
+                    int B, int H, int T, int dk, int dv, int cg_steps, double tol, const double* dout,
+                    double* dq, double* dk_out, double* dv_out, double* dgamma, double* dbeta,
+                    double* dlambda, int32_t* iters_fwd, int32_t* iters_adj);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,19 @@ MUTANTS = {
     "warm stopping test relative to the first residual": ("const double bnorm = sqrt(dot(n, b, b));",
                                                           "const double bnorm = sqrt(rr);"),
     "preprocessing norm left out": ("const double inv = 1.0 / (nrm > 1e-6 ? nrm : 1e-6);", "const double inv = 1.0;"),
+    "backward dk without the transposed H total": (
+        "s += (Hbar[(size_t)i * dk + j] + Hbar[(size_t)j * dk + i]) * kt[j];",
+        "s += 2.0 * Hbar[(size_t)i * dk + j] * kt[j];"),
+    "backward dgamma against the state after the token": ("const double* Hprev = Hs + (size_t)t * SH;",
+                                                          "const double* Hprev = Hs + (size_t)(t + 1) * SH;"),
+    "backward totals not decayed": ("const double gnext = (t + 1 < T) ? gamma[bt + 1] : 0.0;",
+                                    "const double gnext = (t + 1 < T) ? 1.0 : 0.0;"),
+    "backward dlambda sign": ("part[(size_t)bh * dk + i] -= ut[i] * xt[i];",
+                              "part[(size_t)bh * dk + i] += ut[i] * xt[i];"),
+    "adjoint right-hand side G do instead of G^T do": ("for (int i = 0; i < dv; ++i) s += Gm[(size_t)i * dk + j] * dot_[i];",
+                                                       "for (int i = 0; i < dv; ++i) s += Gm[(size_t)j * dk + i] * dot_[i];"),
+    "backward dlambda from one batch row only": ("for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * dk + i];",
+                                                 "for (int b = 0; b < 1; ++b) s += part[((size_t)b * H + h) * dk + i];"),
 }
 
 
@@ -95,6 +108,8 @@ PIN_SUBSET = [
     lambda o: pins.test_preprocess_causal_and_scale_invariant(o),
     lambda o: pins.test_warm_cg_equals_shifted_cold_cg(o),
     lambda o: pins.test_warm_cg_from_the_solution_stops_at_once(o),
+    lambda o: pins.test_backward_matches_finite_differences_of_the_exact_layer(o),
+    lambda o: pins.test_backward_one_step_closed_form(o),
 ]
 
 

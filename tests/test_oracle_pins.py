@@ -444,3 +444,86 @@ def test_warm_step_from_zero_is_the_cold_step(oracle_mod):
         assert np.array_equal(a, b_)
     # the returned x reproduces the output through the updated G
     assert np.allclose(np.einsum("bhij,bhj->bhi", warm[3], warm[4]), warm[0], atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Backward pass (implicit differentiation with an adjoint CG solve)
+# --------------------------------------------------------------------------
+
+def _bwd_inputs(seed, B=2, H=2, T=4, d=3):
+    rng = np.random.default_rng(seed)
+    q, k, v, _, _, _ = rand_inputs(rng, B, H, T, d, d)
+    gamma = rng.uniform(0.5, 1.0, (B, H, T))
+    beta = rng.uniform(0.2, 1.0, (B, H, T))
+    lam = rng.uniform(0.3, 1.3, (H, d))
+    dout = rng.standard_normal((B, H, T, d))
+    return {"q": q, "k": k, "v": v, "gamma": gamma, "beta": beta, "lam": lam}, dout
+
+
+def _exact_loss(oracle_mod, x, dout):
+    o, _, _ = oracle_mod.forward_cholesky(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"])
+    return float(np.sum(o * dout))
+
+
+def test_backward_matches_finite_differences_of_the_exact_layer(oracle_mod):
+    """With CG run to convergence, the implicit gradient is the gradient of
+    the exact layer: central differences of L = sum(dout * o), o from the
+    Cholesky forward (code the backward does not use)."""
+    x, dout = _bwd_inputs(0)
+    d = x["q"].shape[-1]
+    g = oracle_mod.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], dout, 3 * d, 1e-13)
+    h = 1e-6
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("gamma", "dgamma"), ("beta", "dbeta"),
+                      ("lam", "dlambda")):
+        a = x[name]
+        num = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            xp = dict(x)
+            xp[name] = a.copy()
+            xp[name][idx] += h
+            lp = _exact_loss(oracle_mod, xp, dout)
+            xp[name][idx] -= 2 * h
+            lm = _exact_loss(oracle_mod, xp, dout)
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[key], num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_backward_adjoint_solves_converge_like_the_forward(oracle_mod):
+    """The adjoint solves use the same CG rule: with tol > 0 every adjoint
+    count stays within [1, cg_steps], and with a tiny step budget both solves
+    take exactly that many updates."""
+    x, dout = _bwd_inputs(1, B=1, H=1, T=6, d=4)
+    g = oracle_mod.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], dout, 12, 1e-10)
+    assert g["iters_adj"].min() >= 1 and g["iters_adj"].max() <= 12
+    g2 = oracle_mod.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], dout, 2, 0.0)
+    assert (g2["iters_fwd"] == 2).all() and (g2["iters_adj"] == 2).all()
+
+
+def test_backward_one_step_closed_form(oracle_mod):
+    """One CG step gives x = (q.q / q.Aq) q and u = (g.g / g.Ag) g with
+    g = G^T do; on a single token (H = beta k k^T, G = beta v k^T) every
+    gradient then follows from the definitions in closed form."""
+    rng = np.random.default_rng(5)
+    d = 4
+    q = rng.standard_normal(d)
+    k = rng.standard_normal(d)
+    k /= np.linalg.norm(k)
+    v = rng.standard_normal(d)
+    do = rng.standard_normal(d)
+    gam, bet = 0.8, 0.6
+    lam = rng.uniform(0.3, 1.3, d)
+    A = bet * np.outer(k, k) + np.diag(lam)
+    G = bet * np.outer(v, k)
+    x = (q @ q) / (q @ A @ q) * q
+    gv = G.T @ do
+    u = (gv @ gv) / (gv @ A @ gv) * gv
+    Hbar = -np.outer(u, x)
+    Gbar = np.outer(do, x)
+    r = oracle_mod.backward(q[None, None, None], k[None, None, None], v[None, None, None],
+                            np.array([[[gam]]]), np.array([[[bet]]]), lam[None], do[None, None, None], 1, 0.0)
+    np.testing.assert_allclose(r["dq"][0, 0, 0], u, rtol=1e-12)
+    np.testing.assert_allclose(r["dlambda"][0], -u * x, rtol=1e-12)
+    np.testing.assert_allclose(r["dv"][0, 0, 0], bet * Gbar @ k, rtol=1e-12)
+    np.testing.assert_allclose(r["dk"][0, 0, 0], bet * ((Hbar + Hbar.T) @ k + Gbar.T @ v), rtol=1e-12)
+    np.testing.assert_allclose(r["dbeta"][0, 0, 0], k @ Hbar @ k + v @ Gbar @ k, rtol=1e-12)
+    assert r["dgamma"][0, 0, 0] == 0.0              # the state before the first token is zero
