@@ -206,6 +206,7 @@ def run_reference(args, w, rank):
 
 METRIC = "Mesa-layer fwd tokens/s (B*H*T) at T=8192,d=128,15 CG steps; % tensor peak"
 DECODE_METRIC = "Mesa decode tokens/s (sequences x heads per mesa_step), d=128, 15 CG steps; % HBM peak"
+BWD_METRIC = "Mesa-layer bwd tokens/s (B*H*T): implicit-differentiation backward, d=128, 15 CG steps; % fp32 FMA peak"
 PRE_METRIC = "Mesa input preprocessing tokens/s (q and k: causal depthwise conv, window 4, + L2 norm); % HBM peak"
 
 
@@ -400,6 +401,99 @@ def run_preprocess(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# Useful flops per token of each backward kernel (d, chunk C, N CG steps):
+# a CG matvec or a read-out-shaped product counts 2d^2 + 2d(C+1) (the causal
+# intra-chunk terms j <= t only), a chunk-state update 2 d^2 per matrix.
+def bwd_flops_per_token(d, C, N):
+    mv = 2 * d * d + 2 * d * (C + 1)
+    return {"simt_scan": 4 * d * d, "simt_cg": N * mv, "bwd_adjoint": (N + 2) * mv,
+            "bwd_rscan": 4 * d * d, "bwd_grad": 8 * d * d + 8 * d * (C + 1)}
+
+
+def fp32_fma_peak_tflops(sm_mhz):
+    """148 SMs x 128 fp32 lanes x 2 flops per FMA x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_backward(args, w, world, rank, local):
+    """mesa_backward on the workload's shape with device-resident inputs and a
+    seeded upstream gradient: forward solve, adjoint solve, reverse scan and
+    gradient kernels, all fp32 on the CUDA cores."""
+    import torch
+    import torch.distributed as dist
+    from test_sequence_layer_b200 import build as mbuild, mesa
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    x = mi.device_batch(w, dev, seed_offset=rank)
+    g = torch.Generator(device=dev).manual_seed(17 + rank)
+    do = torch.randn((w.B, w.H, w.T, w.dv), generator=g, device=dev)
+    ws = torch.empty(int(mesa._load().mesa_backward_workspace_size(w.B, w.H, w.T, w.dk, w.dv, w.chunk,
+                                                                    1 if w.dtype == "bf16" else 0)),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    N = w.cg_steps
+
+    def step():
+        mesa.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], do, chunk=w.chunk, cg_steps=N,
+                      tol=w.tol, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    mesa.timing_enable(False)
+    kernels = mesa.timing_read()
+    clk = clocks.stop()
+    assert mesa.get_error() == 0
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    tokens = w.B * w.H * w.T
+    fl = bwd_flops_per_token(w.dk, w.chunk, N)
+    top = max((k for k in kernels if k in fl), key=lambda k: kernels[k][1])
+    launches, kms = kernels[top]
+    avg_ms = kms / launches
+    achieved = fl[top] * tokens / (avg_ms / 1e3) / 1e12
+    peak = fp32_fma_peak_tflops(1965.0)
+    line = {
+        "metric": BWD_METRIC, "value": whole_job_rate(tokens, world, ms / args.steps), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": ("bf16-in/" if w.dtype == "bf16" else "") + "f32", "data": "synthetic",
+        "config": {"workload": w.name + "+backward", "B": w.B, "H": w.H, "T": w.T, "d": w.dk, "chunk": w.chunk,
+                   "cg_steps": N, "tol": w.tol, "flops_per_token": sum(fl.values()),
+                   "l2": "inputs larger than L2 (%.2f GB per step)" % (
+                       (3 * x["q"].numel() * x["q"].element_size() + do.numel() * 4) / 1e9)},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": top, "avg_ms": avg_ms,
+                     "peak_kind": "derived fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz"},
+        "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
+        "gpu_launches": sum(v[0] for v in kernels.values()),
+        "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -411,6 +505,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--preprocess", action="store_true",
                     help="time mesa_preprocess (q/k convolution + normalisation) on the workload's shape")
+    ap.add_argument("--backward", action="store_true",
+                    help="time mesa_backward (implicit-differentiation gradients) on the workload's shape")
     ap.add_argument("--warm-start", action="store_true",
                     help="decode: start each step's CG from the previous step's solution (mesa_step_warm)")
     ap.add_argument("--tol", type=float, default=None, help="override the workload's CG tolerance")
@@ -432,6 +528,9 @@ def main():
         return
     if args.preprocess:
         run_preprocess(args, w, world, rank, local)
+        return
+    if args.backward:
+        run_backward(args, w, world, rank, local)
         return
     if w.decode_steps > 0:
         run_decode(args, w, world, rank, local)

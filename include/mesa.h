@@ -171,6 +171,46 @@ mesa_status mesa_preprocess(const void* q_raw, const void* k_raw, const float* c
                             void* stream);
 
 /*
+ * Backward pass of the layer (training): gradients of a scalar loss L given
+ * dout = dL/do for the inputs of a mesa_forward call with zero initial
+ * states. The pages claim training in time linear in T but give no backward
+ * method; the reading implemented is implicit differentiation of the
+ * solution map x_t = (H_t + Lambda)^-1 q_t, with the adjoint system
+ *     u_t = CG(H_t + Lambda, G_t^T dout_t)
+ * solved under the same CG rule as the forward (same cg_steps; the tolerance
+ * test relative to |G_t^T dout_t|). Then dq_t = u_t, dlambda_i = -sum u_ti x_ti,
+ * and back through the gated recurrences of H and G (with
+ * Hbar_t = -sum_{t'>=t} (prod gamma) u_t' x_t'^T and
+ * Gbar_t = sum_{t'>=t} (prod gamma) dout_t' x_t'^T):
+ *     dk_t = beta_t ((Hbar_t + Hbar_t^T) k_t + Gbar_t^T v_t),  dv_t = beta_t Gbar_t k_t,
+ *     dbeta_t = k_t^T Hbar_t k_t + v_t^T Gbar_t k_t,
+ *     dgamma_t = <Hbar_t, H_{t-1}> + <Gbar_t, G_{t-1}>.
+ * When CG has converged this is the exact gradient of the layer.
+ *
+ *   q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps,
+ *                tol: as in mesa_forward (every supported shape and dtype;
+ *                the arithmetic is fp32 on the CUDA cores for every dtype).
+ *   dout         float32 [B,H,T,dv].
+ *   dq, dk_out   float32 [B,H,T,dk];  dv_out float32 [B,H,T,dv].
+ *   dgamma, dbeta float32 [B,H,T].    dlambda float32 [H,dk] (summed over
+ *                the batch).
+ *   workspace    device memory of at least mesa_backward_workspace_size()
+ *                bytes, 256-byte aligned (it holds the chunk states, the
+ *                forward solutions and the reverse gradient states).
+ * All pointers are DEVICE pointers, 16-byte aligned (gamma, beta, lambda,
+ * dgamma, dbeta, dlambda 4-byte aligned); the outputs must not overlap the
+ * inputs. Asynchronous on `stream`. T = 0 writes zeros to dlambda only.
+ */
+size_t mesa_backward_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype);
+
+mesa_status mesa_backward(const void* q, const void* k, const void* v,
+                          const float* gamma, const float* beta, const float* lambda,
+                          int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                          int cg_steps, float tol, const float* dout,
+                          float* dq, float* dk_out, float* dv_out, float* dgamma, float* dbeta, float* dlambda,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Bytes of device workspace mesa_forward_host needs: the mesa_forward
  * workspace plus device staging for every tensor argument.
  */

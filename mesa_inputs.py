@@ -190,3 +190,18 @@ def plant_sequences(dev: dict, w: Workload, pairs, T: int | None = None):
         dev["gamma"][b, h].copy_(torch.from_numpy(host["gamma"][0, i]))
         dev["beta"][b, h].copy_(torch.from_numpy(host["beta"][0, i]))
     return host
+
+
+DOUT_STREAM = 0x444F5554
+
+
+def dout(seed: int, B: int, H: int, T: int, dv: int, seqs=None) -> np.ndarray:
+    """Upstream gradient dL/do for backward runs: standard normal float32,
+    one stream per (b, h) keyed by SeedSequence([seed, DOUT_STREAM, b, h]).
+    Shape [B,H,T,dv], or [1,len(seqs),T,dv] for a list of (b, h) pairs."""
+    pairs = [(b, h) for b in range(B) for h in range(H)] if seqs is None else list(seqs)
+    out = np.empty((len(pairs), T, dv), np.float32)
+    for i, (b, h) in enumerate(pairs):
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, DOUT_STREAM, b, h])))
+        out[i] = rng.standard_normal((T, dv), dtype=np.float32)
+    return out.reshape(B, H, T, dv) if seqs is None else out[None]

@@ -69,7 +69,7 @@ mesa_status launch_forward(const ForwardArgs& a, cudaStream_t st) {
 
 // ---- kernel timing records ----
 const char* const kKindNames[kKindCount] = {"simt_scan", "simt_cg", "decode_step", "tc_scan", "tc_cg",
-                                             "preprocess"};
+                                             "preprocess", "bwd_adjoint", "bwd_rscan", "bwd_grad", "bwd_reduce"};
 struct TimingRec {
     int kind;
     cudaEvent_t start, stop;
@@ -221,6 +221,54 @@ mesa_status mesa_forward(const void* q, const void* k, const void* v,
     ForwardArgs a{q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps, tol,
                   out, iters_out, H_in, G_in, H_out, G_out, workspace, ws_bytes};
     return launch_forward(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t mesa_backward_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
+    if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
+    return backward_workspace_bytes(B, H, T, dk, dv, chunk);
+}
+
+mesa_status mesa_backward(const void* q, const void* k, const void* v,
+                          const float* gamma, const float* beta, const float* lambda,
+                          int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                          int cg_steps, float tol, const float* dout,
+                          float* dq, float* dk_out, float* dv_out, float* dgamma, float* dbeta, float* dlambda,
+                          void* workspace, size_t ws_bytes, void* stream) {
+    mesa_status s = check_shape(B, H, T, dk, dv, chunk, dtype, cg_steps, tol);
+    if (s != MESA_OK) return s;
+    if (!lambda || !dlambda || !aligned(lambda, 4) || !aligned(dlambda, 4)) return MESA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return cudaMemsetAsync(dlambda, 0, (size_t)H * dk * sizeof(float), st) == cudaSuccess
+                           ? MESA_OK : MESA_ERR_CUDA;
+    const void* in16[] = {q, k, v, dout};
+    const void* out16[] = {dq, dk_out, dv_out};
+    for (const void* p : in16)
+        if (!p || !aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    for (const void* p : out16)
+        if (!p || !aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)gamma, (const void*)beta, (const void*)dgamma, (const void*)dbeta})
+        if (!p || !aligned(p, 4)) return MESA_ERR_INVALID_ARG;
+    // no output may overlap an input or another output
+    const size_t tok = (size_t)B * H * T, es = elem_size(dtype);
+    struct Range { const char* p; size_t n; };
+    const Range ranges[] = {
+        {(const char*)q, tok * dk * es}, {(const char*)k, tok * dk * es}, {(const char*)v, tok * dv * es},
+        {(const char*)gamma, tok * 4}, {(const char*)beta, tok * 4}, {(const char*)lambda, (size_t)H * dk * 4},
+        {(const char*)dout, tok * dv * 4}, {(const char*)dq, tok * dk * 4}, {(const char*)dk_out, tok * dk * 4},
+        {(const char*)dv_out, tok * dv * 4}, {(const char*)dgamma, tok * 4}, {(const char*)dbeta, tok * 4},
+        {(const char*)dlambda, (size_t)H * dk * 4}};
+    constexpr int kFirstOut = 7, kRanges = 13;
+    for (int o = kFirstOut; o < kRanges; ++o)
+        for (int r = 0; r < kRanges; ++r)
+            if (r != o && ranges[o].p < ranges[r].p + ranges[r].n && ranges[r].p < ranges[o].p + ranges[o].n)
+                return MESA_ERR_INVALID_ARG;
+    const size_t need = backward_workspace_bytes(B, H, T, dk, dv, chunk);
+    if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
+    BackwardArgs a{{q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps, tol, nullptr, nullptr,
+                    nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes},
+                   dout, dq, dk_out, dv_out, dgamma, dbeta, dlambda};
+    return backward_simt(a, st) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
 }
 
 size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {

@@ -29,13 +29,28 @@ struct ForwardArgs {
     float* G_out;
     void* workspace;
     size_t ws_bytes;
+    float* x_out = nullptr;     // fp32 CUDA-core path only: the CG solutions x_t [B,H,T,dk]
+};
+
+struct BackwardArgs {
+    ForwardArgs f;              // the forward's inputs (out, iters, states unused)
+    const float* dout;          // dL/do [B,H,T,dv]
+    float* dq;                  // [B,H,T,dk]
+    float* dk;                  // [B,H,T,dk]
+    float* dv;                  // [B,H,T,dv]
+    float* dgamma;              // [B,H,T]
+    float* dbeta;               // [B,H,T]
+    float* dlambda;             // [H,dk]
 };
 
 // Device address of the calling device's error word (nullptr on failure).
 unsigned* error_word_ptr();
 
 // Kernel kinds for the optional timing records (mesa_timing_enable).
-enum KernelKind : int { kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindPre, kKindCount };
+enum KernelKind : int {
+    kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindPre,
+    kKindBwdAdj, kKindBwdRscan, kKindBwdGrad, kKindBwdReduce, kKindCount
+};
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
 class LaunchTimer {
@@ -53,6 +68,8 @@ class LaunchTimer {
 // fp32 CUDA-core path (simt_forward.cu).
 size_t simt_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
 cudaError_t forward_simt(const ForwardArgs& a, cudaStream_t st);
+size_t backward_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
+cudaError_t backward_simt(const BackwardArgs& a, cudaStream_t st);
 
 // Tensor-core path (tc_forward.cu): bf16 inputs, dk = dv = 128, chunk = 64.
 bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype);

@@ -22,37 +22,13 @@
 //   simt_cg_kernel    grid (chunks, B*H): one CTA runs all CG iterations of one
 //                     chunk with H_c, K, V, P and the decay mask in shared
 //                     memory, then the read-out.
-#include "mesa_common.cuh"
 #include "mesa_internal.h"
+#include "simt_chunk.cuh"
 
 namespace mesa {
 namespace {
 
-constexpr int kThreads = 256;
-
-// Inclusive log-cumsum of gamma over one chunk (padded tokens count as
-// gamma = 1), done by warp 0. Writes b[t] for t < CH.
-template <int CH>
-__device__ __forceinline__ void chunk_log_cumsum(const float* __restrict__ gamma, size_t base, int n,
-                                                 float* __restrict__ b) {
-    static_assert(CH <= 64, "chunk must be <= 64");
-    if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
-    const int t0 = 2 * lane, t1 = 2 * lane + 1;
-    const float l0 = (t0 < n) ? logf(gamma[base + t0]) : 0.f;
-    const float l1 = (t1 < n) ? logf(gamma[base + t1]) : 0.f;
-    float pair = l0 + l1;
-    // inclusive scan of the pair sums across the warp
-    float incl = pair;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-    }
-    const float excl = incl - pair;
-    if (t0 < CH) b[t0] = excl + l0;
-    if (t1 < CH) b[t1] = excl + l0 + l1;
-}
+using namespace simt;
 
 template <int DK, int DV, int CH, typename Tin>
 __global__ void __launch_bounds__(kThreads)
@@ -136,41 +112,16 @@ simt_scan_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v,
     }
 }
 
-// Sum over the 16 lanes of a half-warp (all 16 receive the total).
-__device__ __forceinline__ float sum16(float v) {
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    return v;
-}
-
-template <int DK, int DV, int CH>
-struct CgSmem {
-    static constexpr int DKP = DK + 1, DVP = DV + 1, CHP = CH + 1;
-    static constexpr int MAXR = DK > DV ? DK : DV;
-    static constexpr int oH = 0;                       // H_c, later G_c   [MAXR][DKP]
-    static constexpr int oK = oH + MAXR * DKP;         // keys            [CH][DKP]
-    static constexpr int oP = oK + CH * DKP;           // CG direction, later x [CH][DKP]
-    static constexpr int oV = oP + CH * DKP;           // values          [CH][DVP]
-    static constexpr int oW = oV + CH * DVP;           // masked scores   [CH][CHP]
-    static constexpr int oM = oW + CH * CHP;           // decay mask      [CH][CHP]
-    static constexpr int oE = oM + CH * CHP;           // e^{b_t}         [CH]
-    static constexpr int oB = oE + CH;                 // b_t             [CH]
-    static constexpr int oL = oB + CH;                 // lambda          [DK]
-    static constexpr int total = oL + DK;
-    static constexpr size_t bytes = sizeof(float) * (size_t)total;
-};
-
 template <int DK, int DV, int CH, typename Tin>
 __global__ void __launch_bounds__(kThreads, 1)
 simt_cg_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                const float* __restrict__ gamma, const float* __restrict__ beta,
                const float* __restrict__ lambda, int H, int T, int nc, int cg_steps, float tol,
-               const float* __restrict__ states, float* __restrict__ out, int32_t* __restrict__ iters) {
+               const float* __restrict__ states, float* __restrict__ out, int32_t* __restrict__ iters,
+               float* __restrict__ x_out) {
     static_assert(DK % 16 == 0 && DV % 16 == 0 && CH % 16 == 0, "multiples of 16");
     using L = CgSmem<DK, DV, CH>;
-    constexpr int TP = CH / 16, IP = DK / 16, VP = DV / 16, JP = CH / 16;
+    constexpr int TP = CH / 16, IP = DK / 16, VP = DV / 16;
     constexpr int DKP = L::DKP, DVP = L::DVP, CHP = L::CHP;
     constexpr size_t SE = (size_t)DK * DK + (size_t)DV * DK;
     extern __shared__ float smem[];
@@ -212,7 +163,7 @@ simt_cg_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* 
     }
 
     // ---- CG init: x = 0, r = p = q ----
-    float x[TP][IP], r[TP][IP], p[TP][IP], y[TP][IP];
+    float x[TP][IP], r[TP][IP], p[TP][IP];
     float rr[TP], qn[TP];
     bool act[TP];
     int it[TP];
@@ -237,119 +188,29 @@ simt_cg_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* 
     }
     __syncthreads();
 
-    for (int step = 0; step < cg_steps; ++step) {
-        bool any = false;
+    chunk_cg<DK, CH>(sP, sH, sK, sW, sM, sE, sL, x, r, p, rr, qn, act, it, cg_steps, tol);
+
+    // ---- the solution, if asked for, then the read-out o = e^{b_t} G_c x + (M (.) X K^T) V ----
+    if (x_out) {
 #pragma unroll
         for (int a = 0; a < TP; ++a) {
-            act[a] = act[a] && cg_may_continue(rr[a], qn[a], tol);
-            any |= act[a];
-        }
-        if (!__syncthreads_or(any)) break;
-
-        // S = P K^T, W = M (.) S
-        {
-            float s[TP][JP];
+            const int t = tt + 16 * a;
+            if (t < n) {
 #pragma unroll
-            for (int a = 0; a < TP; ++a)
-#pragma unroll
-                for (int b = 0; b < JP; ++b) s[a][b] = 0.f;
-#pragma unroll 4
-            for (int kk = 0; kk < DK; ++kk) {
-                float pv[TP], kv[JP];
-#pragma unroll
-                for (int a = 0; a < TP; ++a) pv[a] = sP[(tt + 16 * a) * DKP + kk];
-#pragma unroll
-                for (int b = 0; b < JP; ++b) kv[b] = sK[(ti + 16 * b) * DKP + kk];
-#pragma unroll
-                for (int a = 0; a < TP; ++a)
-#pragma unroll
-                    for (int b = 0; b < JP; ++b) s[a][b] = fmaf(pv[a], kv[b], s[a][b]);
-            }
-#pragma unroll
-            for (int a = 0; a < TP; ++a)
-#pragma unroll
-                for (int b = 0; b < JP; ++b) {
-                    const int t = tt + 16 * a, j = ti + 16 * b;
-                    sW[t * CHP + j] = sM[t * CHP + j] * s[a][b];
-                }
-        }
-        __syncthreads();
-
-        // y = e^{b_t} H_c p + W K + lambda p
-#pragma unroll
-        for (int a = 0; a < TP; ++a)
-#pragma unroll
-            for (int b = 0; b < IP; ++b) y[a][b] = 0.f;
-#pragma unroll 4
-        for (int kk = 0; kk < DK; ++kk) {
-            float pv[TP], hv[IP];
-#pragma unroll
-            for (int a = 0; a < TP; ++a) pv[a] = sP[(tt + 16 * a) * DKP + kk];
-#pragma unroll
-            for (int b = 0; b < IP; ++b) hv[b] = sH[(ti + 16 * b) * DKP + kk];
-#pragma unroll
-            for (int a = 0; a < TP; ++a)
-#pragma unroll
-                for (int b = 0; b < IP; ++b) y[a][b] = fmaf(pv[a], hv[b], y[a][b]);
-        }
-#pragma unroll
-        for (int a = 0; a < TP; ++a) {
-            const float e = sE[tt + 16 * a];
-#pragma unroll
-            for (int b = 0; b < IP; ++b) y[a][b] *= e;
-        }
-#pragma unroll 4
-        for (int jj = 0; jj < CH; ++jj) {
-            float wv[TP], kv[IP];
-#pragma unroll
-            for (int a = 0; a < TP; ++a) wv[a] = sW[(tt + 16 * a) * CHP + jj];
-#pragma unroll
-            for (int b = 0; b < IP; ++b) kv[b] = sK[jj * DKP + ti + 16 * b];
-#pragma unroll
-            for (int a = 0; a < TP; ++a)
-#pragma unroll
-                for (int b = 0; b < IP; ++b) y[a][b] = fmaf(wv[a], kv[b], y[a][b]);
-        }
-
-        // CG update
-#pragma unroll
-        for (int a = 0; a < TP; ++a) {
-            float s = 0.f;
-#pragma unroll
-            for (int b = 0; b < IP; ++b) {
-                y[a][b] = fmaf(sL[ti + 16 * b], p[a][b], y[a][b]);
-                s = fmaf(p[a][b], y[a][b], s);
-            }
-            const float pAp = sum16(s);
-            if (act[a] && !cg_curvature_ok(pAp)) act[a] = false;
-            float s2 = 0.f;
-            if (act[a]) {
-                const float alpha = rr[a] / pAp;
-#pragma unroll
-                for (int b = 0; b < IP; ++b) {
-                    x[a][b] = fmaf(alpha, p[a][b], x[a][b]);
-                    r[a][b] = fmaf(-alpha, y[a][b], r[a][b]);
-                    s2 = fmaf(r[a][b], r[a][b], s2);
-                }
-            }
-            const float rr_new = sum16(s2);
-            if (act[a]) {
-                const float rho = rr_new / rr[a];
-#pragma unroll
-                for (int b = 0; b < IP; ++b) p[a][b] = fmaf(rho, p[a][b], r[a][b]);
-                rr[a] = rr_new;
-                ++it[a];
+                for (int b = 0; b < IP; ++b) x_out[(base + t) * DK + ti + 16 * b] = x[a][b];
             }
         }
-        __syncthreads();
-#pragma unroll
-        for (int a = 0; a < TP; ++a)
-#pragma unroll
-            for (int b = 0; b < IP; ++b) sP[(tt + 16 * a) * DKP + ti + 16 * b] = p[a][b];
-        __syncthreads();
     }
-
-    // ---- read-out: o = e^{b_t} G_c x + (M (.) X K^T) V ----
+    if (!out) {
+        if (iters) {
+#pragma unroll
+            for (int a = 0; a < TP; ++a) {
+                const int t = tt + 16 * a;
+                if (t < n && ti == 0) iters[base + t] = it[a];
+            }
+        }
+        return;
+    }
     __syncthreads();
 #pragma unroll
     for (int a = 0; a < TP; ++a)
@@ -357,32 +218,7 @@ simt_cg_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* 
         for (int b = 0; b < IP; ++b) sP[(tt + 16 * a) * DKP + ti + 16 * b] = x[a][b];
     for (int e = tid; e < DV * DK; e += kThreads) sH[(e / DK) * DKP + e % DK] = Gc[e];
     __syncthreads();
-    {
-        float s[TP][JP];
-#pragma unroll
-        for (int a = 0; a < TP; ++a)
-#pragma unroll
-            for (int b = 0; b < JP; ++b) s[a][b] = 0.f;
-#pragma unroll 4
-        for (int kk = 0; kk < DK; ++kk) {
-            float pv[TP], kv[JP];
-#pragma unroll
-            for (int a = 0; a < TP; ++a) pv[a] = sP[(tt + 16 * a) * DKP + kk];
-#pragma unroll
-            for (int b = 0; b < JP; ++b) kv[b] = sK[(ti + 16 * b) * DKP + kk];
-#pragma unroll
-            for (int a = 0; a < TP; ++a)
-#pragma unroll
-                for (int b = 0; b < JP; ++b) s[a][b] = fmaf(pv[a], kv[b], s[a][b]);
-        }
-#pragma unroll
-        for (int a = 0; a < TP; ++a)
-#pragma unroll
-            for (int b = 0; b < JP; ++b) {
-                const int t = tt + 16 * a, j = ti + 16 * b;
-                sW[t * CHP + j] = sM[t * CHP + j] * s[a][b];
-            }
-    }
+    masked_scores<DK, CH>(sP, sK, sM, sW);
     __syncthreads();
     float o[TP][VP];
 #pragma unroll
@@ -453,7 +289,7 @@ cudaError_t launch_simt(const ForwardArgs& a, cudaStream_t st) {
         LaunchTimer timer(kKindSimtCg, st);
         kern<<<dim3(nc, BH), kThreads, L::bytes, st>>>(
             static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-            a.gamma, a.beta, a.lambda, a.H, a.T, nc, a.cg_steps, a.tol, states, a.out, a.iters);
+            a.gamma, a.beta, a.lambda, a.H, a.T, nc, a.cg_steps, a.tol, states, a.out, a.iters, a.x_out);
     }
     return cudaGetLastError();
 }

@@ -65,6 +65,10 @@ def _load():
     lib.mesa_timing_read.restype = I
     lib.mesa_preprocess.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, P]
     lib.mesa_preprocess.restype = I
+    lib.mesa_backward_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.mesa_backward_workspace_size.restype = Z
+    lib.mesa_backward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, Z, P]
+    lib.mesa_backward.restype = I
     _lib = lib
     return lib
 
@@ -138,6 +142,37 @@ def forward(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=No
     if return_state:
         res += (H_out, G_out)
     return res[0] if len(res) == 1 else res
+
+
+def backward(q, k, v, gamma, beta, lam, dout, *, chunk=64, cg_steps=15, tol=0.0, workspace=None, stream=None):
+    """Gradients of L given dout = dL/do for the inputs of forward() with zero
+    initial states (implicit differentiation, adjoint CG under the same rule).
+
+    dout: [B,H,T,dv] float32. Returns (dq, dk, dv, dgamma, dbeta, dlambda),
+    all float32 with the shapes of q, k, v, gamma, beta, lam.
+    """
+    lib = _load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq = torch.empty((B, H, T, dk), **f32)
+    dk_ = torch.empty((B, H, T, dk), **f32)
+    dv_ = torch.empty((B, H, T, dv), **f32)
+    dgamma = torch.empty((B, H, T), **f32)
+    dbeta = torch.empty((B, H, T), **f32)
+    dlam = torch.empty((H, dk), **f32)
+    need = int(lib.mesa_backward_workspace_size(B, H, T, dk, dv, chunk, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.mesa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                           B, H, T, dk, dv, chunk, code, int(cg_steps), float(tol), _ptr(dout),
+                           _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dgamma), _ptr(dbeta), _ptr(dlam),
+                           _ptr(workspace), ws_bytes, _stream(stream, dev))
+    _check(rc, "mesa_backward")
+    return dq, dk_, dv_, dgamma, dbeta, dlam
 
 
 def forward_host(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None,

@@ -147,3 +147,28 @@ def test_preprocess_argument_errors(lib):
     assert call(q=None) == 1                                    # null input
     assert call(q=ctypes.c_void_p(0x10008)) == 1                # misaligned
     assert call(o=a) == 1                                       # output overlaps input
+
+
+def test_backward_argument_errors(lib):
+    """Host-side checks of mesa_backward (fake, aligned device addresses; every
+    case is rejected before any launch)."""
+    B, H, T, d = 1, 2, 8, 16
+    tok = B * H * T
+    addr = iter(range(1 << 20, 1 << 40, 1 << 20))       # disjoint 1 MiB spans, 256-byte aligned
+    bufs = {n: next(addr) for n in ("q", "k", "v", "g", "b", "lam", "do", "dq", "dk", "dv", "dg", "db", "dl", "ws")}
+    need = lib.mesa_backward_workspace_size(B, H, T, d, d, 16, 0)
+    assert need > tok * d * 4
+
+    def call(ws_bytes=None, dk=d, **over):
+        p = dict(bufs, **over)
+        return lib.mesa_backward(p["q"], p["k"], p["v"], p["g"], p["b"], p["lam"], B, H, T, dk, dk, 16, 0, 15, 0.0,
+                                 p["do"], p["dq"], p["dk"], p["dv"], p["dg"], p["db"], p["dl"], p["ws"],
+                                 need if ws_bytes is None else ws_bytes, None)
+    assert call(dk=24) == 2                               # unsupported width
+    assert call(q=None) == 1
+    assert call(do=bufs["do"] + 4) == 1                   # misaligned
+    assert call(dq=bufs["q"]) == 1                        # output overlaps an input
+    assert call(dv=bufs["dk"] + 64) == 1                  # outputs overlap each other
+    assert call(ws_bytes=need - 1) == 3                   # workspace too small
+    assert call(ws=bufs["ws"] + 16) == 1                  # workspace misaligned
+    assert lib.mesa_backward_workspace_size(B, H, T, 24, 24, 16, 0) == 0
