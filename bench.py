@@ -494,6 +494,82 @@ def run_backward(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+SHARD_METRIC = "Mesa-layer fwd tokens/s (B*H*T), sequence-sharded over ranks (each rank one slice of T); d=128, 15 CG steps"
+
+
+def run_seq_sharded(args, w, world, rank, local):
+    """Sequence-sharded forward: rank r holds tokens [r T/N, (r+1) T/N) of
+    every sequence; per step one scan of the slice (mesa_chunk_state), one
+    all-gather of the slice summaries, the prefix (mesa_state_prefix) and the
+    slice's forward from that state. Total work is fixed as N grows."""
+    import torch
+    import torch.distributed as dist
+    from test_sequence_layer_b200 import build as mbuild, mesa, sharded
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % free_port(), rank=0, world_size=1)
+    Tr = w.T // world
+    x = mi.device_batch(w, dev, T=Tr, seed_offset=rank)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sharded.forward_sequence_sharded(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], chunk=w.chunk,
+                                         cg_steps=w.cg_steps, tol=w.tol, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    mesa.timing_enable(False)
+    kernels = mesa.timing_read()
+    clk = clocks.stop()
+    assert mesa.get_error() == 0
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    dist.destroy_process_group()
+    if rank != 0:
+        return
+    tokens = w.B * w.H * Tr * world
+    line = {
+        "metric": SHARD_METRIC, "value": tokens / (ms / args.steps / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16-in/f16-mma/f32-acc" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name + "+seq-sharded", "B": w.B, "H": w.H, "T": Tr * world, "T_per_rank": Tr,
+                   "d": w.dk, "chunk": w.chunk, "cg_steps": w.cg_steps, "tol": w.tol,
+                   "exchange": "one all-gather of (H, G, decay) per step: %d bytes per rank" % (
+                       w.B * w.H * (w.dk * w.dk + w.dv * w.dk + 1) * 4)},
+        "roofline": None,
+        "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
+        "gpu_launches": sum(v[0] for v in kernels.values()),
+        "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -507,6 +583,8 @@ def main():
                     help="time mesa_preprocess (q/k convolution + normalisation) on the workload's shape")
     ap.add_argument("--backward", action="store_true",
                     help="time mesa_backward (implicit-differentiation gradients) on the workload's shape")
+    ap.add_argument("--seq-sharded", action="store_true",
+                    help="sequence-sharded forward: each rank one slice of T, one all-gather of slice states")
     ap.add_argument("--warm-start", action="store_true",
                     help="decode: start each step's CG from the previous step's solution (mesa_step_warm)")
     ap.add_argument("--tol", type=float, default=None, help="override the workload's CG tolerance")
@@ -531,6 +609,9 @@ def main():
         return
     if args.backward:
         run_backward(args, w, world, rank, local)
+        return
+    if args.seq_sharded:
+        run_seq_sharded(args, w, world, rank, local)
         return
     if w.decode_steps > 0:
         run_decode(args, w, world, rank, local)

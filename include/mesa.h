@@ -211,6 +211,46 @@ mesa_status mesa_backward(const void* q, const void* k, const void* v,
                           void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Sequence sharding (a long sequence split into consecutive slices, one per
+ * GPU). The layer carries the states H_t, G_t from chunk to chunk ("MesaNet"
+ * page, Mesa layer, "Parallelisation"); the state after a slice s from an
+ * initial state S is D_s S + Delta_s, with Delta_s the state after the slice
+ * from zero and D_s = prod_{t in s} gamma_t. So each slice needs only the
+ * state entering it:
+ *     S_0 = 0,  S_{s+1} = D_s S_s + Delta_s.
+ * A sharded forward: mesa_chunk_state on the slice (from zero) -> exchange
+ * (Delta_s, D_s) of every slice (an all-gather) -> mesa_state_prefix for the
+ * caller's slice r -> mesa_forward on the slice with H_in, G_in = S_r.
+ *
+ * mesa_chunk_state: the scan of mesa_forward without the solve. For every
+ * (b, h): H_out, G_out = the states after the T tokens from H_in, G_in (NULL:
+ * zero) and decay_out [B,H] = prod_t gamma_t. Arguments as in mesa_forward;
+ * H_out, G_out float32 [B,H,dk,dk] / [B,H,dv,dk], 16-byte aligned, distinct
+ * from the inputs; decay_out float32 [B,H]. Workspace: at least
+ * mesa_chunk_state_workspace_size() bytes, 256-byte aligned. T = 0 copies
+ * (or zeroes) the state and writes decay 1.
+ */
+size_t mesa_chunk_state_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype);
+
+mesa_status mesa_chunk_state(const void* k, const void* v, const float* gamma, const float* beta,
+                             int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                             const float* H_in, const float* G_in, float* H_out, float* G_out, float* decay_out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The state entering slice r (0 <= r <= n_slices) from the summaries of the
+ * slices before it, in sequence order: H_slices float32 [n_slices,B,H,dk,dk]
+ * and G_slices [n_slices,B,H,dv,dk] (each from a zero state), decay_slices
+ * [n_slices,B,H]. Writes H_in, G_in (float32 [B,H,dk,dk] / [B,H,dv,dk],
+ * 16-byte aligned, not overlapping the inputs or each other). r = 0 writes
+ * zeros; r = n_slices gives the state after the whole sequence. dk == dv in
+ * {16,32,64,128}. Asynchronous on `stream`.
+ */
+mesa_status mesa_state_prefix(const float* H_slices, const float* G_slices, const float* decay_slices,
+                              int n_slices, int r, int B, int H, int dk, int dv,
+                              float* H_in, float* G_in, void* stream);
+
+/*
  * Bytes of device workspace mesa_forward_host needs: the mesa_forward
  * workspace plus device staging for every tensor argument.
  */

@@ -69,7 +69,8 @@ mesa_status launch_forward(const ForwardArgs& a, cudaStream_t st) {
 
 // ---- kernel timing records ----
 const char* const kKindNames[kKindCount] = {"simt_scan", "simt_cg", "decode_step", "tc_scan", "tc_cg",
-                                             "preprocess", "bwd_adjoint", "bwd_rscan", "bwd_grad", "bwd_reduce"};
+                                             "preprocess", "bwd_adjoint", "bwd_rscan", "bwd_grad", "bwd_reduce",
+                                             "shard"};
 struct TimingRec {
     int kind;
     cudaEvent_t start, stop;
@@ -269,6 +270,61 @@ mesa_status mesa_backward(const void* q, const void* k, const void* v,
                     nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes},
                    dout, dq, dk_out, dv_out, dgamma, dbeta, dlambda};
     return backward_simt(a, st) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+size_t mesa_chunk_state_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
+    if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
+    return workspace_bytes(B, H, T, dk, dv, chunk, dtype);
+}
+
+mesa_status mesa_chunk_state(const void* k, const void* v, const float* gamma, const float* beta,
+                             int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                             const float* H_in, const float* G_in, float* H_out, float* G_out, float* decay_out,
+                             void* workspace, size_t ws_bytes, void* stream) {
+    mesa_status s = check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f);
+    if (s != MESA_OK) return s;
+    if (!H_out || !G_out || !decay_out) return MESA_ERR_INVALID_ARG;
+    if (!aligned(H_out, 16) || !aligned(G_out, 16) || !aligned(decay_out, 4)) return MESA_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)H_in, (const void*)G_in})
+        if (p && !aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    if (H_out == H_in || G_out == G_in) return MESA_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!k || !v || !gamma || !beta) return MESA_ERR_INVALID_ARG;
+        if (!aligned(k, 16) || !aligned(v, 16) || !aligned(gamma, 4) || !aligned(beta, 4)) return MESA_ERR_INVALID_ARG;
+        const size_t need = workspace_bytes(B, H, T, dk, dv, chunk, dtype);
+        if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ForwardArgs a{nullptr, k, v, gamma, beta, nullptr, B, H, T, dk, dv, chunk, dtype, 0, 0.f,
+                  nullptr, nullptr, H_in, G_in, H_out, G_out, workspace, ws_bytes};
+    if (T == 0) {   // the state passes through unchanged; the decay of an empty slice is 1
+        if (launch_forward(a, st) != MESA_OK) return MESA_ERR_CUDA;
+    }
+    return chunk_state(a, decay_out, st) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
+}
+
+mesa_status mesa_state_prefix(const float* H_slices, const float* G_slices, const float* decay_slices,
+                              int n_slices, int r, int B, int H, int dk, int dv,
+                              float* H_in, float* G_in, void* stream) {
+    if (B < 1 || H < 1 || n_slices < 0 || r < 0 || r > n_slices) return MESA_ERR_INVALID_ARG;
+    if (!supported_width(dk) || dk != dv) return MESA_ERR_UNSUPPORTED;
+    if (!H_in || !G_in || !aligned(H_in, 16) || !aligned(G_in, 16)) return MESA_ERR_INVALID_ARG;
+    if (r > 0 && (!H_slices || !G_slices || !decay_slices)) return MESA_ERR_INVALID_ARG;
+    const size_t BH = (size_t)B * H;
+    const size_t nh = BH * dk * dk * 4, ng = BH * dv * dk * 4;
+    const char* hi = (const char*)H_in;
+    const char* gi = (const char*)G_in;
+    if (hi < gi + ng && gi < hi + nh) return MESA_ERR_INVALID_ARG;
+    if (r > 0) {
+        const struct { const char* p; size_t n; } in[] = {{(const char*)H_slices, nh * n_slices},
+                                                          {(const char*)G_slices, ng * n_slices},
+                                                          {(const char*)decay_slices, BH * 4 * n_slices}};
+        for (const auto& x : in)
+            if ((hi < x.p + x.n && x.p < hi + nh) || (gi < x.p + x.n && x.p < gi + ng)) return MESA_ERR_INVALID_ARG;
+    }
+    return state_prefix(H_slices, G_slices, decay_slices, r, (int)BH, dk, dv, H_in, G_in,
+                        static_cast<cudaStream_t>(stream)) == cudaSuccess ? MESA_OK : MESA_ERR_CUDA;
 }
 
 size_t mesa_forward_host_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {

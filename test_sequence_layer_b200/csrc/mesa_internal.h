@@ -30,6 +30,7 @@ struct ForwardArgs {
     void* workspace;
     size_t ws_bytes;
     float* x_out = nullptr;     // fp32 CUDA-core path only: the CG solutions x_t [B,H,T,dk]
+    bool scan_only = false;     // fp32 CUDA-core path only: the chunk-state scan, no solve
 };
 
 struct BackwardArgs {
@@ -49,7 +50,7 @@ unsigned* error_word_ptr();
 // Kernel kinds for the optional timing records (mesa_timing_enable).
 enum KernelKind : int {
     kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindPre,
-    kKindBwdAdj, kKindBwdRscan, kKindBwdGrad, kKindBwdReduce, kKindCount
+    kKindBwdAdj, kKindBwdRscan, kKindBwdGrad, kKindBwdReduce, kKindShard, kKindCount
 };
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
@@ -69,11 +70,17 @@ class LaunchTimer {
 size_t simt_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
 cudaError_t forward_simt(const ForwardArgs& a, cudaStream_t st);
 size_t backward_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
+// Sequence sharding: the state after a slice and its total decay; the state
+// entering slice r from the summaries of slices 0..r-1 (sharded.cu).
+cudaError_t chunk_state(const ForwardArgs& a, float* decay_out, cudaStream_t st);
+cudaError_t state_prefix(const float* H_s, const float* G_s, const float* decay_s, int r, int BH, int dk, int dv,
+                         float* H_in, float* G_in, cudaStream_t st);
 cudaError_t backward_simt(const BackwardArgs& a, cudaStream_t st);
 
 // Tensor-core path (tc_forward.cu): bf16 inputs, dk = dv = 128, chunk = 64.
 bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype);
 size_t tc_workspace_bytes(int B, int H, int T);
+size_t tc_images_bytes(int B, int H, int T);     // the state images at the start of the workspace
 cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st);
 // Chunk-state scan of the tensor-core forward: state images and scales into
 // img / scales (layout in tc_layout.cuh), final states into a.H_out / a.G_out.

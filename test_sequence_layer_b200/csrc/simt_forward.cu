@@ -280,7 +280,7 @@ cudaError_t launch_simt(const ForwardArgs& a, cudaStream_t st) {
             a.H_in, a.G_in, states, a.H_out, a.G_out);
     }
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || a.scan_only) return e;
     using L = CgSmem<D, D, CH>;
     auto kern = simt_cg_kernel<D, D, CH, Tin>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);

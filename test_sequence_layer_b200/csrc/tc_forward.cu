@@ -606,21 +606,21 @@ bool tc_supported(int dk, int dv, int chunk, mesa_dtype dtype) {
 }
 
 // One H and one G image (and their scales) per 128-token block.
-static size_t images_bytes(int B, int H, int T) {
+size_t tc_images_bytes(int B, int H, int T) {
     const size_t np = (size_t)((T + kBlk - 1) / kBlk);
     return (size_t)B * H * np * 2 * kImgBytes;
 }
 
 size_t tc_workspace_bytes(int B, int H, int T) {
     const size_t np = (size_t)((T + kBlk - 1) / kBlk);
-    return images_bytes(B, H, T) + ((size_t)B * H * np * 2 * sizeof(float) + 255) / 256 * 256;
+    return tc_images_bytes(B, H, T) + ((size_t)B * H * np * 2 * sizeof(float) + 255) / 256 * 256;
 }
 
 cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     const int nc = (a.T + kC - 1) / kC;
     const int BH = a.B * a.H;
     __half* img = reinterpret_cast<__half*>(a.workspace);
-    float* scales = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + images_bytes(a.B, a.H, a.T));
+    float* scales = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + tc_images_bytes(a.B, a.H, a.T));
     unsigned* err = error_word_ptr();
     const int cg_smem = BlkSmem::bytes + 1024;
     cudaError_t e = tc_scan_launch(a, img, scales, err, st);

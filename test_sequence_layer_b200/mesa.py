@@ -65,6 +65,12 @@ def _load():
     lib.mesa_timing_read.restype = I
     lib.mesa_preprocess.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, P]
     lib.mesa_preprocess.restype = I
+    lib.mesa_chunk_state_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.mesa_chunk_state_workspace_size.restype = Z
+    lib.mesa_chunk_state.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, Z, P]
+    lib.mesa_chunk_state.restype = I
+    lib.mesa_state_prefix.argtypes = [P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.mesa_state_prefix.restype = I
     lib.mesa_backward_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.mesa_backward_workspace_size.restype = Z
     lib.mesa_backward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, Z, P]
@@ -173,6 +179,44 @@ def backward(q, k, v, gamma, beta, lam, dout, *, chunk=64, cg_steps=15, tol=0.0,
                            _ptr(workspace), ws_bytes, _stream(stream, dev))
     _check(rc, "mesa_backward")
     return dq, dk_, dv_, dgamma, dbeta, dlam
+
+
+def chunk_state(k, v, gamma, beta, *, chunk=64, H_in=None, G_in=None, workspace=None, stream=None):
+    """The scan of forward() without the solve: (H_out, G_out, decay) with the
+    states after the T tokens (from H_in, G_in or zero) and decay [B,H] =
+    prod_t gamma_t. The summary a slice of a sequence-sharded forward exchanges."""
+    lib = _load()
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    code = _dtype_code(k)
+    dev = k.device
+    H_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    G_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    decay = torch.empty((B, H), dtype=torch.float32, device=dev)
+    need = int(lib.mesa_chunk_state_workspace_size(B, H, T, dk, dv, chunk, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.mesa_chunk_state(_ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), B, H, T, dk, dv, chunk, code,
+                              _ptr(H_in), _ptr(G_in), _ptr(H_out), _ptr(G_out), _ptr(decay),
+                              _ptr(workspace), ws_bytes, _stream(stream, dev))
+    _check(rc, "mesa_chunk_state")
+    return H_out, G_out, decay
+
+
+def state_prefix(H_slices, G_slices, decay_slices, r, *, stream=None):
+    """State entering slice r from the stacked summaries [n, B, H, ...] of the
+    slices before it (in sequence order). Returns (H_in, G_in)."""
+    lib = _load()
+    n, B, H, dk, _ = H_slices.shape
+    dv = G_slices.shape[3]
+    dev = H_slices.device
+    H_in = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    G_in = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    rc = lib.mesa_state_prefix(_ptr(H_slices), _ptr(G_slices), _ptr(decay_slices), n, int(r), B, H, dk, dv,
+                               _ptr(H_in), _ptr(G_in), _stream(stream, dev))
+    _check(rc, "mesa_state_prefix")
+    return H_in, G_in
 
 
 def forward_host(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=None,

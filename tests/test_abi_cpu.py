@@ -172,3 +172,25 @@ def test_backward_argument_errors(lib):
     assert call(ws_bytes=need - 1) == 3                   # workspace too small
     assert call(ws=bufs["ws"] + 16) == 1                  # workspace misaligned
     assert lib.mesa_backward_workspace_size(B, H, T, 24, 24, 16, 0) == 0
+
+
+def test_sharding_argument_errors(lib):
+    """mesa_chunk_state and mesa_state_prefix reject bad arguments on the host."""
+    B, H, T, d = 1, 2, 8, 16
+    a = 1 << 24
+    need = lib.mesa_chunk_state_workspace_size(B, H, T, d, d, 16, 0)
+    assert need > 0
+    cs = lambda k=a, Ho=a + (1 << 20), Go=a + (2 << 20), dec=a + (3 << 20), ws=a + (4 << 20), wsb=need, dk=d: \
+        lib.mesa_chunk_state(k, a, a, a, B, H, T, dk, dk, 16, 0, None, None, Ho, Go, dec, ws, wsb, None)  # noqa: E731
+    assert cs(dk=24) == 2
+    assert cs(k=None) == 1
+    assert cs(Ho=None) == 1
+    assert cs(Ho=a + (1 << 20) + 8) == 1                     # misaligned
+    assert cs(wsb=need - 1) == 3
+    sp = lambda n=2, r=1, Hi=a + (8 << 20), Gi=a + (9 << 20), dk=d: \
+        lib.mesa_state_prefix(a, a + (1 << 20), a + (2 << 20), n, r, B, H, dk, dk, Hi, Gi, None)  # noqa: E731
+    assert sp(r=3) == 1                                      # r > n_slices
+    assert sp(r=-1) == 1
+    assert sp(dk=24) == 2
+    assert sp(Hi=a) == 1                                     # output overlaps the stacked inputs
+    assert sp(Gi=a + (8 << 20)) == 1                         # outputs overlap each other

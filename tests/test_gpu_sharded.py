@@ -1,0 +1,78 @@
+"""Sequence-sharded forward on one GPU: the ranks are emulated as consecutive
+slices of the same sequences run one after the other (mesa_chunk_state on
+every slice, the summaries stacked as the all-gather would, mesa_state_prefix
+for each slice, then mesa_forward from that state), compared with the fp64
+oracle of the whole sequence."""
+import numpy as np
+import pytest
+import torch
+
+import mesa_inputs as mi
+from helpers import TOL_BF16, TOL_F32, err_report, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mesa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from test_sequence_layer_b200 import build, mesa as m
+    build.build()
+    return m
+
+
+CASES = [
+    # dtype, d, chunk, slice bounds, cg_steps
+    ("f32", 32, 16, (0, 128, 228, 300), 8),
+    ("f32", 64, 64, (0, 1, 90, 200), 10),
+    ("bf16", 128, 64, (0, 256, 556, 700), 15),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[0]}-d{c[1]}-C{c[2]}-W{len(c[3]) - 1}")
+def test_sharded_forward_equals_whole(mesa, oracle_mod, case):
+    dtype, d, chunk, bounds, N = case
+    T = bounds[-1]
+    w = mi.Workload("t", 2, 2, T, d, d, chunk, dtype, N, 0.0, False, 21)
+    x = mi.batch(w)
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    dev = {n: torch.from_numpy(np.ascontiguousarray(x[n])).cuda() for n in ("q", "k", "v", "gamma", "beta", "lam")}
+    for n in ("q", "k", "v"):
+        dev[n] = dev[n].to(dt)
+    sl = [slice(bounds[i], bounds[i + 1]) for i in range(len(bounds) - 1)]
+    part = lambda n, s: dev[n][:, :, s].contiguous()        # noqa: E731
+    summ = [mesa.chunk_state(part("k", s), part("v", s), part("gamma", s), part("beta", s), chunk=chunk) for s in sl]
+    H_all = torch.stack([a[0] for a in summ])
+    G_all = torch.stack([a[1] for a in summ])
+    d_all = torch.stack([a[2] for a in summ])
+    outs = []
+    for r, s in enumerate(sl):
+        H_in, G_in = mesa.state_prefix(H_all, G_all, d_all, r)
+        outs.append(mesa.forward(part("q", s), part("k", s), part("v", s), part("gamma", s), part("beta", s),
+                                 dev["lam"], chunk=chunk, cg_steps=N, H_in=H_in, G_in=G_in))
+    H_fin, G_fin = mesa.state_prefix(H_all, G_all, d_all, len(sl))
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    got = torch.cat(outs, dim=2).cpu().numpy()
+    ref, _, Hf, Gf = oracle_mod.forward_cg(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], N)
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    assert rel_err(got, ref) <= tol, err_report(got, ref)
+    # the decay of each slice and the state after the whole sequence
+    dec = np.stack([np.prod(x["gamma"][:, :, s].astype(np.float64), axis=-1) for s in sl])
+    np.testing.assert_allclose(d_all.cpu().numpy(), dec, rtol=1e-4)      # fp32 sum of log gamma
+    for a, b in ((H_fin, Hf), (G_fin, Gf)):
+        a = a.cpu().numpy()
+        assert np.abs(a - b).max() <= 1e-4 * max(np.abs(b).max(), 1.0)
+
+
+def test_chunk_state_of_an_empty_slice(mesa):
+    B, H, d = 1, 2, 16
+    H_in = torch.randn((B, H, d, d), device="cuda")
+    G_in = torch.randn((B, H, d, d), device="cuda")
+    e = torch.empty((B, H, 0, d), device="cuda")
+    g = torch.empty((B, H, 0), device="cuda")
+    Ho, Go, dec = mesa.chunk_state(e, e, g, g, chunk=16, H_in=H_in, G_in=G_in)
+    torch.cuda.synchronize()
+    assert torch.equal(Ho, H_in) and torch.equal(Go, G_in)
+    assert torch.equal(dec, torch.ones_like(dec))

@@ -527,3 +527,19 @@ def test_backward_one_step_closed_form(oracle_mod):
     np.testing.assert_allclose(r["dk"][0, 0, 0], bet * ((Hbar + Hbar.T) @ k + Gbar.T @ v), rtol=1e-12)
     np.testing.assert_allclose(r["dbeta"][0, 0, 0], k @ Hbar @ k + v @ Gbar @ k, rtol=1e-12)
     assert r["dgamma"][0, 0, 0] == 0.0              # the state before the first token is zero
+
+
+def test_state_after_a_slice_is_affine_in_the_initial_state(oracle_mod):
+    """The recurrence is affine in the state: the state after a slice from S
+    equals prod(gamma) S plus the state after the slice from zero (the fact a
+    sequence-sharded forward rests on)."""
+    rng = np.random.default_rng(8)
+    q, k, v, gamma, beta, lam = rand_inputs(rng, 1, 2, 11, 3, 4)
+    S_H = rng.standard_normal((1, 2, 3, 3))
+    S_H = S_H @ np.swapaxes(S_H, -1, -2)
+    S_G = rng.standard_normal((1, 2, 4, 3))
+    _, _, H1, G1 = oracle_mod.forward_cg(q, k, v, gamma, beta, lam, 3, H0=S_H, G0=S_G)
+    _, _, H0, G0 = oracle_mod.forward_cg(q, k, v, gamma, beta, lam, 3)
+    D = np.prod(gamma, axis=-1)[..., None, None]
+    np.testing.assert_allclose(H1, D * S_H + H0, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(G1, D * S_G + G0, rtol=1e-12, atol=1e-14)
