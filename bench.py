@@ -510,15 +510,16 @@ def run_seq_sharded(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    else:
-        dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % free_port(), rank=0, world_size=1)
     Tr = w.T // world
     x = mi.device_batch(w, dev, T=Tr, seed_offset=rank)
     stream = torch.cuda.current_stream(dev)
+    ws = torch.empty(mesa.workspace_size(w.B, w.H, Tr, w.dk, w.dv, w.chunk,
+                                         torch.bfloat16 if w.dtype == "bf16" else torch.float32),
+                     dtype=torch.uint8, device=dev)
 
     def step():
         sharded.forward_sequence_sharded(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], chunk=w.chunk,
-                                         cg_steps=w.cg_steps, tol=w.tol, stream=stream)
+                                         cg_steps=w.cg_steps, tol=w.tol, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -529,20 +530,23 @@ def run_seq_sharded(args, w, world, rank, local):
     mesa.timing_enable(True)
     mesa.timing_read()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier()
+    if world > 1:
+        dist.barrier()
     torch.cuda.synchronize()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    dist.barrier()
+    if world > 1:
+        dist.barrier()
     mesa.timing_enable(False)
     kernels = mesa.timing_read()
     clk = clocks.stop()
     assert mesa.get_error() == 0
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    dist.destroy_process_group()
+    if world > 1:
+        dist.destroy_process_group()
     if rank != 0:
         return
     tokens = w.B * w.H * Tr * world
@@ -561,13 +565,6 @@ def run_seq_sharded(args, w, world, rank, local):
         "clocks": clk, "e2e": None, "cpu_baseline": None,
     }
     print(json.dumps(line), flush=True)
-
-
-def free_port():
-    import socket
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
 
 
 def main():
