@@ -13,6 +13,11 @@
 // Numerics: w_j a_j is split into an fp16 hi/lo pair, both multiplied by the
 // fp16 keys on the tensor cores with fp32 accumulation, so each chunk's sum
 // carries ~22-bit products into the fp32 running state.
+//
+// Pipeline per chunk c: MMA(c) runs while the CTA builds chunk c+1's operand
+// images (a second set) and warp 1 forms chunk c+2's gates (three gate
+// buffers); then the state takes Delta_c, and the state before every even
+// chunk is staged in shared memory and stored with one bulk copy.
 #include "mesa_internal.h"
 #include "tc_layout.cuh"
 
@@ -57,11 +62,11 @@ constexpr int kScanThreads = 512;
 struct ScanSmem {
     static constexpr int oRawA = 0;               // 2 x [64][128] bf16 rows of a (16 KB each)
     static constexpr int oRawK = 32768;           // 2 x [64][128] bf16 rows of k
-    static constexpr int oAhi = 65536;            // MN-major [64 j][128 i] fp16, 16 KB
-    static constexpr int oAlo = 81920;
-    static constexpr int oB = 98304;              // MN-major [64 j][128 l] fp16, 16 KB
-    static constexpr int oGate = 114688;          // b[2][64], w[2][64], amax[64], kmax[64]
-    static constexpr int oGraw = oGate + 1536;    // 2 x {gamma[64], beta[64]} prefetched with the rows
+    static constexpr int oImg = 65536;            // 2 operand sets {A hi, A lo, B}, MN-major SW128, 16 KB each
+    static constexpr int kSet = 49152;
+    static constexpr int oStage = oImg + 2 * kSet;    // staged state image for the bulk store (32 KB)
+    static constexpr int oGate = oStage + 32768;  // b[3][64], w[3][64], amax[2][64], kmax[2][64]
+    static constexpr int oGraw = oGate + 2560;    // 2 x {gamma[64], beta[64]} prefetched with the rows
     static constexpr int oRed = oGraw + 1024;     // 32 floats; [31] is the abort flag
     static constexpr int oBar = oRed + 128;       // raw[2], mma
     static constexpr int oSlot = oBar + 32;
@@ -75,8 +80,11 @@ struct ScanSmem {
 // w_j = beta_j e^{b_last - b_j},
 //     S <- e^{b_last} S + sum_j (w_j a_j) k_j^T
 // where the sum is one M = 128, N = 128, K = 64 MMA over the chunk's tokens,
-// issued for the hi and the lo fp16 parts of w_j a_j. The gates of chunk c + 1
-// are formed by warp 1 while the MMA of chunk c runs.
+// issued for the hi and the lo fp16 parts of w_j a_j. The chunks are
+// pipelined: while the MMA of chunk c runs, the CTA builds chunk c+1's
+// operand images (a second set) and warp 1 forms chunk c+2's gates. The state
+// before every even chunk is staged in shared memory in the solve's image
+// layout and written with one bulk copy.
 __global__ void __launch_bounds__(kScanThreads, 1)
 tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                const float* __restrict__ gamma, const float* __restrict__ beta, int T, int nc,
@@ -88,13 +96,11 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     const int m = blockIdx.x, bh = blockIdx.y;
     uint8_t* rawK = smem + ScanSmem::oRawK;
     uint8_t* rawA = m ? smem + ScanSmem::oRawA : rawK;     // for H the left factor is k itself
-    uint8_t* Ahi = smem + ScanSmem::oAhi;
-    uint8_t* Alo = smem + ScanSmem::oAlo;
-    uint8_t* Bk = smem + ScanSmem::oB;
-    float* sb = reinterpret_cast<float*>(smem + ScanSmem::oGate);      // [2][64]
-    float* sw = sb + 2 * kC;                                            // [2][64]
-    float* amax = sw + 2 * kC;
-    float* kmax = amax + kC;
+    uint8_t* stage = smem + ScanSmem::oStage;
+    float* sb = reinterpret_cast<float*>(smem + ScanSmem::oGate);      // [3][64]
+    float* sw = sb + 3 * kC;                                            // [3][64]
+    float* amax = sw + 3 * kC;                                          // [2][64]
+    float* kmax = amax + 2 * kC;                                        // [2][64]
     float* graw = reinterpret_cast<float*>(smem + ScanSmem::oGraw);
     float* red = reinterpret_cast<float*>(smem + ScanSmem::oRed);
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(smem + ScanSmem::oBar);
@@ -109,6 +115,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     const float* init = m ? G_in : H_in;
     float* fin = m ? G_out : H_out;
     const size_t seq = (size_t)bh * T;
+    const int np = (nc + 1) >> 1;
     // gamma/beta of a chunk travel with its rows when the chunk is full and its
     // first element is 16-byte aligned (T % 4 == 0); otherwise warp 1 reads them.
     const bool gates_bulk = (T % 4) == 0 && ((reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(beta)) & 15) == 0;
@@ -129,7 +136,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         prefetched = cc + 1;
     };
     // One warp: waits for chunk cc's copies, then b (log-cumsum of gamma) and
-    // w_j = beta_j e^{b_last - b_j} into gate buffer cc & 1.
+    // w_j = beta_j e^{b_last - b_j} into gate buffer cc % 3.
     auto chunk_gates = [&](int cc) {
         const int buf = cc & 1;
         if (!mbar_wait(bar_raw + buf, (cc >> 1) & 1)) red[31] = 1.f;
@@ -139,13 +146,91 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         const bool gb = gates_bulk && nn == kC;
         const float* gsrc = gb ? graw + buf * 128 : gamma + base;
         const float* bsrc = gb ? graw + buf * 128 + 64 : beta + base;
-        float* b = sb + buf * kC;
-        float* wv = sw + buf * kC;
+        float* b = sb + (cc % 3) * kC;
+        float* wv = sw + (cc % 3) * kC;
         warp_gate_cumsum(gsrc, nn, b);
         __syncwarp();
         const float bl = b[kC - 1];                                // b at the chunk's last position
         wv[lane] = (lane < nn) ? bsrc[lane] * expf(bl - b[lane]) : 0.f;
         wv[lane + 32] = (lane + 32 < nn) ? bsrc[lane + 32] * expf(bl - b[lane + 32]) : 0.f;
+    };
+    // Operand images of chunk cc into set cc & 1: A = w_j a_j (hi/lo) [j][i],
+    // B = k_j [j][l], both MN-major SW128 in two 64-column blocks; row maxima
+    // of a and k into buffer cc & 1.
+    auto build = [&](int cc) {
+        const int n = min(kC, T - cc * kC);
+        const float* swc = sw + (cc % 3) * kC;
+        const uint8_t* ra = rawA + (cc & 1) * 16384;
+        const uint8_t* rk = rawK + (cc & 1) * 16384;
+        uint8_t* Ahi = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
+        uint8_t* Alo = Ahi + 16384;
+        uint8_t* Bk = Ahi + 32768;
+        float* am = amax + (cc & 1) * kC;
+        float* km = kmax + (cc & 1) * kC;
+#pragma unroll
+        for (int rep = 0; rep < 2; ++rep) {
+            const int cid = tid + kScanThreads * rep;      // 1024 16-byte chunks of the rows
+            const int j = cid >> 4, cc16 = cid & 15;
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (j < n) raw = *reinterpret_cast<const uint4*>(ra + j * 256 + cc16 * 16);
+            const float wj = swc[j];
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            uint4 hi, lo;
+            uint32_t* hw = reinterpret_cast<uint32_t*>(&hi);
+            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+            float mx = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(a2[i]);
+                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+                const float x0 = wj * f.x, x1 = wj * f.y;
+                const __half2 h2 = __floats2half2_rn(x0, x1);
+                const float2 hb = __half22float2(h2);
+                hw[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                lw[i] = pack_half2(x0 - hb.x, x1 - hb.y);
+            }
+            const uint32_t off = (uint32_t)((cc16 >> 3) * 8192 + j * 128 + (((cc16 & 7) ^ (j & 7)) << 4));
+            *reinterpret_cast<uint4*>(Ahi + off) = hi;
+            *reinterpret_cast<uint4*>(Alo + off) = lo;
+            // row max over the 16 threads (same half-warp) that hold row j
+#pragma unroll
+            for (int o2 = 8; o2 >= 1; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+            if (cc16 == 0) am[j] = mx;
+            uint4 kr = raw;
+            if (m) {   // key rows: the B operand and the key row maxima for the value-state bound
+                kr = make_uint4(0, 0, 0, 0);
+                if (j < n) kr = *reinterpret_cast<const uint4*>(rk + j * 256 + cc16 * 16);
+                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+                float kmx = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(k2[i]);
+                    kmx = fmaxf(kmx, fmaxf(fabsf(f.x), fabsf(f.y)));
+                }
+#pragma unroll
+                for (int o2 = 8; o2 >= 1; o2 >>= 1) kmx = fmaxf(kmx, __shfl_xor_sync(0xffffffffu, kmx, o2));
+                if (cc16 == 0) km[j] = kmx;
+            }
+            *reinterpret_cast<uint4*>(Bk + off) = bf16x8_to_f16x8(kr, 1.f);
+        }
+    };
+    // The state / s as fp16 into the staging image (the solve's layout);
+    // returns the power-of-two scale s from the entry bound.
+    auto stage_state = [&](const float (&St)[32], float bnd) {
+        const float s = pow2_ceil_at_least_one(bnd);
+        const float inv = 1.f / s;
+        uint8_t* dst = stage + (col0 >> 6) * 16384 + row * 128;
+        const int g0 = (col0 & 63) >> 3;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            uint4 o;
+            o.x = pack_half2(St[8 * g] * inv, St[8 * g + 1] * inv);
+            o.y = pack_half2(St[8 * g + 2] * inv, St[8 * g + 3] * inv);
+            o.z = pack_half2(St[8 * g + 4] * inv, St[8 * g + 5] * inv);
+            o.w = pack_half2(St[8 * g + 6] * inv, St[8 * g + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + (((g0 + g) ^ (row & 7)) << 4)) = o;
+        }
+        return s;
     };
 
     if (tid == 0) {
@@ -188,130 +273,68 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
 #pragma unroll
         for (int i = 1; i < kScanThreads / 32; ++i) bound = fmaxf(bound, red[i]);
     }
-    if (w == 1 && nc > 0) chunk_gates(0);
-    __syncthreads();                              // gates of chunk 0 (and the bound's partials) read
+    if (w == 1 && nc > 0) {
+        chunk_gates(0);
+        if (nc > 1) chunk_gates(1);
+    }
+    __syncthreads();                              // gates of chunks 0 and 1 (and the bound's partials) read
     bool ok = red[31] == 0.f;
 
     constexpr uint32_t kIdesc = idesc_f16(128, 128, true, true);
-    const uint64_t dAhi = sdesc(smem_addr(Ahi), 8192, 1024), dAlo = sdesc(smem_addr(Alo), 8192, 1024);
-    const uint64_t dB = sdesc(smem_addr(Bk), 8192, 1024);
-    uint32_t mma_phase = 0;
-    bool mma_out = false;                         // thread 0: a committed MMA not yet observed
-    int c = 0;
-    for (; ok; ++c) {
-        // ---- emit the state before chunk c (fp16 image + scale) when c starts a
-        //      128-token block of the solve, or the final state ----
-        if (c < nc && (c & 1) == 0) {
-            const float s = pow2_ceil_at_least_one(bound);
-            const float inv = 1.f / s;
-            const size_t ci = image_index(bh, (nc + 1) >> 1, c >> 1, m);
-            if (tid == 0) scales[ci] = s;
-            uint8_t* dst = reinterpret_cast<uint8_t*>(img + ci * kImgHalves) + (col0 >> 6) * 16384 + row * 128;
-            const int g0 = (col0 & 63) >> 3;
+    auto issue_mma = [&](int cc) {                // thread 0: the chunk's 8 K steps (hi, then lo) into TMEM
+        const uint8_t* Ahi = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
+        const uint64_t dAhi = sdesc(smem_addr(Ahi), 8192, 1024), dAlo = sdesc(smem_addr(Ahi + 16384), 8192, 1024);
+        const uint64_t dB = sdesc(smem_addr(Ahi + 32768), 8192, 1024);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint4 o;
-                o.x = pack_half2(S[8 * g] * inv, S[8 * g + 1] * inv);
-                o.y = pack_half2(S[8 * g + 2] * inv, S[8 * g + 3] * inv);
-                o.z = pack_half2(S[8 * g + 4] * inv, S[8 * g + 5] * inv);
-                o.w = pack_half2(S[8 * g + 6] * inv, S[8 * g + 7] * inv);
-                *reinterpret_cast<uint4*>(dst + (((g0 + g) ^ (row & 7)) << 4)) = o;
-            }
-        } else if (c == nc) {
-            if (fin) {
-                float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
-            }
-            break;
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t ko = ((ks & 3) * 2048) >> 4;
+            mma_f16(tbase, (ks < 4 ? dAhi : dAlo) + ko, dB + ko, kIdesc, ks > 0 ? 1u : 0u);
         }
-        const int n = min(kC, T - c * kC);
-        const int buf = c & 1;
-        const float* swc = sw + buf * kC;
-        const float blast = sb[buf * kC + kC - 1];
-        // ---- operand images: A = w_j a_j (hi/lo) [j][i], B = k_j [j][l], both
-        //      MN-major SW128 in two 64-column blocks; row maxima of a and k ----
-        const uint8_t* ra = rawA + buf * 16384;
-        const uint8_t* rk = rawK + buf * 16384;
-#pragma unroll
-        for (int rep = 0; rep < 2; ++rep) {
-            const int cid = tid + kScanThreads * rep;      // 1024 16-byte chunks of the rows
-            const int j = cid >> 4, cc = cid & 15;
-            uint4 raw = make_uint4(0, 0, 0, 0);
-            if (j < n) raw = *reinterpret_cast<const uint4*>(ra + j * 256 + cc * 16);
-            const float wj = swc[j];
-            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-            uint4 hi, lo;
-            uint32_t* hw = reinterpret_cast<uint32_t*>(&hi);
-            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
-            float mx = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(a2[i]);
-                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-                const float x0 = wj * f.x, x1 = wj * f.y;
-                const __half2 h2 = __floats2half2_rn(x0, x1);
-                const float2 hb = __half22float2(h2);
-                hw[i] = *reinterpret_cast<const uint32_t*>(&h2);
-                lw[i] = pack_half2(x0 - hb.x, x1 - hb.y);
-            }
-            const uint32_t off = (uint32_t)((cc >> 3) * 8192 + j * 128 + (((cc & 7) ^ (j & 7)) << 4));
-            *reinterpret_cast<uint4*>(Ahi + off) = hi;
-            *reinterpret_cast<uint4*>(Alo + off) = lo;
-            // row max over the 16 threads (same half-warp) that hold row j
-#pragma unroll
-            for (int o2 = 8; o2 >= 1; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-            if (cc == 0) amax[j] = mx;
-            uint4 kr = raw;
-            if (m) {   // key rows: the B operand and the key row maxima for the value-state bound
-                kr = make_uint4(0, 0, 0, 0);
-                if (j < n) kr = *reinterpret_cast<const uint4*>(rk + j * 256 + cc * 16);
-                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-                float km = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(k2[i]);
-                    km = fmaxf(km, fmaxf(fabsf(f.x), fabsf(f.y)));
-                }
-#pragma unroll
-                for (int o2 = 8; o2 >= 1; o2 >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o2));
-                if (cc == 0) kmax[j] = km;
-            }
-            *reinterpret_cast<uint4*>(Bk + off) = bf16x8_to_f16x8(kr, 1.f);
-        }
+        mma_commit(bar_mma);
+    };
+    int mma_issued = 0, mma_seen = 0;             // thread 0
+    if (ok && nc > 0) {
+        // the state before chunk 0 (block 0's image) and chunk 0's operands
+        const float s0 = stage_state(S, bound);
+        build(0);
         fence_proxy_async();
         tc_fence_before();
-        __syncthreads();                          // images written; every thread's last TMEM read done
+        __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            if (c + 2 < nc) prefetch(c + 2);       // raw buffer `buf` is consumed
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t ko = ((ks & 3) * 2048) >> 4;
-                mma_f16(tbase, (ks < 4 ? dAhi : dAlo) + ko, dB + ko, kIdesc, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(bar_mma);
-            mma_out = true;
+            const size_t ci = image_index(bh, np, 0, m);
+            bulk_s2g(img + ci * kImgHalves, stage, kImgBytes);
+            bulk_commit();
+            scales[ci] = s0;
+            issue_mma(0);
+            ++mma_issued;
+            if (nc > 2) prefetch(2);              // raw buffer 0 is consumed
         }
-        if (w == 1 && c + 1 < nc) chunk_gates(c + 1);
-        // bound update: every warp reduces the same 64 terms in the same order,
-        // so every thread gets the same value
+    }
+    int c = 0;
+    for (; ok && c < nc; ++c) {
+        // ---- while MMA(c) runs: chunk c+1's operands, chunk c+2's gates, the bound after chunk c ----
+        if (c + 1 < nc) build(c + 1);
+        if (w == 1 && c + 2 < nc) chunk_gates(c + 2);
+        const float blast = sb[(c % 3) * kC + kC - 1];
         {
-            const float* km = m ? kmax : amax;
-            float add = swc[lane] * (amax[lane] * km[lane]) + swc[lane + 32] * (amax[lane + 32] * km[lane + 32]);
+            // every warp reduces the same 64 terms in the same order, so every
+            // thread gets the same value
+            const float* swc = sw + (c % 3) * kC;
+            const float* am = amax + (c & 1) * kC;
+            const float* km = (m ? kmax : amax) + (c & 1) * kC;
+            float add = swc[lane] * (am[lane] * km[lane]) + swc[lane + 32] * (am[lane + 32] * km[lane + 32]);
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) add += __shfl_xor_sync(0xffffffffu, add, off);
             bound = fmaf(expf(blast), bound, add);
         }
+        const bool emit = c + 1 < nc && ((c + 1) & 1) == 0;
         if (tid == 0) {
-            if (mbar_wait(bar_mma, mma_phase & 1)) {
-                ++mma_phase;
-                mma_out = false;
-            } else {
-                red[31] = 1.f;
-            }
+            if (mbar_wait(bar_mma, c & 1)) mma_seen = mma_issued;
+            else red[31] = 1.f;
+            if (emit) bulk_wait_read_all();       // the staging buffer is free again
         }
-        __syncthreads();                          // MMA done; gates of chunk c + 1 written
+        __syncthreads();                          // MMA(c) done; operands of c+1 and gates of c+2 written
         tc_fence_after();
         if (red[31] != 0.f) {
             ok = false;
@@ -324,12 +347,45 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) S[i] = fmaf(Gam, S[i], dv[i]);
+        if (c + 1 == nc) {                        // the final state
+            if (fin) {
+                float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+            }
+            break;
+        }
+        float s_img = 0.f;
+        if (emit) s_img = stage_state(S, bound);  // the state before chunk c+1 starts block (c+1)/2
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();                          // TMEM read; staging image written
+        tc_fence_after();
+        if (tid == 0) {
+            if (emit) {
+                const size_t ci = image_index(bh, np, (c + 1) >> 1, m);
+                bulk_s2g(img + ci * kImgHalves, stage, kImgBytes);
+                bulk_commit();
+                scales[ci] = s_img;
+            }
+            issue_mma(c + 1);
+            ++mma_issued;
+            if (c + 3 < nc) prefetch(c + 3);      // raw buffer (c+1) & 1 is consumed
+        }
     }
-    if (!ok && tid == 0) {
-        record_error(err, kErrTimeout);
-        // one more bounded chance for the MMA and the row copies in flight to drain
-        if (mma_out) mbar_wait(bar_mma, mma_phase & 1);
-        for (int cc = c; cc < prefetched; ++cc) mbar_wait(bar_raw + (cc & 1), (cc >> 1) & 1);
+    if (nc == 0 && fin) {                         // no tokens: the final state is the initial one
+        float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+    }
+    if (tid == 0) {
+        if (!ok) {
+            record_error(err, kErrTimeout);
+            // one more bounded chance for the MMA and the row copies in flight to drain
+            if (mma_issued > mma_seen) mbar_wait(bar_mma, (mma_issued - 1) & 1);
+            for (int cc = 0; cc < prefetched; ++cc) mbar_wait(bar_raw + (cc & 1), (cc >> 1) & 1);
+        }
+        bulk_wait_all();                          // the image stores have landed before the CTA leaves
     }
     tc_fence_before();
     __syncthreads();
