@@ -226,7 +226,7 @@ mesa_status mesa_forward(const void* q, const void* k, const void* v,
 
 size_t mesa_backward_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
     if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
-    return backward_workspace_bytes(B, H, T, dk, dv, chunk);
+    return backward_workspace_bytes(B, H, T, dk, dv, chunk, dtype);
 }
 
 mesa_status mesa_backward(const void* q, const void* k, const void* v,
@@ -263,7 +263,7 @@ mesa_status mesa_backward(const void* q, const void* k, const void* v,
         for (int r = 0; r < kRanges; ++r)
             if (r != o && ranges[o].p < ranges[r].p + ranges[r].n && ranges[r].p < ranges[o].p + ranges[o].n)
                 return MESA_ERR_INVALID_ARG;
-    const size_t need = backward_workspace_bytes(B, H, T, dk, dv, chunk);
+    const size_t need = backward_workspace_bytes(B, H, T, dk, dv, chunk, dtype);
     if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
     BackwardArgs a{{q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps, tol, nullptr, nullptr,

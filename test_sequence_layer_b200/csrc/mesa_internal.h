@@ -29,7 +29,7 @@ struct ForwardArgs {
     float* G_out;
     void* workspace;
     size_t ws_bytes;
-    float* x_out = nullptr;     // fp32 CUDA-core path only: the CG solutions x_t [B,H,T,dk]
+    float* x_out = nullptr;     // the CG solutions x_t [B,H,T,dk] (fp32), when not null
     bool scan_only = false;     // fp32 CUDA-core path only: the chunk-state scan, no solve
 };
 
@@ -69,7 +69,7 @@ class LaunchTimer {
 // fp32 CUDA-core path (simt_forward.cu).
 size_t simt_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
 cudaError_t forward_simt(const ForwardArgs& a, cudaStream_t st);
-size_t backward_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk);
+size_t backward_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype);
 // Sequence sharding: the state after a slice and its total decay; the state
 // entering slice r from the summaries of slices 0..r-1 (sharded.cu).
 cudaError_t chunk_state(const ForwardArgs& a, float* decay_out, cudaStream_t st);

@@ -530,10 +530,12 @@ __global__ void dlambda_kernel(const float* __restrict__ part, int B, int H, int
 }
 
 struct BwdLayout {
-    size_t states, x, z, rstates, part, total;
+    size_t states, x, z, rstates, part, tcws, oscr, total;
 };
 
-BwdLayout bwd_layout(int B, int H, int T, int dk, int dv, int chunk) {
+// With the tensor-core solve (bf16, d = 128, C = 64) the forward solutions
+// come from it: its workspace and a scratch read-out follow the rest.
+BwdLayout bwd_layout(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t nc = (size_t)((T + chunk - 1) / chunk);
     const size_t BH = (size_t)B * H;
@@ -544,7 +546,13 @@ BwdLayout bwd_layout(int B, int H, int T, int dk, int dv, int chunk) {
     l.z = l.x + up(BH * T * dk * sizeof(float));
     l.rstates = l.z + up(BH * T * sizeof(float));
     l.part = l.rstates + up(BH * se);
-    l.total = l.part + up(BH * nc * dk * sizeof(float));
+    l.tcws = l.part + up(BH * nc * dk * sizeof(float));
+    l.oscr = l.tcws;
+    l.total = l.tcws;
+    if (tc_supported(dk, dv, chunk, dtype)) {
+        l.oscr = l.tcws + up(tc_workspace_bytes(B, H, T));
+        l.total = l.oscr + up(BH * T * dv * sizeof(float));
+    }
     return l;
 }
 
@@ -553,7 +561,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
     const ForwardArgs& f = a.f;
     const int nc = (f.T + CH - 1) / CH;
     const int BH = f.B * f.H;
-    const BwdLayout l = bwd_layout(f.B, f.H, f.T, D, D, CH);
+    const BwdLayout l = bwd_layout(f.B, f.H, f.T, D, D, CH, f.dtype);
     char* ws = static_cast<char*>(f.workspace);
     float* states = reinterpret_cast<float*>(ws + l.states);
     float* X = reinterpret_cast<float*>(ws + l.x);
@@ -561,7 +569,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
     float* R = reinterpret_cast<float*>(ws + l.rstates);
     float* part = reinterpret_cast<float*>(ws + l.part);
 
-    // forward: chunk-start states and the solutions x_t (no read-out)
+    // forward: fp32 chunk-start states and the solutions x_t
     ForwardArgs fa = f;
     fa.out = nullptr;
     fa.iters = nullptr;
@@ -569,8 +577,19 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
     fa.H_out = fa.G_out = nullptr;
     fa.workspace = states;
     fa.x_out = X;
-    cudaError_t e = forward_simt(fa, st);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (tc_supported(f.dk, f.dv, f.chunk, f.dtype)) {
+        // bf16 inputs at d = 128, C = 64: x from the tensor-core solve (the
+        // bf16-mode precision), the fp32 states from the scan alone
+        ForwardArgs ft = fa;
+        ft.workspace = ws + l.tcws;
+        ft.ws_bytes = l.oscr - l.tcws;
+        ft.out = reinterpret_cast<float*>(ws + l.oscr);
+        if ((e = forward_tc(ft, st)) != cudaSuccess) return e;
+        fa.scan_only = true;
+        fa.x_out = nullptr;
+    }
+    if ((e = forward_simt(fa, st)) != cudaSuccess) return e;
 
     using L = CgSmem<D, D, CH>;
     auto adj = simt_adj_kernel<D, D, CH, Tin>;
@@ -624,8 +643,8 @@ cudaError_t dispatch_backward(const BackwardArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-size_t backward_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk) {
-    return bwd_layout(B, H, T, dk, dv, chunk).total;
+size_t backward_workspace_bytes(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
+    return bwd_layout(B, H, T, dk, dv, chunk, dtype).total;
 }
 
 cudaError_t backward_simt(const BackwardArgs& a, cudaStream_t st) {

@@ -164,7 +164,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
              const __nv_bfloat16* __restrict__ v, const float* __restrict__ gamma,
              const float* __restrict__ beta, const float* __restrict__ lambda, int H, int T, int np,
              int cg_steps, float tol, const __half* __restrict__ img, const float* __restrict__ scales,
-             float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err) {
+             float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err,
+             float* __restrict__ x_out) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Hs = smem + BlkSmem::oH;
@@ -491,6 +492,11 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
             for (int i = 0; i < 8; ++i) xr[8 * h2 + i] = make_float2(xv[2 * i], xv[2 * i + 1]);
         }
+        if (x_out && valid) {                          // the solutions themselves, when asked for (fp32)
+            float4* dst = reinterpret_cast<float4*>(x_out + (base + tok) * kD + col0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(xr[2 * i].x, xr[2 * i].y, xr[2 * i + 1].x, xr[2 * i + 1].y);
+        }
         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
@@ -641,7 +647,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
         tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
-            img, scales, a.out, a.iters, err);
+            img, scales, a.out, a.iters, err, a.x_out);
     }
 #ifdef MESA_DEBUG
     if (inject) {

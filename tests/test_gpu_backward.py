@@ -3,20 +3,25 @@
 Every gradient (dq, dk, dv, dgamma, dbeta, dlambda) is compared on small
 cases that span several chunks with a ragged tail; the full-size workload
 compares sampled (b, h) sequences (dlambda, a sum over the batch, is covered
-by the small cases). The backward computes in fp32 for every input dtype, so
-the fp32 bound applies to bf16 inputs too (the oracle reads the same
-bf16-rounded values).
+by the small cases). The backward computes in fp32 on the CUDA cores, so the
+fp32 bound applies (the oracle reads the same bf16-rounded inputs), except
+for bf16 inputs at d = 128, C = 64: there the forward solutions come from the
+tensor-core solve (fp16 operands), and the bf16-mode bound applies.
 """
 import numpy as np
 import pytest
 import torch
 
 import mesa_inputs as mi
-from helpers import TOL_F32, err_report, rel_err
+from helpers import TOL_BF16, TOL_F32, err_report, rel_err
 
 pytestmark = pytest.mark.gpu
 
 NAMES = ("dq", "dk", "dv", "dgamma", "dbeta", "dlambda")
+
+
+def bound(dtype, d, chunk):
+    return TOL_BF16 if (dtype, d, chunk) == ("bf16", 128, 64) else TOL_F32
 
 
 @pytest.fixture(scope="module")
@@ -51,6 +56,7 @@ CASES = [
     ("f32", 128, 64, 150, 1, 2, 15, 0.0),
     ("f32", 128, 16, 40, 2, 1, 15, 0.0),
     ("bf16", 128, 64, 200, 2, 1, 15, 0.0),
+    ("bf16", 64, 64, 150, 1, 2, 15, 0.0),
     ("f32", 64, 32, 64, 1, 1, 3, 0.0),
 ]
 
@@ -64,7 +70,7 @@ def test_backward_matches_oracle(mesa, oracle_mod, case):
     g = gpu_backward(mesa, to_dev(x, dtype), torch.from_numpy(do).cuda(), chunk, N, tol)
     ref = oracle_mod.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], do, N, tol)
     for n in NAMES:
-        assert rel_err(g[n], ref[n]) <= TOL_F32, (n, err_report(g[n], ref[n]))
+        assert rel_err(g[n], ref[n]) <= bound(dtype, d, chunk), (n, err_report(g[n], ref[n]))
 
 
 def test_backward_tolerance_stopping(mesa, oracle_mod):
@@ -128,4 +134,4 @@ def test_backward_full_size_sampled(mesa, oracle_mod):
     ref = oracle_mod.backward(host["q"], host["k"], host["v"], host["gamma"], host["beta"], host["lam"], do_host, 15)
     for n, t in zip(NAMES[:5], res[:5]):
         got = np.stack([t[b, h].cpu().numpy() for (b, h) in pairs])[None]
-        assert rel_err(got, ref[n]) <= TOL_F32, (n, err_report(got, ref[n]))
+        assert rel_err(got, ref[n]) <= TOL_BF16, (n, err_report(got, ref[n]))
