@@ -135,3 +135,27 @@ def test_backward_full_size_sampled(mesa, oracle_mod):
     for n, t in zip(NAMES[:5], res[:5]):
         got = np.stack([t[b, h].cpu().numpy() for (b, h) in pairs])[None]
         assert rel_err(got, ref[n]) <= TOL_BF16, (n, err_report(got, ref[n]))
+
+
+@pytest.mark.parametrize("dtype,d,chunk,T", [("f32", 16, 16, 1), ("bf16", 128, 64, 1), ("f32", 64, 64, 64),
+                                              ("bf16", 128, 64, 128)])
+def test_backward_edge_lengths(mesa, oracle_mod, dtype, d, chunk, T):
+    """A single token (the state is one outer product) and sequences that end
+    exactly on a chunk or block boundary."""
+    w = mi.Workload("t", 1, 2, T, d, d, chunk, dtype, 15, 0.0, False, 31)
+    x = mi.batch(w)
+    do = mi.dout(31, 1, 2, T, d)
+    g = gpu_backward(mesa, to_dev(x, dtype), torch.from_numpy(do).cuda(), chunk, 15, 0.0)
+    ref = oracle_mod.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], do, 15)
+    for n in NAMES:
+        assert rel_err(g[n], ref[n]) <= bound(dtype, d, chunk), (n, err_report(g[n], ref[n]))
+
+
+def test_backward_empty_sequence(mesa):
+    e = torch.empty((1, 2, 0, 16), device="cuda")
+    g = torch.empty((1, 2, 0), device="cuda")
+    lam = torch.ones((2, 16), device="cuda")
+    res = mesa.backward(e, e, e, g, g, lam, e, chunk=16, cg_steps=4)
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    assert torch.equal(res[5], torch.zeros_like(lam))
