@@ -1,4 +1,4 @@
-// simt_backward.cu -- fp32 CUDA-core chunkwise backward of the Mesa layer.
+// simt_backward.cu -- chunkwise backward of the Mesa layer on the CUDA cores (fp32).
 //
 // The pages claim the layer trains in time linear in T but give no backward
 // method. Reading taken here: implicit differentiation of the solution map
@@ -26,7 +26,10 @@
 //   Gbar_s = sum_{t in c, t>=s} N_st do_t x_t^T + e^{b_last - b_s} Ghat_c.
 //
 // Kernels (all fp32, 256 threads, thread layout of simt_chunk.cuh):
-//   forward scan + CG (simt_forward.cu) with the solutions x_t saved;
+//   the forward solutions x_t: the fp32 scan + CG of simt_forward.cu, or,
+//                     for bf16 inputs at d = 128, C = 64, the tensor-core
+//                     scan and solve (x stored in fp32) next to the fp32 scan
+//                     alone for the chunk states;
 //   simt_adj_kernel   grid (chunks, B*H): right-hand side G_t^T do_t, the
 //                     adjoint CG, H_t x_t, then dq, e_t and per-chunk dlambda sums;
 //   simt_rscan_kernel grid (state tiles, B*H): the reverse chunk scan of
