@@ -32,7 +32,7 @@
 //                     alone for the chunk states;
 //   simt_adj_kernel   grid (chunks, B*H): right-hand side G_t^T do_t, the
 //                     adjoint CG, H_t x_t, then dq, e_t and per-chunk dlambda sums;
-//   simt_rscan_kernel grid (state tiles, B*H): the reverse chunk scan of
+//   simt_rscan_kernel grid (64 x 64 state tiles, B*H): the reverse chunk scan of
 //                     Hhat_c and Ghat_c;
 //   simt_grad_kernel  grid (chunks, B*H): dk, dv, dbeta and z_t;
 //   dgamma_kernel     grid (B*H): the suffix sums of z;
@@ -221,14 +221,15 @@ __global__ void __launch_bounds__(kThreads)
 simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, const float* __restrict__ xsol,
                   const float* __restrict__ gamma, int T, int nc, float* __restrict__ rstates) {
     static_assert(DK == DV, "dk == dv");
-    constexpr int TL = DK < 32 ? DK : 32;
+    constexpr int TL = DK < 64 ? DK : 64;                  // tile edge
+    constexpr int R = TL / 16;                             // each thread: R x R elements of the tile
+    constexpr int TS = TL + 4;                             // shared row stride (16-byte rows)
     constexpr int TPR = DK / TL;
     constexpr int H_TILES = TPR * TPR;
-    constexpr int EPT = (TL * TL + kThreads - 1) / kThreads;
     constexpr size_t SE = (size_t)DK * DK + (size_t)DV * DK;
 
-    __shared__ float sA[CH][TL + 1];
-    __shared__ float sX[CH][TL + 1];
+    __shared__ __align__(16) float sA[CH * TS];
+    __shared__ __align__(16) float sX[CH * TS];
     __shared__ float sb[CH];
     __shared__ float sw[CH];
 
@@ -236,23 +237,23 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
     int tile = blockIdx.x;
     const bool isG = tile >= H_TILES;
     if (isG) tile -= H_TILES;
-    const int i0 = (tile / TPR) * TL, j0 = (tile % TPR) * TL;
+    const int trow = (tile / TPR) * TL, tcol = (tile % TPR) * TL;
+    const int i0 = trow + (threadIdx.x >> 4) * R, j0 = tcol + (threadIdx.x & 15) * R;
     const float* A = isG ? dout : u;
     const size_t mat_off = isG ? (size_t)DK * DK : 0;
 
-    float S[EPT];
+    float S[R][R];
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) S[e] = 0.f;
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int c = 0; c < R; ++c) S[r][c] = 0.f;
     for (int c = nc - 1; c >= 0; --c) {
         const int t0 = c * CH;
         const int n = min(CH, T - t0);
         const size_t base = (size_t)bh * T + t0;
         float* dst = rstates + ((size_t)bh * nc + c) * SE + mat_off;
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int idx = threadIdx.x + kThreads * e;
-            if (idx < TL * TL) dst[(size_t)(i0 + idx / TL) * DK + j0 + idx % TL] = S[e];
-        }
+        for (int r = 0; r < R; ++r) store_n<R>(dst + (size_t)(i0 + r) * DK + j0, S[r]);
         chunk_log_cumsum<CH>(gamma, base, n, sb);
         __syncthreads();
         const float blast = sb[CH - 1];
@@ -261,22 +262,17 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
         for (int idx = threadIdx.x; idx < CH * TL; idx += kThreads) {
             const int t = idx / TL, col = idx % TL;
             const bool ok = t < n;
-            sA[t][col] = ok ? sw[t] * A[(base + t) * DK + i0 + col] : 0.f;
-            sX[t][col] = ok ? xsol[(base + t) * DK + j0 + col] : 0.f;
+            sA[t * TS + col] = ok ? sw[t] * A[(base + t) * DK + trow + col] : 0.f;
+            sX[t * TS + col] = ok ? xsol[(base + t) * DK + tcol + col] : 0.f;
         }
         __syncthreads();
         const float Gam = expf(blast);
+        float acc[R][R];
+        tile_outer<CH, TL>(sA, sX, acc);
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int idx = threadIdx.x + kThreads * e;
-            if (idx < TL * TL) {
-                const int i = idx / TL, j = idx % TL;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int t = 0; t < CH; ++t) acc = fmaf(sA[t][i], sX[t][j], acc);
-                S[e] = fmaf(Gam, S[e], acc);
-            }
-        }
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int cc = 0; cc < R; ++cc) S[r][cc] = fmaf(Gam, S[r][cc], acc[r][cc]);
         __syncthreads();
     }
 }
@@ -605,7 +601,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
             f.T, nc, f.cg_steps, f.tol, states, a.dq, Z, part);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    constexpr int TL = D < 32 ? D : 32;
+    constexpr int TL = D < 64 ? D : 64;
     constexpr int tiles = 2 * (D / TL) * (D / TL);
     {
         LaunchTimer timer(kKindBwdRscan, st);

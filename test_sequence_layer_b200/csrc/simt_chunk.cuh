@@ -53,6 +53,53 @@ __device__ __forceinline__ float sum16(float v) {
     return v;
 }
 
+// N consecutive floats (N = 1, 2 or 4; the address aligned to N floats).
+template <int N>
+__device__ __forceinline__ void load_n(const float* p, float (&v)[N]) {
+    if constexpr (N == 4) {
+        const float4 f = *reinterpret_cast<const float4*>(p);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else if constexpr (N == 2) {
+        const float2 f = *reinterpret_cast<const float2*>(p);
+        v[0] = f.x; v[1] = f.y;
+    } else {
+        v[0] = p[0];
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void store_n(float* p, const float (&v)[N]) {
+    if constexpr (N == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else if constexpr (N == 2) *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    else p[0] = v[0];
+}
+
+// One chunk's contribution to a TL x TL tile of a chunk state: thread
+// (ty, tx) = (tid / 16, tid % 16) owns tile rows ty R .. + R - 1 and columns
+// tx R .. + R - 1 (R = TL / 16) and forms
+//     acc[r][c] = sum_{t < CH} sA[t][ty R + r] * sB[t][tx R + c]
+// in order of t, from two [CH][TL + 4] shared tiles (16-byte aligned rows):
+// R + R loads per R x R FMAs.
+template <int CH, int TL>
+__device__ __forceinline__ void tile_outer(const float* sA, const float* sB, float (&acc)[TL / 16][TL / 16]) {
+    constexpr int R = TL / 16, TS = TL + 4;
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int c = 0; c < R; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < CH; ++t) {
+        float av[R], bv[R];
+        load_n<R>(sA + t * TS + ty * R, av);
+        load_n<R>(sB + t * TS + tx * R, bv);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int c = 0; c < R; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+}
+
 template <int DK, int DV, int CH>
 struct CgSmem {
     static constexpr int DKP = DK + 1, DVP = DV + 1, CHP = CH + 1;

@@ -37,14 +37,15 @@ simt_scan_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v,
                  int T, int nc, const float* __restrict__ H_in, const float* __restrict__ G_in,
                  float* __restrict__ states, float* __restrict__ H_out, float* __restrict__ G_out) {
     static_assert(DK == DV, "dk == dv");
-    constexpr int TL = DK < 32 ? DK : 32;                  // tile edge
+    constexpr int TL = DK < 64 ? DK : 64;                  // tile edge
+    constexpr int R = TL / 16;                             // each thread: R x R elements of the tile
+    constexpr int TS = TL + 4;                             // shared row stride (16-byte rows)
     constexpr int TPR = DK / TL;                           // tiles per row of a matrix
     constexpr int H_TILES = TPR * TPR;
-    constexpr int EPT = (TL * TL + kThreads - 1) / kThreads;
     constexpr size_t SE = (size_t)DK * DK + (size_t)DV * DK;
 
-    __shared__ float sA[CH][TL + 1];
-    __shared__ float sKc[CH][TL + 1];
+    __shared__ __align__(16) float sA[CH * TS];
+    __shared__ __align__(16) float sKc[CH * TS];
     __shared__ float sb[CH];
     __shared__ float sw[CH];
 
@@ -52,18 +53,20 @@ simt_scan_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v,
     int tile = blockIdx.x;
     const bool isG = tile >= H_TILES;
     if (isG) tile -= H_TILES;
-    const int i0 = (tile / TPR) * TL, j0 = (tile % TPR) * TL;
+    const int i0 = (tile / TPR) * TL + (threadIdx.x >> 4) * R;   // this thread's first row ...
+    const int j0 = (tile % TPR) * TL + (threadIdx.x & 15) * R;   // ... and column in the matrix
+    const int tcol = (tile % TPR) * TL, trow = (tile / TPR) * TL;
     const Tin* A = isG ? v : k;
     const size_t mat_off = isG ? (size_t)DK * DK : 0;
     const float* init = isG ? G_in : H_in;
     float* fin = isG ? G_out : H_out;
 
-    float S[EPT];
+    float S[R][R];
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-        const int idx = threadIdx.x + kThreads * e;
-        S[e] = 0.f;
-        if (idx < TL * TL && init) S[e] = init[(size_t)bh * DK * DK + (size_t)(i0 + idx / TL) * DK + j0 + idx % TL];
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int c = 0; c < R; ++c)
+            S[r][c] = init ? init[(size_t)bh * DK * DK + (size_t)(i0 + r) * DK + j0 + c] : 0.f;
     }
 
     for (int c = 0; c < nc; ++c) {
@@ -72,10 +75,7 @@ simt_scan_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v,
         const size_t base = (size_t)bh * T + t0;
         float* dst = states + ((size_t)bh * nc + c) * SE + mat_off;
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int idx = threadIdx.x + kThreads * e;
-            if (idx < TL * TL) dst[(size_t)(i0 + idx / TL) * DK + j0 + idx % TL] = S[e];
-        }
+        for (int r = 0; r < R; ++r) store_n<R>(dst + (size_t)(i0 + r) * DK + j0, S[r]);
         chunk_log_cumsum<CH>(gamma, base, n, sb);
         __syncthreads();
         const float blast = sb[CH - 1];
@@ -85,30 +85,22 @@ simt_scan_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v,
         for (int idx = threadIdx.x; idx < CH * TL; idx += kThreads) {
             const int t = idx / TL, col = idx % TL;
             const bool ok = t < n;
-            sA[t][col] = ok ? sw[t] * ld_in(A, (base + t) * DK + i0 + col) : 0.f;
-            sKc[t][col] = ok ? ld_in(k, (base + t) * DK + j0 + col) : 0.f;
+            sA[t * TS + col] = ok ? sw[t] * ld_in(A, (base + t) * DK + trow + col) : 0.f;
+            sKc[t * TS + col] = ok ? ld_in(k, (base + t) * DK + tcol + col) : 0.f;
         }
         __syncthreads();
         const float Gam = expf(blast);
+        float acc[R][R];
+        tile_outer<CH, TL>(sA, sKc, acc);
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int idx = threadIdx.x + kThreads * e;
-            if (idx < TL * TL) {
-                const int i = idx / TL, j = idx % TL;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int t = 0; t < CH; ++t) acc = fmaf(sA[t][i], sKc[t][j], acc);
-                S[e] = fmaf(Gam, S[e], acc);
-            }
-        }
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int cc = 0; cc < R; ++cc) S[r][cc] = fmaf(Gam, S[r][cc], acc[r][cc]);
         __syncthreads();
     }
     if (fin) {
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int idx = threadIdx.x + kThreads * e;
-            if (idx < TL * TL) fin[(size_t)bh * DK * DK + (size_t)(i0 + idx / TL) * DK + j0 + idx % TL] = S[e];
-        }
+        for (int r = 0; r < R; ++r) store_n<R>(fin + (size_t)bh * DK * DK + (size_t)(i0 + r) * DK + j0, S[r]);
     }
 }
 
@@ -271,7 +263,7 @@ cudaError_t launch_simt(const ForwardArgs& a, cudaStream_t st) {
     const int nc = (a.T + CH - 1) / CH;
     const int BH = a.B * a.H;
     float* states = reinterpret_cast<float*>(a.workspace);
-    constexpr int TL = D < 32 ? D : 32;
+    constexpr int TL = D < 64 ? D : 64;
     constexpr int tiles = 2 * (D / TL) * (D / TL);
     {
         LaunchTimer timer(kKindSimtScan, st);
