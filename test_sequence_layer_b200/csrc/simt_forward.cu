@@ -17,7 +17,8 @@
 //
 // Kernels:
 //   simt_scan_kernel  grid (state tiles, B*H): one CTA walks the chunks of one
-//                     sequence for one 32x32 (or 16x16) tile of H or G, writing
+//                     sequence for one 64x64 (d < 64: d x d) tile of H or G, each
+//                     thread a 4x4 block of it (1x1, 2x2 for d = 16, 32), writing
 //                     the chunk-start states to the workspace.
 //   simt_cg_kernel    grid (chunks, B*H): one CTA runs all CG iterations of one
 //                     chunk with H_c, K, V, P and the decay mask in shared
