@@ -58,6 +58,9 @@ MUTANTS = {
                               "part[(size_t)bh * dk + i] += ut[i] * xt[i];"),
     "adjoint right-hand side G do instead of G^T do": ("for (int i = 0; i < dv; ++i) s += Gm[(size_t)i * dk + j] * dot_[i];",
                                                        "for (int i = 0; i < dv; ++i) s += Gm[(size_t)j * dk + i] * dot_[i];"),
+    "backward dbeta without the value statistics": (
+        "for (int j = 0; j < dk; ++j) db += vt[i] * Gbar[(size_t)i * dk + j] * kt[j];",
+        "for (int j = 0; j < dk; ++j) db += 0.0 * vt[i] * Gbar[(size_t)i * dk + j] * kt[j];"),
     "backward dlambda from one batch row only": ("for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * dk + i];",
                                                  "for (int b = 0; b < 1; ++b) s += part[((size_t)b * H + h) * dk + i];"),
 }
@@ -110,6 +113,7 @@ PIN_SUBSET = [
     lambda o: pins.test_warm_cg_from_the_solution_stops_at_once(o),
     lambda o: pins.test_backward_matches_finite_differences_of_the_exact_layer(o),
     lambda o: pins.test_backward_one_step_closed_form(o),
+    lambda o: pins.test_backward_respects_the_beta_lambda_scale_invariance(o),
 ]
 
 

@@ -543,3 +543,16 @@ def test_state_after_a_slice_is_affine_in_the_initial_state(oracle_mod):
     D = np.prod(gamma, axis=-1)[..., None, None]
     np.testing.assert_allclose(H1, D * S_H + H0, rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(G1, D * S_G + G0, rtol=1e-12, atol=1e-14)
+
+
+def test_backward_respects_the_beta_lambda_scale_invariance(oracle_mod):
+    """(beta, Lambda) -> (c beta, c Lambda) leaves o unchanged (the objective
+    is scaled as a whole), so the exact gradient has no component along that
+    direction: per head, sum over its tokens of beta dbeta plus
+    sum_i lambda_i dlambda_i is zero. Holds when the adjoint has converged."""
+    x, dout = _bwd_inputs(4, B=2, H=2, T=5, d=3)
+    g = oracle_mod.backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], dout, 9, 1e-14)
+    for h in range(2):
+        along = np.sum(x["beta"][:, h] * g["dbeta"][:, h]) + np.sum(x["lam"][h] * g["dlambda"][h])
+        scale = np.sum(np.abs(x["beta"][:, h] * g["dbeta"][:, h])) + np.sum(np.abs(x["lam"][h] * g["dlambda"][h]))
+        assert abs(along) <= 1e-10 * scale, (h, along, scale)
