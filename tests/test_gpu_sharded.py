@@ -76,3 +76,30 @@ def test_chunk_state_of_an_empty_slice(mesa):
     torch.cuda.synchronize()
     assert torch.equal(Ho, H_in) and torch.equal(Go, G_in)
     assert torch.equal(dec, torch.ones_like(dec))
+
+
+def test_sharded_forward_with_tolerance_stopping(mesa, oracle_mod):
+    """tol = 1e-3 with the gamma mixture: each slice's solve starts from the
+    prefix state and stops per token as the unsharded forward does."""
+    bounds = (0, 70, 140, 200)
+    w = mi.Workload("t", 1, 2, 200, 32, 32, 16, "f32", 30, 1e-3, True, 23)
+    x = mi.batch(w)
+    dev = {n: torch.from_numpy(np.ascontiguousarray(x[n])).cuda() for n in ("q", "k", "v", "gamma", "beta", "lam")}
+    sl = [slice(bounds[i], bounds[i + 1]) for i in range(len(bounds) - 1)]
+    part = lambda n, s: dev[n][:, :, s].contiguous()        # noqa: E731
+    summ = [mesa.chunk_state(part("k", s), part("v", s), part("gamma", s), part("beta", s), chunk=16) for s in sl]
+    H_all, G_all, d_all = (torch.stack([a[i] for a in summ]) for i in range(3))
+    outs, its = [], []
+    for r, s in enumerate(sl):
+        H_in, G_in = mesa.state_prefix(H_all, G_all, d_all, r)
+        o, it = mesa.forward(part("q", s), part("k", s), part("v", s), part("gamma", s), part("beta", s), dev["lam"],
+                             chunk=16, cg_steps=30, tol=1e-3, H_in=H_in, G_in=G_in, return_iters=True)
+        outs.append(o)
+        its.append(it)
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    got = torch.cat(outs, dim=2).cpu().numpy()
+    ref, it_ref, _, _ = oracle_mod.forward_cg(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], 30, 1e-3)
+    assert rel_err(got, ref) <= 2e-2, err_report(got, ref)
+    diff = np.abs(torch.cat(its, dim=2).cpu().numpy().astype(np.int64) - it_ref)
+    assert diff.max() <= 1
