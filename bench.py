@@ -49,9 +49,8 @@ def load_peaks():
 
 
 # DRAM bytes moved per token (per head for the decode step) by each kernel, from
-# one ncu capture (profiles/tc_kernels_bf16_T2048.md, profiles/decode_step_4096heads.md,
-# profiles/preprocess_bf16_T8192.md:
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch / units of that launch).
+# one ncu capture of that kernel on a small case of its workload
+# (dram__bytes_read.sum + dram__bytes_write.sum of one launch / units of that launch).
 # Reported only while the kernel source still hashes to the captured version;
 # otherwise the field is null.
 MEASURED_TRAFFIC = {

@@ -91,7 +91,14 @@ size_t mesa_forward_workspace_size(int B, int H, int T, int dk, int dv, int chun
  *                (the tail behaves as if padded with beta = 0, gamma = 1).
  *                The tensor-core path serves dtype = MESA_BF16,
  *                dk = dv = 128, chunk = 64; every other supported shape runs
- *                the fp32 CUDA-core path.
+ *                the fp32 CUDA-core path. The tensor-core path divides every
+ *                MMA operand (keys, values, decay mask, states, CG
+ *                directions) by a power of two at or above its largest entry
+ *                before rounding it to fp16, so it accepts the same range of
+ *                magnitudes as float32; its rounding is ~2^-11 relative per
+ *                operand, which the solve amplifies by up to the condition
+ *                number of H_t + Lambda (bf16-mode accuracy holds while
+ *                beta |k|^2 stays within a few hundred times lambda).
  *   cg_steps     maximum CG updates per token, 0..1024.
  *   tol          relative residual tolerance; <= 0 runs exactly cg_steps
  *                updates (unless breakdown). NaN is an argument error.

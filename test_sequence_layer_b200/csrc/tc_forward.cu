@@ -13,13 +13,17 @@
 //     H_{c+1} = e^{b_last} H_c + K^T diag(w) K,  w_j = beta_j e^{b_last-b_j}
 //
 // Numerics. Every tensor-core operand is fp16 (same tensor rate as bf16,
-// 8x finer rounding), accumulation is fp32:
-//   * bf16 q, k, v convert exactly to fp16 (normalised keys and queries are
-//     far inside the fp16 range; v is scaled per chunk by a power of two);
-//   * the chunk-start states are stored as fp16 images scaled per chunk by a
-//     power of two s >= 1 (so |H/s| <= 1);
-//   * the CG direction of each token is scaled by 1/|r| before rounding, so
-//     its fp16 image has unit-order entries; every CG vector (x, r, p) and
+// 8x finer rounding), accumulation is fp32. Each fp16 image is divided by a
+// power of two chosen from a bound on its entries, so that it lies in
+// [-1, 1] (or, for the score images, within a small fixed multiple of 1)
+// whatever the magnitudes of beta, Lambda, k or v; every scale is undone
+// exactly in the fp32 epilogue:
+//   * keys: K / sK, sK >= max |k| over the block; values: V / sV likewise;
+//   * the decay mask: M sK^2 / sW with sW >= max_j beta_j sK^2 >= max M sK^2;
+//   * the chunk-start states: fp16 images H / sH, G / sG with sH, sG >= a
+//     bound on the state's entries (tc_scan.cu);
+//   * the CG direction of each token is scaled by ~1/|r| before rounding, and
+//     the solution by 1/|x| for the read-out; every CG vector (x, r, p) and
 //     scalar stays fp32;
 //   * the scan splits beta_j e^{b_last-b_j} k_j into an fp16 hi/lo pair, so
 //     the fp32 running states carry ~22-bit products (tc_scan.cu).
@@ -68,7 +72,9 @@ __device__ __forceinline__ void wait_mma_each(uint64_t* bar, uint32_t parity, fl
 // chunks with the second chunk's state H_{c+1} expanded into its definition,
 // so one chunk-start state serves 128 tokens and every product has M = N = 128:
 //   S = P K^T,  W = M o S (lower triangular),  U = P H_c^T,  Z = W K,
-//   y_t = s_t sH (e^{b_t} U_t + Z_t) + lambda p_t.
+//   y_t = s_t (sH e^{b_t} U_t + sW Z_t) + lambda p_t
+// with P the direction images p_t / s_t, K = k / sK and M the mask image
+// M_tj sK^2 / sW.
 // Thread layout: 16 warps; warp w holds the 32 tokens of TMEM lane quadrant
 // w % 4 (lane = token) and the 32 columns 32 * (w / 4) .. + 31 of each.
 // TMEM columns: U [0,128), S / Z / y [128,256), x [256,384), r [384,512);
@@ -83,7 +89,7 @@ struct BlkSmem {
     static constexpr int oW = 98304;              // masked scores [128 t][128 j] (32 KB)
     static constexpr int oG = 131072;             // value-state image [128 i][128 k] (32 KB), fetched at start
     static constexpr int kMS = 136;               // mask row stride in halves (conflict-free 16-byte rows)
-    static constexpr int oM = 163840;             // decay mask / sH, fp16 [128 t][128 j], stride kMS
+    static constexpr int oM = 163840;             // decay mask M sK^2 / sW, fp16 [128 t][128 j], stride kMS
     static constexpr int oLam = oM + kBlk * kMS * 2;   // lambda [128]
     static constexpr int oEb = oLam + 512;        // e^{b_t} [128]
     static constexpr int oB = oEb + 512;          // b_t [128]
@@ -251,17 +257,36 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     if (tid == 0 && !mbar_wait(bar_in, 0)) *abort_flag = 1.f;
     __syncthreads();
 
-    // gates, beta, key image (from the staged rows)
+    // gates and beta; the raw key rows (held in registers until the key image
+    // is written) and the block's maxima of |k| and beta, per warp into misc
     if (w == 0) warp_gate_cumsum128(gates_bulk ? gstage : gamma + base, n, sbc);
-    if (tid < kBlk) sbeta[tid] = (tid < n) ? (gates_bulk ? gstage[kBlk + tid] : beta[base + tid]) : 0.f;
+    float bmax = 0.f, kmax = 0.f;
+    if (tid < kBlk) {
+        bmax = (tid < n) ? (gates_bulk ? gstage[kBlk + tid] : beta[base + tid]) : 0.f;
+        sbeta[tid] = bmax;
+    }
+    uint4 kraw[4];
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
         const int cid = tid + kBlkThreads * rep;       // 2048 16-byte chunks
         const int j = cid >> 4, cc = cid & 15;
-        uint4 rk = make_uint4(0, 0, 0, 0);
-        if (j < n) rk = *reinterpret_cast<const uint4*>(Ps + j * 256 + cc * 16);
-        *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
-            bf16x8_to_f16x8(rk, 1.f);
+        kraw[rep] = make_uint4(0, 0, 0, 0);
+        if (j < n) kraw[rep] = *reinterpret_cast<const uint4*>(Ps + j * 256 + cc * 16);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[rep]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(b2[i]);
+            kmax = fmaxf(kmax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
+    }
+    if (lane == 0) {
+        misc[w] = kmax;
+        if (w < 4) misc[16 + w] = bmax;
     }
     // CG state: x = 0 and r = q in TMEM, p = q in registers; this thread: token tok, columns col0..col0+31
     float2 p[16];
@@ -286,21 +311,41 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tmem_st32_x8(tl + kColX + col0 + 8 * h2, z);
         tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
     }
-    __syncthreads();                                   // gates and beta visible, staged rows consumed
+    __syncthreads();                                   // gates, beta, maxima visible; staged rows consumed
+    // key scale sK >= max |k| and mask scale sW >= max_j beta_j sK^2 (powers of two)
+    float sK, sW;
+    {
+        float km = misc[0], bm = misc[16];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) km = fmaxf(km, misc[i]);
+#pragma unroll
+        for (int i = 17; i < 20; ++i) bm = fmaxf(bm, misc[i]);
+        sK = pow2_ceil(km);
+        sW = pow2_ceil(bm * sK * sK);
+        const float inv_sK = 1.f / sK;
+#pragma unroll
+        for (int rep = 0; rep < 4; ++rep) {            // key image K / sK
+            const int cid = tid + kBlkThreads * rep;
+            const int j = cid >> 4, cc = cid & 15;
+            *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
+                bf16x8_to_f16x8(kraw[rep], inv_sK);
+        }
+    }
     if (tid < kBlk) seb[tid] = expf(sbc[tid]);
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) reinterpret_cast<uint4*>(Ws)[tid + kBlkThreads * rep] = make_uint4(0, 0, 0, 0);
     {
-        // M_tj / sH for j <= t, as fp16 pairs. The exponent b_t - b_j is <= 0; the
-        // fast exponential's few-ulp error is far below the fp16 rounding that follows.
-        const float inv_sH = 1.f / sH;                 // power of two: exact
+        // M_tj sK^2 / sW for j <= t (at most 1), as fp16 pairs. The exponent b_t - b_j
+        // is <= 0; the fast exponential's few-ulp error is far below the fp16 rounding
+        // that follows.
+        const float msc = sK * sK / sW;                // powers of two: exact
         for (int e = tid; e < kBlk * kBlk / 2; e += kBlkThreads) {
             const int tt = e >> 6, j = 2 * (e & 63);
             float m0 = 0.f, m1 = 0.f;
             if (tt < n) {
                 const float bt = sbc[tt];
-                if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * inv_sH;
-                if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * inv_sH;
+                if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * msc;
+                if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * msc;
             }
             *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
         }
@@ -331,9 +376,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     auto issue_Z = [&]() {      // Z = W K -> columns [128, 256)
         issue_k128(tbase + kColS, smem_addr(Ws), smem_addr(Ks), 16384, 16384, 8192, 2048, kIdKM);
     };
-    // S (TMEM) -> decay-masked, scaled scores -> score image. The quarter of
+    // S (TMEM) -> decay-masked scores -> score image. The quarter of
     // tokens 0..63 against keys 64..127 lies above the diagonal: it stays zero.
-    auto masked_scores = [&](float extra) {
+    auto masked_scores = [&]() {
         if (q4 < 2 && cq >= 2) return;                 // warp-uniform
         const __half* mrow = Mk + tok * BlkSmem::kMS + col0;
         float2 wv[16];
@@ -349,8 +394,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int c = 4 * g + i;
-                    wv[8 * h2 + c] = __fmul2_rn(__half22float2(m2[i]),
-                                                make_float2(sv[2 * c] * extra, sv[2 * c + 1] * extra));
+                    wv[8 * h2 + c] = __fmul2_rn(__half22float2(m2[i]), make_float2(sv[2 * c], sv[2 * c + 1]));
                 }
             }
         }
@@ -373,7 +417,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             mma_commit(bar_u);
         }
         wait_mma_each(bar_s, ph & 1, abort_flag);
-        masked_scores(1.f);
+        masked_scores();
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -390,8 +434,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         wait_mma_each(bar_z, ph & 1, abort_flag);
         ++ph;
 
-        // y = s sH (e^b U + Z) + lambda p (written over Z); partials p.y, r.y, y.y, r.r
-        const float c_u = s * sH * eb, c_z = s * sH;
+        // y = s (sH e^b U + sW Z) + lambda p (written over Z); partials p.y, r.y, y.y, r.r
+        const float c_u = s * sH * eb, c_z = s * sW;
         float4 d;
         {
             float2 a = make_float2(0.f, 0.f), b = a, cc = a, e = a;
@@ -475,7 +519,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tmem_wait_st();
     }
 
-    // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern ----
+    // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern,
+    // with X-hat = x / |x|, V / sV (sV >= max |v|) and the same key and mask images ----
     if (tid == 0) {            // raw value rows into the dead H buffer, while x is normalised
         mbar_arrive_expect_tx(bar_v, row_bytes);
         bulk_g2s(Hs, v + base * kD, row_bytes, bar_v);
@@ -531,7 +576,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     float vm = misc[0];
 #pragma unroll
     for (int i = 1; i < 16; ++i) vm = fmaxf(vm, misc[i]);
-    const float sV = pow2_ceil_at_least_one(vm);
+    const float sV = pow2_ceil(vm);
     const float sG = scales[iG];
     bool ok = *abort_flag == 0.f;
     if (ok) {
@@ -540,7 +585,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             mma_commit(bar_s);
         }
         wait_mma_each(bar_s, ph & 1, abort_flag);
-        masked_scores(sH * sV / sG);           // mask holds 1/sH
+        masked_scores();                       // W' = (M sK^2 / sW) o (X-hat (K / sK)^T)
         const float inv_sV = 1.f / sV;
 #pragma unroll
         for (int rep = 0; rep < 4; ++rep) {    // the key image is dead: values take its place
@@ -575,7 +620,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         ok = *abort_flag == 0.f;
     }
     if (ok) {
-        const float cu = xs * sG * eb, cz = xs * sG;
+        // G x = xs sG U';  sum_j M_tj (x.k_j) v_j = xs sV sW / sK Z'
+        const float cu = xs * sG * eb, cz = xs * sV * sW / sK;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
             float uv[16], zv[16];

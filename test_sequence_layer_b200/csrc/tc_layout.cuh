@@ -22,12 +22,18 @@ constexpr int kC = 64;           // chunk length
 constexpr uint32_t kImgBytes = kD * kD * 2;      // one fp16 state image
 constexpr size_t kImgHalves = (size_t)kD * kD;
 
-// Power of two >= max(m, 1).
-__device__ __forceinline__ float pow2_ceil_at_least_one(float m) {
-    if (!(m > 1.f)) return 1.f;
-    int e;
-    const float f = frexpf(m, &e);       // m = f * 2^e, f in [0.5, 1)
-    return ldexpf(1.f, f == 0.5f ? e - 1 : e);
+// The smallest power of two >= m, for a bound m >= 0 on the magnitudes a
+// tensor-core operand is divided by before it is rounded to fp16 (so the
+// operand's entries lie in [-1, 1], inside fp16's normal range down to 2^-14
+// of its largest entry). The exponent is kept in [-120, 126] so that the
+// scale and its reciprocal are normal floats; m = 0 (an all-zero operand) or
+// a non-finite m gives 1.
+__device__ __forceinline__ float pow2_ceil(float m) {
+    if (!(m > 0.f) || !(m <= 3.0e38f)) return 1.f;
+    const uint32_t b = __float_as_uint(m);
+    int e = (int)((b >> 23) & 0xffu) - 127 + ((b & 0x7fffffu) ? 1 : 0);
+    e = max(-120, min(126, e));
+    return __uint_as_float((uint32_t)(e + 127) << 23);
 }
 
 // Power of two 2^floor(e/2) with 2^e <= rr < 2^(e+1): a scale within a factor

@@ -10,9 +10,12 @@
 // fp32 registers and writes the state before every 128-token block of the
 // solve as a scaled fp16 image (format in tc_layout.cuh), plus the final state.
 //
-// Numerics: w_j a_j is split into an fp16 hi/lo pair, both multiplied by the
-// fp16 keys on the tensor cores with fp32 accumulation, so each chunk's sum
-// carries ~22-bit products into the fp32 running state.
+// Numerics: per chunk, w_j a_j / sA is split into an fp16 hi/lo pair and
+// multiplied by the fp16 keys k_j / sK on the tensor cores with fp32
+// accumulation, so each chunk's sum carries ~22-bit products into the fp32
+// running state. sA and sK are the powers of two at or above the chunk's
+// largest |w_j a_j| and |k_j| entries, so every operand lies in [-1, 1]
+// whatever the size of beta, k or v; the state takes sA sK times the sum.
 //
 // Pipeline per chunk c: MMA(c) runs while the CTA builds chunk c+1's operand
 // images (a second set) and warp 1 forms chunk c+2's gates (three gate
@@ -68,7 +71,8 @@ struct ScanSmem {
     static constexpr int oGate = oStage + 32768;  // b[3][64], w[3][64], amax[2][64], kmax[2][64]
     static constexpr int oGraw = oGate + 2560;    // 2 x {gamma[64], beta[64]} prefetched with the rows
     static constexpr int oRed = oGraw + 1024;     // 32 floats; [31] is the abort flag
-    static constexpr int oBar = oRed + 128;       // raw[2], mma
+    static constexpr int oCmax = oRed + 128;      // [2 buffers][16 warps] {max w|a|, max |k|} of a chunk
+    static constexpr int oBar = oCmax + 256;      // raw[2], mma
     static constexpr int oSlot = oBar + 32;
     static constexpr int bytes = oSlot + 16;
 };
@@ -103,6 +107,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     float* kmax = amax + 2 * kC;                                        // [2][64]
     float* graw = reinterpret_cast<float*>(smem + ScanSmem::oGraw);
     float* red = reinterpret_cast<float*>(smem + ScanSmem::oRed);
+    float2* cmax = reinterpret_cast<float2*>(smem + ScanSmem::oCmax);
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(smem + ScanSmem::oBar);
     uint64_t* bar_mma = bar_raw + 2;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + ScanSmem::oSlot);
@@ -154,54 +159,46 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         wv[lane] = (lane < nn) ? bsrc[lane] * expf(bl - b[lane]) : 0.f;
         wv[lane + 32] = (lane + 32 < nn) ? bsrc[lane + 32] * expf(bl - b[lane + 32]) : 0.f;
     };
-    // Operand images of chunk cc into set cc & 1: A = w_j a_j (hi/lo) [j][i],
-    // B = k_j [j][l], both MN-major SW128 in two 64-column blocks; row maxima
-    // of a and k into buffer cc & 1.
-    auto build = [&](int cc) {
+    // Operand images of chunk cc, in two phases around a CTA barrier.
+    // build_load: this thread's two 16-byte pieces of the rows of a (and of k
+    // for G) into registers, the row maxima of |a| and |k| into buffer cc & 1
+    // (for the state bound) and this warp's maxima of w_j |a_j| and |k_j| into
+    // cmax (for the chunk's operand scales).
+    // build_store: sA, sK from cmax, then A = w_j a_j / sA (hi/lo) [j][i] and
+    // B = k_j / sK [j][l] into set cc & 1, both MN-major SW128 in two
+    // 64-column blocks; returns sA sK, the factor the chunk's product carries.
+    uint4 ra[2], rk[2];
+    auto build_load = [&](int cc) {
         const int n = min(kC, T - cc * kC);
         const float* swc = sw + (cc % 3) * kC;
-        const uint8_t* ra = rawA + (cc & 1) * 16384;
-        const uint8_t* rk = rawK + (cc & 1) * 16384;
-        uint8_t* Ahi = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
-        uint8_t* Alo = Ahi + 16384;
-        uint8_t* Bk = Ahi + 32768;
+        const uint8_t* rpa = rawA + (cc & 1) * 16384;
+        const uint8_t* rpk = rawK + (cc & 1) * 16384;
         float* am = amax + (cc & 1) * kC;
         float* km = kmax + (cc & 1) * kC;
+        float wa = 0.f, wk = 0.f;
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
             const int cid = tid + kScanThreads * rep;      // 1024 16-byte chunks of the rows
             const int j = cid >> 4, cc16 = cid & 15;
-            uint4 raw = make_uint4(0, 0, 0, 0);
-            if (j < n) raw = *reinterpret_cast<const uint4*>(ra + j * 256 + cc16 * 16);
-            const float wj = swc[j];
-            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-            uint4 hi, lo;
-            uint32_t* hw = reinterpret_cast<uint32_t*>(&hi);
-            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+            ra[rep] = make_uint4(0, 0, 0, 0);
+            if (j < n) ra[rep] = *reinterpret_cast<const uint4*>(rpa + j * 256 + cc16 * 16);
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ra[rep]);
             float mx = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float2 f = __bfloat1622float2(a2[i]);
                 mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-                const float x0 = wj * f.x, x1 = wj * f.y;
-                const __half2 h2 = __floats2half2_rn(x0, x1);
-                const float2 hb = __half22float2(h2);
-                hw[i] = *reinterpret_cast<const uint32_t*>(&h2);
-                lw[i] = pack_half2(x0 - hb.x, x1 - hb.y);
             }
-            const uint32_t off = (uint32_t)((cc16 >> 3) * 8192 + j * 128 + (((cc16 & 7) ^ (j & 7)) << 4));
-            *reinterpret_cast<uint4*>(Ahi + off) = hi;
-            *reinterpret_cast<uint4*>(Alo + off) = lo;
             // row max over the 16 threads (same half-warp) that hold row j
 #pragma unroll
             for (int o2 = 8; o2 >= 1; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
             if (cc16 == 0) am[j] = mx;
-            uint4 kr = raw;
+            float kmx = mx;
             if (m) {   // key rows: the B operand and the key row maxima for the value-state bound
-                kr = make_uint4(0, 0, 0, 0);
-                if (j < n) kr = *reinterpret_cast<const uint4*>(rk + j * 256 + cc16 * 16);
-                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-                float kmx = 0.f;
+                rk[rep] = make_uint4(0, 0, 0, 0);
+                if (j < n) rk[rep] = *reinterpret_cast<const uint4*>(rpk + j * 256 + cc16 * 16);
+                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&rk[rep]);
+                kmx = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float2 f = __bfloat1622float2(k2[i]);
@@ -211,13 +208,56 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
                 for (int o2 = 8; o2 >= 1; o2 >>= 1) kmx = fmaxf(kmx, __shfl_xor_sync(0xffffffffu, kmx, o2));
                 if (cc16 == 0) km[j] = kmx;
             }
-            *reinterpret_cast<uint4*>(Bk + off) = bf16x8_to_f16x8(kr, 1.f);
+            wa = fmaxf(wa, swc[j] * mx);
+            wk = fmaxf(wk, kmx);
         }
+        wa = fmaxf(wa, __shfl_xor_sync(0xffffffffu, wa, 16));   // the warp's other row
+        wk = fmaxf(wk, __shfl_xor_sync(0xffffffffu, wk, 16));
+        if (lane == 0) cmax[(cc & 1) * 16 + w] = make_float2(wa, wk);
+    };
+    auto build_store = [&](int cc) -> float {
+        const float* swc = sw + (cc % 3) * kC;
+        uint8_t* Ahi = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
+        uint8_t* Alo = Ahi + 16384;
+        uint8_t* Bk = Ahi + 32768;
+        float wa = 0.f, wk = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float2 c2 = cmax[(cc & 1) * 16 + i];
+            wa = fmaxf(wa, c2.x);
+            wk = fmaxf(wk, c2.y);
+        }
+        const float sA = pow2_ceil(wa), sK = pow2_ceil(wk);
+        const float inv_sA = 1.f / sA, inv_sK = 1.f / sK;       // powers of two: exact
+#pragma unroll
+        for (int rep = 0; rep < 2; ++rep) {
+            const int cid = tid + kScanThreads * rep;
+            const int j = cid >> 4, cc16 = cid & 15;
+            const float wj = swc[j] * inv_sA;
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ra[rep]);
+            uint4 hi, lo;
+            uint32_t* hw = reinterpret_cast<uint32_t*>(&hi);
+            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(a2[i]);
+                const float x0 = wj * f.x, x1 = wj * f.y;
+                const __half2 h2 = __floats2half2_rn(x0, x1);
+                const float2 hb = __half22float2(h2);
+                hw[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                lw[i] = pack_half2(x0 - hb.x, x1 - hb.y);
+            }
+            const uint32_t off = (uint32_t)((cc16 >> 3) * 8192 + j * 128 + (((cc16 & 7) ^ (j & 7)) << 4));
+            *reinterpret_cast<uint4*>(Ahi + off) = hi;
+            *reinterpret_cast<uint4*>(Alo + off) = lo;
+            *reinterpret_cast<uint4*>(Bk + off) = bf16x8_to_f16x8(m ? rk[rep] : ra[rep], inv_sK);
+        }
+        return sA * sK;
     };
     // The state / s as fp16 into the staging image (the solve's layout);
     // returns the power-of-two scale s from the entry bound.
     auto stage_state = [&](const float (&St)[32], float bnd) {
-        const float s = pow2_ceil_at_least_one(bnd);
+        const float s = pow2_ceil(bnd);
         const float inv = 1.f / s;
         uint8_t* dst = stage + (col0 >> 6) * 16384 + row * 128;
         const int g0 = (col0 & 63) >> 3;
@@ -293,10 +333,13 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         mma_commit(bar_mma);
     };
     int mma_issued = 0, mma_seen = 0;             // thread 0
+    float ds_cur = 1.f, ds_next = 1.f;            // sA sK of the chunk in the MMA, of the next chunk
     if (ok && nc > 0) {
         // the state before chunk 0 (block 0's image) and chunk 0's operands
+        build_load(0);
+        __syncthreads();                          // chunk 0's maxima
+        ds_cur = build_store(0);
         const float s0 = stage_state(S, bound);
-        build(0);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -313,8 +356,8 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     }
     int c = 0;
     for (; ok && c < nc; ++c) {
-        // ---- while MMA(c) runs: chunk c+1's operands, chunk c+2's gates, the bound after chunk c ----
-        if (c + 1 < nc) build(c + 1);
+        // ---- while MMA(c) runs: chunk c+1's rows and maxima, chunk c+2's gates, the bound after chunk c ----
+        if (c + 1 < nc) build_load(c + 1);
         if (w == 1 && c + 2 < nc) chunk_gates(c + 2);
         const float blast = sb[(c % 3) * kC + kC - 1];
         {
@@ -334,19 +377,20 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             else red[31] = 1.f;
             if (emit) bulk_wait_read_all();       // the staging buffer is free again
         }
-        __syncthreads();                          // MMA(c) done; operands of c+1 and gates of c+2 written
+        __syncthreads();                          // MMA(c) done; maxima of c+1 and gates of c+2 written
         tc_fence_after();
         if (red[31] != 0.f) {
             ok = false;
             break;
         }
-        // ---- S <- e^{b_last} S + Delta ----
+        // ---- chunk c+1's operand images; S <- e^{b_last} S + sA sK Delta ----
         const float Gam = expf(blast);
         float dv[32];
         tmem_ld32_x32(tbase + ((uint32_t)(32 * q4) << 16) + col0, dv);
+        if (c + 1 < nc) ds_next = build_store(c + 1);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] = fmaf(Gam, S[i], dv[i]);
+        for (int i = 0; i < 32; ++i) S[i] = fmaf(Gam, S[i], ds_cur * dv[i]);
         if (c + 1 == nc) {                        // the final state
             if (fin) {
                 float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
@@ -372,6 +416,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             ++mma_issued;
             if (c + 3 < nc) prefetch(c + 3);      // raw buffer (c+1) & 1 is consumed
         }
+        ds_cur = ds_next;
     }
     if (nc == 0 && fin) {                         // no tokens: the final state is the initial one
         float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);

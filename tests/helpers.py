@@ -45,3 +45,17 @@ def count_agreement(iters, iters_ref) -> tuple[int, float]:
     if diff.size == 0:
         return 0, 0.0
     return int(diff.max()), float((diff > 0).mean())
+
+
+def log_parity(case: str, o, ref, **extra) -> dict:
+    """err_report of one parity comparison; when MESA_PARITY_LOG names a file,
+    the report is also appended to it as one JSON line (with the case name),
+    so a run keeps both error floors of every case it checked."""
+    import json
+    import os
+    rep = dict(case=case, **err_report(o, ref), **extra)
+    path = os.environ.get("MESA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rep) + "\n")
+    return rep

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import mesa_inputs as mi
-from helpers import TOL_BF16, TOL_F32, count_agreement, err_report, rel_err
+from helpers import TOL_BF16, TOL_F32, count_agreement, err_report, log_parity, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -71,7 +71,8 @@ def test_bf16_d128_chunk64(mesa, oracle_mod, T):
     x = mi.batch(w)
     ref, _, _, _ = oracle_mod.forward_cg(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], w.cg_steps)
     out, it = run(mesa, to_dev(x, "bf16"), 64, w.cg_steps, 0.0)
-    assert rel_err(out, ref) <= TOL_BF16, err_report(out, ref)
+    rep = log_parity(f"bf16_d128_T{T}", out, ref)
+    assert rep["rel"] <= TOL_BF16, rep
     assert np.all(it == 15)
 
 
@@ -224,7 +225,8 @@ def test_full_size_sampled(mesa, oracle_mod, name):
                                               host["lam"], w.cg_steps, w.tol)
     got = np.stack([out[b, h].cpu().numpy() for b, h in pairs])[None]
     got_it = np.stack([it[b, h].cpu().numpy() for b, h in pairs])[None]
-    assert rel_err(got, ref) <= TOL_BF16, err_report(got, ref)
+    rep = log_parity(f"full:{name}", got, ref)
+    assert rep["rel"] <= TOL_BF16, rep
     if w.tol > 0:
         mx, frac = count_agreement(got_it, it_ref)
         assert mx <= 1 and frac <= 0.01, (mx, frac)
