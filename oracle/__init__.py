@@ -49,6 +49,7 @@ def _configure(lib):
     I32 = ctypes.POINTER(ctypes.c_int32)
     i, d = ctypes.c_int, ctypes.c_double
     lib.oracle_forward_cg.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, I32, D, D]
+    lib.oracle_forward_cg_x0.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, D, I32, D, D, D]
     lib.oracle_forward_cholesky.argtypes = [D, D, D, D, D, D, i, i, i, i, i, D, D, D, D, D]
     lib.oracle_forward_chunked.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, i, d, D, D, D, I32, D, D]
     lib.oracle_step.argtypes = [D, D, D, D, D, D, i, i, i, i, D, D, i, d, D, I32]
@@ -56,7 +57,7 @@ def _configure(lib):
     lib.oracle_cg_dense.argtypes = [i, D, D, D, i, d, D, I32]
     lib.oracle_preprocess.argtypes = [D, D, i, i, i, i, i, D]
     lib.oracle_backward.argtypes = [D, D, D, D, D, D, i, i, i, i, i, i, d, D, D, D, D, D, D, D, I32, I32]
-    for f in (lib.oracle_forward_cg, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
+    for f in (lib.oracle_forward_cg, lib.oracle_forward_cg_x0, lib.oracle_forward_cholesky, lib.oracle_forward_chunked,
               lib.oracle_step, lib.oracle_step_warm, lib.oracle_cg_dense, lib.oracle_preprocess,
               lib.oracle_backward):
         f.restype = ctypes.c_int
@@ -112,6 +113,24 @@ def forward_cg(q, k, v, gamma, beta, lam, cg_steps, tol=0.0, H0=None, G0=None):
                                    _ptr(out), _ptr(iters), _ptr(Hf), _ptr(Gf))
     _check(rc, "oracle_forward_cg")
     return out, iters, Hf, Gf
+
+
+def forward_cg_x0(q, k, v, gamma, beta, lam, cg_steps, tol=0.0, x0=None, H0=None, G0=None):
+    """Per-token recurrence + CG started from x0 [B,H,T,dk] (None: zero).
+    Returns (out, iters, x, H_final, G_final)."""
+    q, k, v, gamma, beta, lam = map(_f64, (q, k, v, gamma, beta, lam))
+    x0, H0, G0 = _f64(x0), _f64(H0), _f64(G0)
+    B, H, T, dk, dv = _shapes(q, v)
+    out = np.zeros((B, H, T, dv))
+    iters = np.zeros((B, H, T), dtype=np.int32)
+    x = np.zeros((B, H, T, dk))
+    Hf = np.zeros((B, H, dk, dk))
+    Gf = np.zeros((B, H, dv, dk))
+    rc = _load().oracle_forward_cg_x0(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                      B, H, T, dk, dv, int(cg_steps), float(tol), _ptr(x0), _ptr(H0), _ptr(G0),
+                                      _ptr(out), _ptr(iters), _ptr(x), _ptr(Hf), _ptr(Gf))
+    _check(rc, "oracle_forward_cg_x0")
+    return out, iters, x, Hf, Gf
 
 
 def forward_cholesky(q, k, v, gamma, beta, lam, H0=None, G0=None):

@@ -204,6 +204,58 @@ int oracle_forward_cg(const double* q, const double* k, const double* v,
     return err ? -2 : 0;
 }
 
+/* The per-token forward with a warm-started CG (MesaNet page, Significance
+ * and claims: warm starts named as the way to cut the solver's cost): token
+ * t's CG starts from x0[b,h,t,:] (NULL: from zero, which is exactly
+ * oracle_forward_cg), r_0 = q_t - (H_t + Lambda) x0_t, p_0 = r_0, and the
+ * stopping test stays |r_k| <= tol |q_t|. x_out [B,H,T,dk] (or NULL)
+ * receives every token's solution. */
+int oracle_forward_cg_x0(const double* q, const double* k, const double* v,
+                         const double* gamma, const double* beta, const double* lambda,
+                         int B, int H, int T, int dk, int dv, int cg_steps, double tol,
+                         const double* x0, const double* H_init, const double* G_init,
+                         double* out, int32_t* iters, double* x_out, double* H_final, double* G_final) {
+    if (bad_dims(B, H, T, dk, dv) || cg_steps < 0) return -1;
+    if (T > 0 && (!q || !k || !v || !gamma || !beta || !out)) return -1;
+    if (!lambda) return -1;
+    const int BH = B * H;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int bh = 0; bh < BH; ++bh) {
+        const int h = bh % H;
+        double* Hm = (double*)malloc(sizeof(double) * (size_t)dk * dk);
+        double* Gm = (double*)malloc(sizeof(double) * (size_t)dv * dk);
+        double* A = (double*)malloc(sizeof(double) * (size_t)dk * dk);
+        double* x = (double*)malloc(sizeof(double) * (size_t)dk);
+        double* work = (double*)malloc(sizeof(double) * 3 * (size_t)dk);
+        if (!Hm || !Gm || !A || !x || !work) {
+            err |= 1;
+        } else {
+            init_state((size_t)dk * dk, H_init ? H_init + (size_t)bh * dk * dk : NULL, Hm);
+            init_state((size_t)dv * dk, G_init ? G_init + (size_t)bh * dv * dk : NULL, Gm);
+            for (int t = 0; t < T; ++t) {
+                const size_t bt = (size_t)bh * T + t;
+                update_state(dk, dv, gamma[bt], beta[bt], k + bt * dk, v + bt * dv, Hm, Gm);
+                for (int i = 0; i < dk; ++i) {
+                    for (int j = 0; j < dk; ++j) A[(size_t)i * dk + j] = Hm[(size_t)i * dk + j];
+                    A[(size_t)i * dk + i] += lambda[(size_t)h * dk + i];
+                }
+                dense_ctx c = {dk, A};
+                const int it = cg_generic_x0(dk, dense_mv, &c, q + bt * dk, x0 ? x0 + bt * dk : NULL, cg_steps, tol,
+                                             x, work);
+                if (iters) iters[bt] = it;
+                if (x_out) memcpy(x_out + bt * dk, x, sizeof(double) * (size_t)dk);
+                double* ot = out + bt * dv;
+                for (int i = 0; i < dv; ++i) ot[i] = dot(dk, Gm + (size_t)i * dk, x);
+            }
+            if (H_final) memcpy(H_final + (size_t)bh * dk * dk, Hm, sizeof(double) * (size_t)dk * dk);
+            if (G_final) memcpy(G_final + (size_t)bh * dv * dk, Gm, sizeof(double) * (size_t)dv * dk);
+        }
+        free(Hm); free(Gm); free(A); free(x); free(work);
+    }
+    return err ? -2 : 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Per-token recurrence + exact Cholesky solve                                */
 /* ------------------------------------------------------------------------ */

@@ -33,6 +33,14 @@ int oracle_forward_cg(const double* q, const double* k, const double* v,
                       const double* H_init, const double* G_init,
                       double* out, int32_t* iters, double* H_final, double* G_final);
 
+/* oracle_forward_cg with every token's CG started from x0 [B,H,T,dk] (NULL:
+ * zero); x_out [B,H,T,dk] or NULL receives the solutions. */
+int oracle_forward_cg_x0(const double* q, const double* k, const double* v,
+                         const double* gamma, const double* beta, const double* lambda,
+                         int B, int H, int T, int dk, int dv, int cg_steps, double tol,
+                         const double* x0, const double* H_init, const double* G_init,
+                         double* out, int32_t* iters, double* x_out, double* H_final, double* G_final);
+
 /* Per-token recurrence with an exact Cholesky solve of (H_t + Lambda) x = q. */
 int oracle_forward_cholesky(const double* q, const double* k, const double* v,
                             const double* gamma, const double* beta, const double* lambda,

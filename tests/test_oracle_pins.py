@@ -446,6 +446,71 @@ def test_warm_step_from_zero_is_the_cold_step(oracle_mod):
     assert np.allclose(np.einsum("bhij,bhj->bhi", warm[3], warm[4]), warm[0], atol=1e-12)
 
 
+# Warm-started forward (the same reading applied to every token of a
+# sequence): token t's CG starts from a caller-given x0_t.
+
+def _explicit_systems(q, k, v, gamma, beta, lam):
+    """(A_t, G_t) for every token from the gated recurrences written out in numpy."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    A = np.zeros((B, H, T, dk, dk))
+    G = np.zeros((B, H, T, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            Hm = np.zeros((dk, dk))
+            Gm = np.zeros((dv, dk))
+            for t in range(T):
+                Hm = gamma[b, h, t] * Hm + beta[b, h, t] * np.outer(k[b, h, t], k[b, h, t])
+                Gm = gamma[b, h, t] * Gm + beta[b, h, t] * np.outer(v[b, h, t], k[b, h, t])
+                A[b, h, t] = Hm + np.diag(lam[h])
+                G[b, h, t] = Gm
+    return A, G
+
+
+def test_warm_forward_from_zero_is_the_cold_forward(oracle_mod):
+    rng = np.random.default_rng(31)
+    q, k, v, gamma, beta, lam = rand_inputs(rng, 2, 2, 9, 5, 4)
+    cold, it_c, Hc, Gc = oracle_mod.forward_cg(q, k, v, gamma, beta, lam, 3, 1e-2)
+    for x0 in (None, np.zeros((2, 2, 9, 5))):
+        warm, it_w, x, Hw, Gw = oracle_mod.forward_cg_x0(q, k, v, gamma, beta, lam, 3, 1e-2, x0=x0)
+        assert np.array_equal(warm, cold) and np.array_equal(it_w, it_c)
+        assert np.array_equal(Hw, Hc) and np.array_equal(Gw, Gc)
+        # the returned solutions reproduce the outputs through G_t
+        _, G = _explicit_systems(q, k, v, gamma, beta, lam)
+        assert np.allclose(np.einsum("bhtij,bhtj->bhti", G, x), warm, rtol=0, atol=1e-12)
+
+
+def test_warm_forward_is_the_shifted_cold_solve_per_token(oracle_mod):
+    """With a fixed step count, CG from x0_t on A_t x = q_t equals x0_t plus
+    CG from zero on A_t e = q_t - A_t x0_t, token by token (dk != dv)."""
+    rng = np.random.default_rng(32)
+    q, k, v, gamma, beta, lam = rand_inputs(rng, 1, 2, 7, 6, 3)
+    x0 = rng.standard_normal((1, 2, 7, 6))
+    A, G = _explicit_systems(q, k, v, gamma, beta, lam)
+    for N in (1, 2, 4):
+        out, it, x, _, _ = oracle_mod.forward_cg_x0(q, k, v, gamma, beta, lam, N, 0.0, x0=x0)
+        assert np.all(it == N)
+        for h in range(2):
+            for t in range(7):
+                At = A[0, h, t]
+                e, _ = oracle_mod.cg_dense(At, q[0, h, t] - At @ x0[0, h, t], N, 0.0)
+                assert np.allclose(x[0, h, t], x0[0, h, t] + e, rtol=0, atol=1e-10), (N, h, t)
+                assert np.allclose(out[0, h, t], G[0, h, t] @ x[0, h, t], rtol=0, atol=1e-10)
+
+
+def test_warm_forward_from_the_exact_solutions(oracle_mod):
+    """x0_t = A_t^-1 q_t: no token takes a step under a tolerance, and the
+    outputs equal the exact (Cholesky) layer."""
+    rng = np.random.default_rng(33)
+    q, k, v, gamma, beta, lam = rand_inputs(rng, 2, 1, 8, 5, 5)
+    A, _ = _explicit_systems(q, k, v, gamma, beta, lam)
+    xs = np.linalg.solve(A, q[..., None])[..., 0]
+    out, it, x, _, _ = oracle_mod.forward_cg_x0(q, k, v, gamma, beta, lam, 10, 1e-8, x0=xs)
+    assert np.all(it == 0) and np.array_equal(x, xs)
+    exact, _, _ = oracle_mod.forward_cholesky(q, k, v, gamma, beta, lam)
+    assert np.allclose(out, exact, rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # Backward pass (implicit differentiation with an adjoint CG solve)
 # --------------------------------------------------------------------------
