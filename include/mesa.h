@@ -143,6 +143,9 @@ mesa_status mesa_forward(const void* q, const void* k, const void* v,
  *     any device work.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is cached per device for the device's primary context
+ *     (the CUDA runtime's): calls from another driver context, or after
+ *     cudaDeviceReset, are not supported.
  *   - All calls on a device share the array, which keeps the previous call's
  *     contents; every byte is written before it is read, so no clearing is
  *     needed. Calls that overlap on the GPU (different streams, or host

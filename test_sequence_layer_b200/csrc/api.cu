@@ -461,7 +461,10 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
                       H_out ? dHo + s0 * hs : nullptr, G_out ? dGo + s0 * gs : nullptr,
                       fws[i % ncomp], fws_slice};
         s = launch_forward(a, cs);
-        if (s != MESA_OK) return s;
+        if (s != MESA_OK) {
+            ok = false;
+            break;
+        }
         ok = cudaEventRecord(hp->done[i], cs) == cudaSuccess;
     }
     for (int i = 0; ok && i < nslices; ++i) {
@@ -477,7 +480,16 @@ mesa_status mesa_forward_host(const void* q, const void* k, const void* v,
     }
     // the caller's stream resumes after the last copy; the call returns once it has landed
     ok = ok && cudaEventRecord(hp->end, hp->out) == cudaSuccess && cudaStreamWaitEvent(st, hp->end, 0) == cudaSuccess;
+    if (!ok) {
+        // a failure after the first copy was queued: the caller's stream still
+        // waits for whatever the pipeline streams hold (copies reading the
+        // caller's host buffers, kernels on the workspace), so that an error
+        // return keeps the ordering guarantee of a successful call
+        for (cudaStream_t sm : {hp->in, hp->comp[0], hp->comp[1], hp->out})
+            if (cudaEventRecord(hp->end, sm) == cudaSuccess) cudaStreamWaitEvent(st, hp->end, 0);
+    }
     const bool synced = cudaStreamSynchronize(st) == cudaSuccess;
+    if (s != MESA_OK) return s;
     return ok && synced ? MESA_OK : MESA_ERR_CUDA;
 }
 

@@ -14,6 +14,8 @@
 // forward writes every byte it later reads (chunk-start states and their
 // scales), so nothing needs clearing between calls; calls that overlap on the
 // GPU (other streams, or host threads, without ordering) race on it.
+#include <atomic>
+
 #include "mesa_common.cuh"
 #include "mesa_internal.h"
 
@@ -24,20 +26,23 @@ constexpr size_t kScratchBytes = MESA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDev = 64;
-void* g_scratch_addr[kMaxDev] = {nullptr};
+std::atomic<void*> g_scratch_addr[kMaxDev];
 
 // Device address of the scratch array on the current device. Looked up once
-// per device (the host-side name of the array is only a stand-in, never a
-// device address). Returns nullptr if the lookup fails.
+// per device, in the device's primary context (the runtime API's context; the
+// host-side name of the array is only a stand-in, never a device address).
+// Host threads that race on the first call each store the same address, so
+// the cached value is written atomically and read without a lock. Returns
+// nullptr if the lookup fails.
 void* scratch_address() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_release);
     }
-    return g_scratch_addr[dev];
+    return p;
 }
 
 }  // namespace

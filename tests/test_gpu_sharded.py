@@ -103,3 +103,11 @@ def test_sharded_forward_with_tolerance_stopping(mesa, oracle_mod):
     assert rel_err(got, ref) <= 2e-2, err_report(got, ref)
     diff = np.abs(torch.cat(its, dim=2).cpu().numpy().astype(np.int64) - it_ref)
     assert diff.max() <= 1
+    # each o_t depends only on token t's own solve: where the counts agree,
+    # the fp32 path must meet the fp32 bound (a prefix state off by one gamma
+    # factor would move these tokens by ~1 %)
+    same = (diff == 0)
+    assert same.mean() > 0.9
+    d_tok = np.abs(got - ref).max(-1)
+    den = np.maximum(np.abs(ref).max(-1), np.sqrt(np.mean(ref ** 2)))
+    assert (d_tok / den)[same].max() <= TOL_F32

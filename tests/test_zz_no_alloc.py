@@ -2,9 +2,12 @@
 memory (it takes its scratch from a fixed library-owned device array instead
 of a caller workspace). Called through the C ABI and checked against
 mesa_forward on the same inputs, on two calls in a row (the second call finds
-the previous call's data in the shared array).
+the previous call's data in the shared array), and on a smaller shape after a
+larger one (stale bytes beyond the smaller call's layout must go unread).
 
-This file is collected last on purpose."""
+The file name sorts after every other test file, so pytest collects it last:
+a run that stops at the first failure has then already run every other test
+before this one. The tests pass alone in a fresh process as well."""
 import ctypes
 
 import numpy as np
@@ -80,3 +83,29 @@ def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
     rc = lib.mesa_forward_noalloc(ptr(dummy), ptr(dummy), ptr(dummy), ptr(dummy), ptr(dummy), ptr(dummy), B, H, T,
                                   128, 128, 64, 1, 15, 0.0, ptr(dummy), None, None, None, None, None, stream)
     assert rc == 3    # MESA_ERR_WORKSPACE, refused before any device work
+
+
+@pytest.mark.parametrize("dtype,d,chunk", [("bf16", 128, 64), ("f32", 32, 16)])
+def test_noalloc_smaller_call_after_larger(lib, dtype, d, chunk):
+    """A large call fills more of the shared array than the small call that
+    follows it; the small call must match mesa_forward all the same."""
+    from test_sequence_layer_b200 import mesa
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    for B, H, T, seed in ((4, 4, 700, 51), (1, 2, 130, 52)):
+        w = mi.Workload("na", B, H, T, d, d, chunk, dtype, 15, 0.0, False, seed)
+        x = mi.batch(w)
+        dev = {n: torch.from_numpy(np.ascontiguousarray(x[n])).cuda() for n in ("q", "k", "v", "gamma", "beta", "lam")}
+        for n in ("q", "k", "v"):
+            dev[n] = dev[n].to(dt)
+        ref, ref_it, rH, rG = mesa.forward(dev["q"], dev["k"], dev["v"], dev["gamma"], dev["beta"], dev["lam"],
+                                           chunk=chunk, cg_steps=15, return_iters=True, return_state=True)
+        out = torch.full_like(ref, float("nan"))
+        iters = torch.full_like(ref_it, -1)
+        Ho, Go = torch.empty_like(rH), torch.empty_like(rG)
+        assert call_noalloc(lib, dev, w, out, iters, Ho, Go) == 0
+        torch.cuda.synchronize()
+        assert mesa.get_error() == 0
+        assert rel_err(out.cpu().numpy(), ref.cpu().numpy()) <= tol, (B, H, T)
+        assert torch.equal(iters, ref_it)
+        assert torch.allclose(Ho, rH, rtol=1e-5, atol=1e-6) and torch.allclose(Go, rG, rtol=1e-5, atol=1e-6)
