@@ -566,6 +566,111 @@ def run_seq_sharded(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_forward_warm(args, w, world, rank, local):
+    """Forward warm start on a forward workload: the sequences are solved
+    once, then one token is inserted at the front of each (the last drops out,
+    T is unchanged: a context edited since it was solved), and the edited
+    batch is solved again, cold (mesa_forward) and from the shifted earlier
+    solutions (mesa_forward_warm). Both are timed over the same steps; the
+    line's value is the warm re-solve's rate, with the cold one beside it."""
+    import torch
+    import torch.distributed as dist
+    from test_sequence_layer_b200 import build as mbuild, mesa
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    tol = w.tol if args.tol is None else args.tol
+    x = mi.device_batch(w, dev, seed_offset=rank)
+    B, H, T, d, C = w.B, w.H, w.T, w.dk, w.chunk
+    tokens = B * H * T
+    stream = torch.cuda.current_stream(dev)
+    ws = torch.empty(max(mesa.workspace_size(B, H, T, d, d, C, x["q"].dtype), 1), dtype=torch.uint8, device=dev)
+    _, x_old = mesa.forward_warm(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["lam"], None, chunk=C,
+                                 cg_steps=w.cg_steps, tol=tol, workspace=ws, stream=stream)
+    g = torch.Generator(device=dev)
+    g.manual_seed(777 + rank)
+    y = {}
+    for n in ("q", "k", "v", "gamma", "beta"):
+        y[n] = torch.roll(x[n], 1, dims=2).contiguous()
+    for n in ("q", "k"):
+        e = torch.randn((B, H, d), generator=g, device=dev)
+        y[n][:, :, 0] = (e / e.norm(dim=-1, keepdim=True)).to(y[n].dtype)
+    y["v"][:, :, 0] = torch.randn((B, H, d), generator=g, device=dev).to(y["v"].dtype)
+    y["gamma"][:, :, 0] = 0.9
+    y["beta"][:, :, 0] = 0.5
+    x0 = torch.roll(x_old, 1, dims=2).contiguous()
+    x0[:, :, 0] = 0.0
+    del x_old, x
+    out = torch.empty((B, H, T, d), device=dev)
+    xs = torch.empty((B, H, T, d), device=dev)
+    it_c = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+    it_w = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+
+    def cold():
+        mesa.forward(y["q"], y["k"], y["v"], y["gamma"], y["beta"], x_lam, chunk=C, cg_steps=w.cg_steps, tol=tol,
+                     out=out, iters=it_c, return_iters=True, workspace=ws, stream=stream)
+
+    def warm():
+        mesa.forward_warm(y["q"], y["k"], y["v"], y["gamma"], y["beta"], x_lam, x0, chunk=C, cg_steps=w.cg_steps,
+                          tol=tol, out=out, x_out=xs, iters=it_w, return_iters=True, workspace=ws, stream=stream)
+
+    x_lam = torch.from_numpy(mi.lambdas(w.seed, w.H, w.dk)).to(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ms_cold = timed(cold)
+    kernels_cold = mesa.timing_read()
+    ms_warm = timed(warm)
+    kernels = mesa.timing_read()
+    mesa.timing_enable(False)
+    clk = clocks.stop()
+    assert mesa.get_error(stream) == 0
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "Mesa-layer fwd tokens/s (B*H*T), re-solve of an edited context (one token inserted at the "
+                  "front) warm-started from the earlier solutions",
+        "value": whole_job_rate(tokens, world, ms_warm), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_warm, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-in/f16-mma/f32-acc" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name + "+edit-warm-start", "B": B, "H": H, "T": T, "d": d, "chunk": C,
+                   "cg_steps": w.cg_steps, "tol": tol, "l2": "inputs larger than L2"},
+        "warm": {"ms_per_step": ms_warm, "mean_iters": float(it_w.double().mean().item()),
+                 "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()}},
+        "cold": {"ms_per_step": ms_cold, "mean_iters": float(it_c.double().mean().item()),
+                 "value": whole_job_rate(tokens, world, ms_cold),
+                 "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels_cold.items()}},
+        "roofline": None, "gpu_launches": sum(v[0] for v in kernels.values()),
+        "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -582,7 +687,9 @@ def main():
     ap.add_argument("--seq-sharded", action="store_true",
                     help="sequence-sharded forward: each rank one slice of T, one all-gather of slice states")
     ap.add_argument("--warm-start", action="store_true",
-                    help="decode: start each step's CG from the previous step's solution (mesa_step_warm)")
+                    help="decode: start each step's CG from the previous step's solution (mesa_step_warm); "
+                         "forward workloads: re-solve an edited context from its earlier solutions "
+                         "(mesa_forward_warm) against a cold re-solve")
     ap.add_argument("--tol", type=float, default=None, help="override the workload's CG tolerance")
     ap.add_argument("--query-walk", type=float, default=0.0,
                     help="decode: queries as a random walk on the sphere with this step size (correlated stream)")
@@ -611,6 +718,9 @@ def main():
         return
     if w.decode_steps > 0:
         run_decode(args, w, world, rank, local)
+        return
+    if args.warm_start:
+        run_forward_warm(args, w, world, rank, local)
         return
 
     import torch

@@ -121,6 +121,36 @@ mesa_status mesa_forward(const void* q, const void* k, const void* v,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * mesa_forward with a warm-started CG: token t's solve starts from a caller-
+ * given guess x0_t instead of zero. Source: the MesaNet page, Significance
+ * and claims (warm starts are named as the way to cut the solver's cost; the
+ * pages give no rule). Reading taken: x_0 = x0_t, r_0 = q_t - (H_t + Lambda)
+ * x0_t, p_0 = r_0, and the stopping test stays |r_k| <= tol |q_t|, so a
+ * guess within the tolerance takes no step; iters counts the updates after
+ * the start. In the one-pass forward every token of a block is solved at
+ * once, so no token's neighbour has a solution to offer; the guesses come
+ * from the caller, e.g. the solutions of an earlier forward over a context
+ * that has since been edited or extended (x_out below).
+ *
+ *   x0       float32 [B,H,T,dk], 16-byte aligned, or NULL (start from zero:
+ *            then the call equals mesa_forward).
+ *   x_out    float32 [B,H,T,dk], 16-byte aligned, or NULL: every token's
+ *            solution x_t. May be the same buffer as x0 (updated in place);
+ *            otherwise neither may overlap the other or `out`.
+ * Every other argument, and the cost of a cold call, as for mesa_forward; a
+ * warm start adds one matrix-vector product per token (one more CG-step's
+ * worth of work) and the read of x0.
+ */
+mesa_status mesa_forward_warm(const void* q, const void* k, const void* v,
+                              const float* gamma, const float* beta, const float* lambda,
+                              int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                              int cg_steps, float tol, const float* x0, float* x_out,
+                              float* out, int32_t* iters_out,
+                              const float* H_in, const float* G_in,
+                              float* H_out, float* G_out,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Size of the fixed device scratch array behind mesa_forward_noalloc.
  */
 #define MESA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -224,6 +224,55 @@ mesa_status mesa_forward(const void* q, const void* k, const void* v,
     return launch_forward(a, static_cast<cudaStream_t>(stream));
 }
 
+mesa_status mesa_forward_warm(const void* q, const void* k, const void* v,
+                              const float* gamma, const float* beta, const float* lambda,
+                              int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                              int cg_steps, float tol, const float* x0, float* x_out,
+                              float* out, int32_t* iters_out,
+                              const float* H_in, const float* G_in,
+                              float* H_out, float* G_out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    if (T > 0) {
+        if ((x0 && !aligned(x0, 16)) || (x_out && !aligned(x_out, 16))) return MESA_ERR_INVALID_ARG;
+        // x0 and x_out are read and written row by row by the same block of
+        // threads, so they may be the same buffer; they must not overlap anything else
+        const size_t xb = (size_t)B * H * T * dk * sizeof(float);
+        const char* ob = reinterpret_cast<const char*>(out);
+        const size_t outb = (size_t)B * H * T * dv * sizeof(float);
+        for (const void* xp : {(const void*)x0, (const void*)x_out}) {
+            const char* c = static_cast<const char*>(xp);
+            if (c && ob && c < ob + outb && ob < c + xb) return MESA_ERR_INVALID_ARG;
+        }
+        if (x0 && x_out && x0 != x_out) {
+            const char* a = reinterpret_cast<const char*>(x0);
+            const char* b = reinterpret_cast<const char*>(x_out);
+            if (a < b + xb && b < a + xb) return MESA_ERR_INVALID_ARG;
+        }
+    }
+    mesa_status s = check_shape(B, H, T, dk, dv, chunk, dtype, cg_steps, tol);
+    if (s != MESA_OK) return s;
+    if (!lambda || !aligned(lambda, 4)) return MESA_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!q || !k || !v || !gamma || !beta || !out) return MESA_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return MESA_ERR_INVALID_ARG;
+        if (!aligned(gamma, 4) || !aligned(beta, 4)) return MESA_ERR_INVALID_ARG;
+        if (iters_out && !aligned(iters_out, 4)) return MESA_ERR_INVALID_ARG;
+    }
+    for (const void* p : {(const void*)H_in, (const void*)G_in, (const void*)H_out, (const void*)G_out})
+        if (p && !aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    if ((H_out && H_out == H_in) || (G_out && G_out == G_in)) return MESA_ERR_INVALID_ARG;
+    const size_t need = workspace_bytes(B, H, T, dk, dv, chunk, dtype);
+    if (T > 0 && need > 0) {
+        if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
+    }
+    ForwardArgs a{q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps, tol,
+                  out, iters_out, H_in, G_in, H_out, G_out, workspace, ws_bytes};
+    a.x0 = T > 0 ? x0 : nullptr;
+    a.x_out = T > 0 ? x_out : nullptr;
+    return launch_forward(a, static_cast<cudaStream_t>(stream));
+}
+
 size_t mesa_backward_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
     if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
     return backward_workspace_bytes(B, H, T, dk, dv, chunk, dtype);

@@ -30,6 +30,7 @@ struct ForwardArgs {
     void* workspace;
     size_t ws_bytes;
     float* x_out = nullptr;     // the CG solutions x_t [B,H,T,dk] (fp32), when not null
+    const float* x0 = nullptr;  // per-token CG starting guesses [B,H,T,dk] (fp32), when not null
     bool scan_only = false;     // fp32 CUDA-core path only: the chunk-state scan, no solve
 };
 

@@ -111,7 +111,7 @@ simt_cg_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* 
                const float* __restrict__ gamma, const float* __restrict__ beta,
                const float* __restrict__ lambda, int H, int T, int nc, int cg_steps, float tol,
                const float* __restrict__ states, float* __restrict__ out, int32_t* __restrict__ iters,
-               float* __restrict__ x_out) {
+               float* __restrict__ x_out, const float* __restrict__ x0) {
     static_assert(DK % 16 == 0 && DV % 16 == 0 && CH % 16 == 0, "multiples of 16");
     using L = CgSmem<DK, DV, CH>;
     constexpr int TP = CH / 16, IP = DK / 16, VP = DV / 16;
@@ -180,6 +180,42 @@ simt_cg_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* 
         it[a] = 0;
     }
     __syncthreads();
+    if (x0) {
+        // warm start: x = x0, r = p = q - (H_t + Lambda) x0 (one more matvec);
+        // the stopping test stays relative to |q|
+#pragma unroll
+        for (int a = 0; a < TP; ++a) {
+            const int t = tt + 16 * a;
+#pragma unroll
+            for (int b = 0; b < IP; ++b) {
+                const int i = ti + 16 * b;
+                x[a][b] = (t < n) ? x0[(base + t) * DK + i] : 0.f;
+                sP[t * DKP + i] = x[a][b];
+            }
+        }
+        __syncthreads();
+        float y[TP][IP];
+        chunk_matvec<DK, CH>(sP, sH, sK, sW, sM, sE, y);
+#pragma unroll
+        for (int a = 0; a < TP; ++a) {
+            const int t = tt + 16 * a;
+            float s = 0.f;
+#pragma unroll
+            for (int b = 0; b < IP; ++b) {
+                r[a][b] = r[a][b] - fmaf(sL[ti + 16 * b], x[a][b], y[a][b]);
+                p[a][b] = r[a][b];
+                s = fmaf(r[a][b], r[a][b], s);
+            }
+            rr[a] = sum16(s);
+            if (!(t < n)) rr[a] = 0.f;
+        }
+        __syncthreads();                                 // every thread past its reads of sP
+#pragma unroll
+        for (int a = 0; a < TP; ++a)
+#pragma unroll
+            for (int b = 0; b < IP; ++b) sP[(tt + 16 * a) * DKP + ti + 16 * b] = p[a][b];
+        __syncthreads();
+    }
 
     chunk_cg<DK, CH>(sP, sH, sK, sW, sM, sE, sL, x, r, p, rr, qn, act, it, cg_steps, tol);
 
@@ -282,7 +318,7 @@ cudaError_t launch_simt(const ForwardArgs& a, cudaStream_t st) {
         LaunchTimer timer(kKindSimtCg, st);
         kern<<<dim3(nc, BH), kThreads, L::bytes, st>>>(
             static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-            a.gamma, a.beta, a.lambda, a.H, a.T, nc, a.cg_steps, a.tol, states, a.out, a.iters, a.x_out);
+            a.gamma, a.beta, a.lambda, a.H, a.T, nc, a.cg_steps, a.tol, states, a.out, a.iters, a.x_out, a.x0);
     }
     return cudaGetLastError();
 }

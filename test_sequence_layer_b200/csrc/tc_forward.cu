@@ -171,7 +171,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
              const float* __restrict__ beta, const float* __restrict__ lambda, int H, int T, int np,
              int cg_steps, float tol, const __half* __restrict__ img, const float* __restrict__ scales,
              float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err,
-             float* __restrict__ x_out) {
+             float* __restrict__ x_out, const float* __restrict__ x0) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Hs = smem + BlkSmem::oH;
@@ -298,15 +298,31 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
         for (int i = 0; i < 4; ++i) p[4 * g + i] = __bfloat1622float2(b2[i]);
     }
+    // r = q; x = x0 (a warm start) or 0. With x0, p = x0 for the extra first
+    // step that forms r = q - (H_t + Lambda) x0 (below).
+    float qq = 0.f;
+    {
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = __ffma2_rn(p[i], p[i], a);
+        qq = a.x + a.y;
+    }
 #pragma unroll
     for (int h2 = 0; h2 < 4; ++h2) {
         float z[8], rv[8];
+        float4 xa = make_float4(0.f, 0.f, 0.f, 0.f), xb = xa;
+        if (x0 && valid) {
+            const float4* src = reinterpret_cast<const float4*>(x0 + (base + tok) * kD + col0 + 8 * h2);
+            xa = src[0];
+            xb = src[1];
+        }
+        z[0] = xa.x; z[1] = xa.y; z[2] = xa.z; z[3] = xa.w;
+        z[4] = xb.x; z[5] = xb.y; z[6] = xb.z; z[7] = xb.w;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            z[2 * i] = 0.f;
-            z[2 * i + 1] = 0.f;
             rv[2 * i] = p[4 * h2 + i].x;
             rv[2 * i + 1] = p[4 * h2 + i].y;
+            if (x0) p[4 * h2 + i] = make_float2(z[2 * i], z[2 * i + 1]);
         }
         tmem_st32_x8(tl + kColX + col0 + 8 * h2, z);
         tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
@@ -350,19 +366,21 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
         }
     }
-    float rr;
+    float rr, pp;
     {
         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) a = __ffma2_rn(p[i], p[i], a);
-        rr = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;   // barrier publishes seb, Mk
+        const float4 d = quarter_sum(make_float4(qq, a.x + a.y, 0.f, 0.f), red, cq, tok);   // barrier publishes seb, Mk
+        rr = d.x;                                      // |q|^2 = |r|^2
+        pp = d.y;                                      // |p|^2 (|x0|^2 for a warm start)
     }
     tmem_wait_st();
     const float qn = sqrtf(rr);
     bool act = valid;
     int it = 0;
     const float eb = seb[tok];
-    float s = pow2_sqrt_scale(rr), is = 1.f / s;
+    float s = pow2_sqrt_scale(pp), is = 1.f / s;
     store_row32(Ps, tok, col0, p, is);
 
     constexpr uint32_t kIdKK = idesc_f16(128, 128, false, false);     // A and B K-major
@@ -403,8 +421,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 
     if (tid == 0 && !mbar_wait(bar_ld, 0)) *abort_flag = 1.f;
     uint32_t ph = 0;
-    for (int step = 0; step < cg_steps; ++step) {
-        act = act && cg_may_continue(rr, qn, tol);
+    // step -1 (warm start only): the matvec of x0; its update leaves x = x0 and
+    // turns r = q into r_0 = q - (H_t + Lambda) x0, with p_0 = r_0
+    for (int step = x0 ? -1 : 0; step < cg_steps; ++step) {
+        if (step >= 0) act = act && cg_may_continue(rr, qn, tol);
         fence_proxy_async();
         tc_fence_before();
         const int any = __syncthreads_or(act ? 1 : 0);
@@ -467,13 +487,15 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         }
         tmem_wait_st();
         d = quarter_sum(d, red, cq, tok);
-        if (act && !cg_curvature_ok(d.x)) act = false;
+        const bool warm = step < 0;
+        if (act && !warm && !cg_curvature_ok(d.x)) act = false;
         if (act) rr = d.w;                             // true |r|^2 of the current residual
         // alpha and rho feed recurrences that CG corrects: the fast division suffices
-        const float al = act ? __fdividef(rr, d.x) : 0.f;
+        const float al = act ? (warm ? 1.f : __fdividef(rr, d.x)) : 0.f;
         const float rn = fmaxf(fmaf(al, fmaf(al, d.z, -2.f * d.y), rr), 0.f);
-        const float rho = act ? __fdividef(rn, rr) : 0.f;
-        const float2 pa = make_float2(al, al), na = make_float2(-al, -al), rh = make_float2(rho, rho);
+        const float rho = (act && !warm) ? __fdividef(rn, rr) : 0.f;
+        const float ax = warm ? 0.f : al;              // the warm step keeps x = x0
+        const float2 pa = make_float2(ax, ax), na = make_float2(-al, -al), rh = make_float2(rho, rho);
         // the next direction's image is written round by round (its scale is known here)
         const float s_new = act ? pow2_sqrt_scale(rn) : s;
         const float is_new = 1.f / s_new;
@@ -512,7 +534,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         }
         if (act) {
             rr = rn;
-            ++it;
+            if (!warm) ++it;
         }
         s = s_new;
         is = is_new;
@@ -693,7 +715,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
         tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
-            img, scales, a.out, a.iters, err, a.x_out);
+            img, scales, a.out, a.iters, err, a.x_out, a.x0);
     }
 #ifdef MESA_DEBUG
     if (inject) {

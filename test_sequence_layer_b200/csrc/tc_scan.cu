@@ -17,10 +17,11 @@
 // largest |w_j a_j| and |k_j| entries, so every operand lies in [-1, 1]
 // whatever the size of beta, k or v; the state takes sA sK times the sum.
 //
-// Pipeline per chunk c: MMA(c) runs while the CTA builds chunk c+1's operand
-// images (a second set) and warp 1 forms chunk c+2's gates (three gate
-// buffers); then the state takes Delta_c, and the state before every even
-// chunk is staged in shared memory and stored with one bulk copy.
+// Pipeline per chunk c: MMA(c) runs while the CTA writes chunk c+1's operand
+// images (a second set), reads chunk c+2's rows and forms their maxima, and
+// warp 1 forms chunk c+3's gates; then the state takes Delta_c, and the state
+// before every even chunk is staged in shared memory and stored with one bulk
+// copy.
 #include "mesa_internal.h"
 #include "tc_layout.cuh"
 
@@ -29,32 +30,10 @@ namespace {
 
 using namespace tc;
 
-// Inclusive log-cumsum of gamma over a 64-token chunk by warp 0 (padded
-// tokens count as gamma = 1).
-// b[t] for t < 64: in-chunk inclusive cumulative sum of log gamma over the
-// chunk's first n positions, held constant past n. One warp; g points at the
-// chunk's gamma (global or shared memory).
-__device__ __forceinline__ void warp_gate_cumsum(const float* g, int n, float* b) {
-    const int lane = threadIdx.x & 31;
-    const int t0 = 2 * lane, t1 = 2 * lane + 1;
-    const float l0 = (t0 < n) ? logf(g[t0]) : 0.f;
-    const float l1 = (t1 < n) ? logf(g[t1]) : 0.f;
-    const float pair = l0 + l1;
-    float incl = pair;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-    }
-    const float excl = incl - pair;
-    b[t0] = excl + l0;
-    b[t1] = excl + l0 + l1;
-}
-
 // =====================================================================
 // Chunk-state scan
 // =====================================================================
-// The fp16 image of a chunk-start state is scaled by s = 2^ceil(log2 max(Bnd,1))
+// The fp16 image of a chunk-start state is scaled by s = 2^ceil(log2 Bnd)
 // where Bnd bounds every entry: Bnd_0 = max|S_in| and
 // Bnd_{c+1} = e^{b_last} Bnd_c + sum_j w_j |a_j|_inf |k_j|_inf (a = k for H,
 // a = v for G), since |(a_j k_j^T)_il| <= |a_j|_inf |k_j|_inf. Every warp of
@@ -68,9 +47,8 @@ struct ScanSmem {
     static constexpr int oImg = 65536;            // 2 operand sets {A hi, A lo, B}, MN-major SW128, 16 KB each
     static constexpr int kSet = 49152;
     static constexpr int oStage = oImg + 2 * kSet;    // staged state image for the bulk store (32 KB)
-    static constexpr int oGate = oStage + 32768;  // b[3][64], w[3][64], amax[2][64], kmax[2][64]
-    static constexpr int oGraw = oGate + 2560;    // 2 x {gamma[64], beta[64]} prefetched with the rows
-    static constexpr int oRed = oGraw + 1024;     // 32 floats; [31] is the abort flag
+    static constexpr int oGate = oStage + 32768;  // b[4][64], w[4][64], amax[4][64], kmax[4][64]
+    static constexpr int oRed = oGate + 4096;     // 32 floats; [31] is the abort flag
     static constexpr int oCmax = oRed + 128;      // [2 buffers][16 warps] {max w|a|, max |k|} of a chunk
     static constexpr int oBar = oCmax + 256;      // raw[2], mma
     static constexpr int oSlot = oBar + 32;
@@ -82,13 +60,17 @@ struct ScanSmem {
 // serves TMEM lane quadrant w % 4 (state rows 32 (w % 4) .. + 31, one per
 // thread) and the 32 columns 32 (w / 4) .. + 31. Per chunk, with
 // w_j = beta_j e^{b_last - b_j},
-//     S <- e^{b_last} S + sum_j (w_j a_j) k_j^T
+//     S <- e^{b_last} S + sA sK sum_j (w_j a_j / sA) (k_j / sK)^T
 // where the sum is one M = 128, N = 128, K = 64 MMA over the chunk's tokens,
-// issued for the hi and the lo fp16 parts of w_j a_j. The chunks are
-// pipelined: while the MMA of chunk c runs, the CTA builds chunk c+1's
-// operand images (a second set) and warp 1 forms chunk c+2's gates. The state
-// before every even chunk is staged in shared memory in the solve's image
-// layout and written with one bulk copy.
+// issued for the hi and the lo fp16 parts of w_j a_j / sA. The chunks are
+// pipelined so that everything but the state update runs under the MMA of
+// chunk c: the operand images of chunk c+1 are written (a second set, with
+// scales from chunk c+1's maxima, formed one chunk earlier), the rows of
+// chunk c+2 are read into registers and their maxima formed, warp 1 forms
+// chunk c+3's gates from gamma and beta it loaded a chunk earlier, and the
+// rows of chunk c+4 are on their way. The state before every even chunk is
+// staged in shared memory in the solve's image layout and written with one
+// bulk copy.
 __global__ void __launch_bounds__(kScanThreads, 1)
 tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                const float* __restrict__ gamma, const float* __restrict__ beta, int T, int nc,
@@ -101,11 +83,10 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     uint8_t* rawK = smem + ScanSmem::oRawK;
     uint8_t* rawA = m ? smem + ScanSmem::oRawA : rawK;     // for H the left factor is k itself
     uint8_t* stage = smem + ScanSmem::oStage;
-    float* sb = reinterpret_cast<float*>(smem + ScanSmem::oGate);      // [3][64]
-    float* sw = sb + 3 * kC;                                            // [3][64]
-    float* amax = sw + 3 * kC;                                          // [2][64]
-    float* kmax = amax + 2 * kC;                                        // [2][64]
-    float* graw = reinterpret_cast<float*>(smem + ScanSmem::oGraw);
+    float* sb = reinterpret_cast<float*>(smem + ScanSmem::oGate);      // [4][64]
+    float* sw = sb + 4 * kC;                                            // [4][64]
+    float* amax = sw + 4 * kC;                                          // [4][64]
+    float* kmax = amax + 4 * kC;                                        // [4][64]
     float* red = reinterpret_cast<float*>(smem + ScanSmem::oRed);
     float2* cmax = reinterpret_cast<float2*>(smem + ScanSmem::oCmax);
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(smem + ScanSmem::oBar);
@@ -121,60 +102,68 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     float* fin = m ? G_out : H_out;
     const size_t seq = (size_t)bh * T;
     const int np = (nc + 1) >> 1;
-    // gamma/beta of a chunk travel with its rows when the chunk is full and its
-    // first element is 16-byte aligned (T % 4 == 0); otherwise warp 1 reads them.
-    const bool gates_bulk = (T % 4) == 0 && ((reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(beta)) & 15) == 0;
 
-    int prefetched = 0;                           // chunks whose copies were issued (thread 0)
-    auto prefetch = [&](int cc) {                 // rows (and gates) of chunk cc -> buffer cc & 1 (thread 0)
+    int prefetched = 0;                           // chunks whose row copies were issued (thread 0)
+    auto prefetch = [&](int cc) {                 // rows of chunk cc -> buffer cc & 1 (thread 0)
         const int nn = min(kC, T - cc * kC);
         const uint32_t bytes = (uint32_t)nn * kD * 2;
         const int buf = cc & 1;
-        const bool gb = gates_bulk && nn == kC;
-        mbar_arrive_expect_tx(bar_raw + buf, (m ? 2 * bytes : bytes) + (gb ? 512u : 0u));
+        mbar_arrive_expect_tx(bar_raw + buf, m ? 2 * bytes : bytes);
         bulk_g2s(rawK + buf * 16384, k + (seq + (size_t)cc * kC) * kD, bytes, bar_raw + buf);
         if (m) bulk_g2s(rawA + buf * 16384, A + (seq + (size_t)cc * kC) * kD, bytes, bar_raw + buf);
-        if (gb) {
-            bulk_g2s(graw + buf * 128, gamma + seq + (size_t)cc * kC, 256, bar_raw + buf);
-            bulk_g2s(graw + buf * 128 + 64, beta + seq + (size_t)cc * kC, 256, bar_raw + buf);
-        }
         prefetched = cc + 1;
     };
-    // One warp: waits for chunk cc's copies, then b (log-cumsum of gamma) and
-    // w_j = beta_j e^{b_last - b_j} into gate buffer cc % 3.
-    auto chunk_gates = [&](int cc) {
-        const int buf = cc & 1;
-        if (!mbar_wait(bar_raw + buf, (cc >> 1) & 1)) red[31] = 1.f;
-        __syncwarp();
+    auto wait_rows = [&](int cc) {                // every thread: chunk cc's rows have landed
+        if (!mbar_wait(bar_raw + (cc & 1), (cc >> 1) & 1)) red[31] = 1.f;
+    };
+    // Warp 1: gamma and beta of chunk cc into registers (lane: positions 2 lane, 2 lane + 1;
+    // padding positions read as gamma = 1, beta = 0).
+    float pg0 = 1.f, pg1 = 1.f, pb0 = 0.f, pb1 = 0.f;
+    auto load_gates = [&](int cc) {
         const int nn = min(kC, T - cc * kC);
         const size_t base = seq + (size_t)cc * kC;
-        const bool gb = gates_bulk && nn == kC;
-        const float* gsrc = gb ? graw + buf * 128 : gamma + base;
-        const float* bsrc = gb ? graw + buf * 128 + 64 : beta + base;
-        float* b = sb + (cc % 3) * kC;
-        float* wv = sw + (cc % 3) * kC;
-        warp_gate_cumsum(gsrc, nn, b);
-        __syncwarp();
-        const float bl = b[kC - 1];                                // b at the chunk's last position
-        wv[lane] = (lane < nn) ? bsrc[lane] * expf(bl - b[lane]) : 0.f;
-        wv[lane + 32] = (lane + 32 < nn) ? bsrc[lane + 32] * expf(bl - b[lane + 32]) : 0.f;
+        const int t0 = 2 * lane, t1 = 2 * lane + 1;
+        pg0 = t0 < nn ? gamma[base + t0] : 1.f;
+        pg1 = t1 < nn ? gamma[base + t1] : 1.f;
+        pb0 = t0 < nn ? beta[base + t0] : 0.f;
+        pb1 = t1 < nn ? beta[base + t1] : 0.f;
     };
-    // Operand images of chunk cc, in two phases around a CTA barrier.
-    // build_load: this thread's two 16-byte pieces of the rows of a (and of k
-    // for G) into registers, the row maxima of |a| and |k| into buffer cc & 1
-    // (for the state bound) and this warp's maxima of w_j |a_j| and |k_j| into
-    // cmax (for the chunk's operand scales).
-    // build_store: sA, sK from cmax, then A = w_j a_j / sA (hi/lo) [j][i] and
-    // B = k_j / sK [j][l] into set cc & 1, both MN-major SW128 in two
+    // Warp 1: from the loaded gates of chunk cc, b (the in-chunk inclusive
+    // log-cumsum of gamma) and w_j = beta_j e^{b_last - b_j} into buffer cc & 3.
+    auto chunk_gates = [&](int cc) {
+        float* b = sb + (cc & 3) * kC;
+        float* wv = sw + (cc & 3) * kC;
+        const float l0 = logf(pg0), l1 = logf(pg1);
+        const float pair = l0 + l1;
+        float incl = pair;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        const float b0 = incl - pair + l0, b1 = incl;
+        const float bl = __shfl_sync(0xffffffffu, incl, 31);     // b at the chunk's last position
+        b[2 * lane] = b0;
+        b[2 * lane + 1] = b1;
+        wv[2 * lane] = pb0 * expf(bl - b0);
+        wv[2 * lane + 1] = pb1 * expf(bl - b1);
+    };
+    // Operand images of chunk cc, in two phases a pipeline stage apart.
+    // build_load (stage cc-2): this thread's two 16-byte pieces of the rows of
+    // a (and of k for G) into registers, the row maxima of |a| and |k| into
+    // buffer cc & 3 (for the state bound) and this warp's maxima of w_j |a_j|
+    // and |k_j| into cmax buffer cc & 1 (for the chunk's operand scales).
+    // build_store (stage cc-1): sA, sK from cmax, then A = w_j a_j / sA (hi/lo)
+    // [j][i] and B = k_j / sK [j][l] into set cc & 1, both MN-major SW128 in two
     // 64-column blocks; returns sA sK, the factor the chunk's product carries.
     uint4 ra[2], rk[2];
     auto build_load = [&](int cc) {
         const int n = min(kC, T - cc * kC);
-        const float* swc = sw + (cc % 3) * kC;
+        const float* swc = sw + (cc & 3) * kC;
         const uint8_t* rpa = rawA + (cc & 1) * 16384;
         const uint8_t* rpk = rawK + (cc & 1) * 16384;
-        float* am = amax + (cc & 1) * kC;
-        float* km = kmax + (cc & 1) * kC;
+        float* am = amax + (cc & 3) * kC;
+        float* km = kmax + (cc & 3) * kC;
         float wa = 0.f, wk = 0.f;
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
@@ -216,7 +205,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         if (lane == 0) cmax[(cc & 1) * 16 + w] = make_float2(wa, wk);
     };
     auto build_store = [&](int cc) -> float {
-        const float* swc = sw + (cc % 3) * kC;
+        const float* swc = sw + (cc & 3) * kC;
         uint8_t* Ahi = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
         uint8_t* Alo = Ahi + 16384;
         uint8_t* Bk = Ahi + 32768;
@@ -313,11 +302,14 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
 #pragma unroll
         for (int i = 1; i < kScanThreads / 32; ++i) bound = fmaxf(bound, red[i]);
     }
-    if (w == 1 && nc > 0) {
-        chunk_gates(0);
-        if (nc > 1) chunk_gates(1);
+    if (w == 1) {                                  // gates of chunks 0..2, gamma and beta of chunk 3
+        for (int cc = 0; cc < 3 && cc < nc; ++cc) {
+            load_gates(cc);
+            chunk_gates(cc);
+        }
+        if (nc > 3) load_gates(3);
     }
-    __syncthreads();                              // gates of chunks 0 and 1 (and the bound's partials) read
+    __syncthreads();                              // gates visible (and the bound's partials read)
     bool ok = red[31] == 0.f;
 
     constexpr uint32_t kIdesc = idesc_f16(128, 128, true, true);
@@ -335,7 +327,8 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     int mma_issued = 0, mma_seen = 0;             // thread 0
     float ds_cur = 1.f, ds_next = 1.f;            // sA sK of the chunk in the MMA, of the next chunk
     if (ok && nc > 0) {
-        // the state before chunk 0 (block 0's image) and chunk 0's operands
+        // the state before chunk 0 (block 0's image), chunk 0's operands, chunk 1's rows
+        wait_rows(0);
         build_load(0);
         __syncthreads();                          // chunk 0's maxima
         ds_cur = build_store(0);
@@ -349,23 +342,40 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             bulk_s2g(img + ci * kImgHalves, stage, kImgBytes);
             bulk_commit();
             scales[ci] = s0;
-            issue_mma(0);
-            ++mma_issued;
+            if (red[31] == 0.f) {
+                issue_mma(0);
+                ++mma_issued;
+            }
             if (nc > 2) prefetch(2);              // raw buffer 0 is consumed
         }
+        if (nc > 1) {
+            wait_rows(1);
+            build_load(1);
+        }
+        __syncthreads();                          // chunk 1's maxima; raw buffer 1 consumed
+        if (tid == 0 && nc > 3) prefetch(3);
+        ok = red[31] == 0.f;
     }
     int c = 0;
     for (; ok && c < nc; ++c) {
-        // ---- while MMA(c) runs: chunk c+1's rows and maxima, chunk c+2's gates, the bound after chunk c ----
-        if (c + 1 < nc) build_load(c + 1);
-        if (w == 1 && c + 2 < nc) chunk_gates(c + 2);
-        const float blast = sb[(c % 3) * kC + kC - 1];
+        // ---- under MMA(c): chunk c+1's images, chunk c+2's rows and maxima,
+        //      chunk c+3's gates, the bound after chunk c ----
+        if (c + 1 < nc) ds_next = build_store(c + 1);
+        if (c + 2 < nc) {
+            wait_rows(c + 2);
+            build_load(c + 2);
+        }
+        if (w == 1 && c + 3 < nc) {
+            chunk_gates(c + 3);
+            if (c + 4 < nc) load_gates(c + 4);
+        }
+        const float blast = sb[(c & 3) * kC + kC - 1];
         {
             // every warp reduces the same 64 terms in the same order, so every
             // thread gets the same value
-            const float* swc = sw + (c % 3) * kC;
-            const float* am = amax + (c & 1) * kC;
-            const float* km = (m ? kmax : amax) + (c & 1) * kC;
+            const float* swc = sw + (c & 3) * kC;
+            const float* am = amax + (c & 3) * kC;
+            const float* km = (m ? kmax : amax) + (c & 3) * kC;
             float add = swc[lane] * (am[lane] * km[lane]) + swc[lane + 32] * (am[lane + 32] * km[lane + 32]);
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) add += __shfl_xor_sync(0xffffffffu, add, off);
@@ -377,20 +387,21 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             else red[31] = 1.f;
             if (emit) bulk_wait_read_all();       // the staging buffer is free again
         }
-        __syncthreads();                          // MMA(c) done; maxima of c+1 and gates of c+2 written
+        __syncthreads();                          // MMA(c) done; images of c+1, maxima of c+2, gates of c+3 written
         tc_fence_after();
         if (red[31] != 0.f) {
             ok = false;
             break;
         }
-        // ---- chunk c+1's operand images; S <- e^{b_last} S + sA sK Delta ----
+        // ---- S <- e^{b_last} S + sA sK Delta ----
         const float Gam = expf(blast);
-        float dv[32];
-        tmem_ld32_x32(tbase + ((uint32_t)(32 * q4) << 16) + col0, dv);
-        if (c + 1 < nc) ds_next = build_store(c + 1);
-        tmem_wait_ld();
+        {
+            float dv[32];
+            tmem_ld32_x32(tbase + ((uint32_t)(32 * q4) << 16) + col0, dv);
+            tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] = fmaf(Gam, S[i], ds_cur * dv[i]);
+            for (int i = 0; i < 32; ++i) S[i] = fmaf(Gam, S[i], ds_cur * dv[i]);
+        }
         if (c + 1 == nc) {                        // the final state
             if (fin) {
                 float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0);
@@ -403,7 +414,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         if (emit) s_img = stage_state(S, bound);  // the state before chunk c+1 starts block (c+1)/2
         fence_proxy_async();
         tc_fence_before();
-        __syncthreads();                          // TMEM read; staging image written
+        __syncthreads();                          // TMEM read; staging image and chunk c+1's images written
         tc_fence_after();
         if (tid == 0) {
             if (emit) {
@@ -414,7 +425,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             }
             issue_mma(c + 1);
             ++mma_issued;
-            if (c + 3 < nc) prefetch(c + 3);      // raw buffer (c+1) & 1 is consumed
+            if (c + 4 < nc) prefetch(c + 4);      // raw buffer c & 1 is consumed (chunk c+2's rows)
         }
         ds_cur = ds_next;
     }

@@ -43,6 +43,8 @@ def _load():
     lib.mesa_forward.argtypes = fwd
     lib.mesa_forward.restype = I
     lib.mesa_forward_host.argtypes = fwd
+    lib.mesa_forward_warm.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, Z, P]
+    lib.mesa_forward_warm.restype = I
     lib.mesa_forward_host.restype = I
     lib.mesa_forward_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.mesa_forward_workspace_size.restype = Z
@@ -148,6 +150,43 @@ def forward(q, k, v, gamma, beta, lam, *, chunk=64, cg_steps=15, tol=0.0, out=No
     if return_state:
         res += (H_out, G_out)
     return res[0] if len(res) == 1 else res
+
+
+def forward_warm(q, k, v, gamma, beta, lam, x0, *, chunk=64, cg_steps=15, tol=0.0, out=None, x_out=None,
+                 return_iters=False, iters=None, H_in=None, G_in=None, return_state=False, workspace=None,
+                 stream=None):
+    """forward() with every token's CG started from x0 [B,H,T,dk] float32
+    (None: from zero). Returns (out, x) where x [B,H,T,dk] float32 holds the
+    solutions (written into `x_out` when given; x_out may be x0 itself), plus
+    iters if return_iters, plus (H_out, G_out) if return_state."""
+    lib = _load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32, device=dev)
+    if x_out is None:
+        x_out = torch.empty((B, H, T, dk), dtype=torch.float32, device=dev)
+    if return_iters and iters is None:
+        iters = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+    H_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev) if return_state else None
+    G_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev) if return_state else None
+    need = int(lib.mesa_forward_workspace_size(B, H, T, dk, dv, chunk, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.mesa_forward_warm(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                               B, H, T, dk, dv, chunk, code, int(cg_steps), float(tol), _ptr(x0), _ptr(x_out),
+                               _ptr(out), _ptr(iters), _ptr(H_in), _ptr(G_in), _ptr(H_out), _ptr(G_out),
+                               _ptr(workspace), ws_bytes, _stream(stream, dev))
+    _check(rc, "mesa_forward_warm")
+    res = (out, x_out)
+    if return_iters:
+        res += (iters,)
+    if return_state:
+        res += (H_out, G_out)
+    return res
 
 
 def backward(q, k, v, gamma, beta, lam, dout, *, chunk=64, cg_steps=15, tol=0.0, workspace=None, stream=None):
