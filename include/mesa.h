@@ -211,6 +211,40 @@ mesa_status mesa_preprocess(const void* q_raw, const void* k_raw, const float* c
                             void* stream);
 
 /*
+ * The forward with the q/k input preprocessing of mesa_preprocess applied on
+ * the way in: equals mesa_preprocess(q_raw, k_raw, conv_q, conv_k, W)
+ * followed by mesa_forward on its outputs, bit for bit. Source: the MesaNet
+ * page, Technical summary > Architecture > "Preprocessing" (read as for
+ * mesa_preprocess: causal depthwise convolution, then L2 normalisation, the
+ * convolution starting from zero rows at the call's first token).
+ *
+ * On the tensor-core shape (MESA_BF16, dk = dv = 128, chunk = 64) nothing is
+ * preprocessed ahead: the chunk-state scan and the solve convolve and
+ * normalise the raw rows as they stage them (each 128-token block with the
+ * three rows before it), so the preprocessed q and k never go to memory.
+ * Every other shape runs the two steps, with the preprocessed q and k in
+ * the workspace.
+ *
+ *   q_raw, k_raw  raw queries and keys, [B,H,T,dk] in `dtype`, 16-byte aligned.
+ *   conv_q, conv_k  float32 [H,W,dk] weights (w = lag), 4-byte aligned.
+ *   W             window, 1..4.
+ *   workspace     at least mesa_forward_preprocessed_workspace_size() bytes,
+ *                 256-byte aligned.
+ * Every other argument as for mesa_forward.
+ */
+size_t mesa_forward_preprocessed_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                                mesa_dtype dtype);
+mesa_status mesa_forward_preprocessed(const void* q_raw, const void* k_raw, const void* v,
+                                      const float* gamma, const float* beta, const float* lambda,
+                                      const float* conv_q, const float* conv_k, int W,
+                                      int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                                      int cg_steps, float tol,
+                                      float* out, int32_t* iters_out,
+                                      const float* H_in, const float* G_in,
+                                      float* H_out, float* G_out,
+                                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Backward pass of the layer (training): gradients of a scalar loss L given
  * dout = dL/do for the inputs of a mesa_forward call with zero initial
  * states. The pages claim training in time linear in T but give no backward

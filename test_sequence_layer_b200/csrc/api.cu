@@ -273,6 +273,65 @@ mesa_status mesa_forward_warm(const void* q, const void* k, const void* v,
     return launch_forward(a, static_cast<cudaStream_t>(stream));
 }
 
+size_t mesa_forward_preprocessed_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                                mesa_dtype dtype) {
+    if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
+    const size_t fw = workspace_bytes(B, H, T, dk, dv, chunk, dtype);
+    if (tc_supported(dk, dv, chunk, dtype)) return fw;          // fused: the forward's own workspace
+    return round_up((size_t)B * H * T * dk * elem_size(dtype), 256) * 2 + fw;   // + preprocessed q, k
+}
+
+mesa_status mesa_forward_preprocessed(const void* q_raw, const void* k_raw, const void* v,
+                                      const float* gamma, const float* beta, const float* lambda,
+                                      const float* conv_q, const float* conv_k, int W,
+                                      int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype,
+                                      int cg_steps, float tol,
+                                      float* out, int32_t* iters_out,
+                                      const float* H_in, const float* G_in,
+                                      float* H_out, float* G_out,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+    mesa_status s = check_shape(B, H, T, dk, dv, chunk, dtype, cg_steps, tol);
+    if (s != MESA_OK) return s;
+    if (W < 1 || W > 4 || !conv_q || !conv_k || !aligned(conv_q, 4) || !aligned(conv_k, 4)) return MESA_ERR_INVALID_ARG;
+    if (!lambda || !aligned(lambda, 4)) return MESA_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!q_raw || !k_raw || !v || !gamma || !beta || !out) return MESA_ERR_INVALID_ARG;
+        if (!aligned(q_raw, 16) || !aligned(k_raw, 16) || !aligned(v, 16) || !aligned(out, 16))
+            return MESA_ERR_INVALID_ARG;
+        if (!aligned(gamma, 4) || !aligned(beta, 4)) return MESA_ERR_INVALID_ARG;
+        if (iters_out && !aligned(iters_out, 4)) return MESA_ERR_INVALID_ARG;
+    }
+    for (const void* p : {(const void*)H_in, (const void*)G_in, (const void*)H_out, (const void*)G_out})
+        if (p && !aligned(p, 16)) return MESA_ERR_INVALID_ARG;
+    if ((H_out && H_out == H_in) || (G_out && G_out == G_in)) return MESA_ERR_INVALID_ARG;
+    const size_t need = mesa_forward_preprocessed_workspace_size(B, H, T, dk, dv, chunk, dtype);
+    if (T > 0 && need > 0) {
+        if (!workspace || ws_bytes < need) return MESA_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return MESA_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ForwardArgs a{q_raw, k_raw, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps, tol,
+                  out, iters_out, H_in, G_in, H_out, G_out, workspace, ws_bytes};
+    if (T > 0 && tc_supported(dk, dv, chunk, dtype)) {
+        // the scan and the solve convolve and normalise the raw rows as they stage them
+        a.conv_q = conv_q;
+        a.conv_k = conv_k;
+        a.conv_w = W;
+        return launch_forward(a, st);
+    }
+    if (T > 0) {      // the other shapes: preprocessing into the workspace, then the forward
+        const size_t qb = round_up((size_t)B * H * T * dk * elem_size(dtype), 256);
+        char* w = static_cast<char*>(workspace);
+        PreArgs pa{q_raw, k_raw, conv_q, conv_k, B, H, T, dk, W, dtype, w, w + qb};
+        if (preprocess_launch(pa, st) != cudaSuccess) return MESA_ERR_CUDA;
+        a.q = w;
+        a.k = w + qb;
+        a.workspace = w + 2 * qb;
+        a.ws_bytes = ws_bytes - 2 * qb;
+    }
+    return launch_forward(a, st);
+}
+
 size_t mesa_backward_workspace_size(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype dtype) {
     if (check_shape(B, H, T, dk, dv, chunk, dtype, 0, 0.f) != MESA_OK) return 0;
     return backward_workspace_bytes(B, H, T, dk, dv, chunk, dtype);

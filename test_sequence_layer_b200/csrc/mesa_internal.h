@@ -31,6 +31,11 @@ struct ForwardArgs {
     size_t ws_bytes;
     float* x_out = nullptr;     // the CG solutions x_t [B,H,T,dk] (fp32), when not null
     const float* x0 = nullptr;  // per-token CG starting guesses [B,H,T,dk] (fp32), when not null
+    // fused input preprocessing (tensor-core path): q and k are raw, and the
+    // kernels convolve and normalise them as they stage them (weights [H,W,dk])
+    const float* conv_q = nullptr;
+    const float* conv_k = nullptr;
+    int conv_w = 0;
     bool scan_only = false;     // fp32 CUDA-core path only: the chunk-state scan, no solve
 };
 

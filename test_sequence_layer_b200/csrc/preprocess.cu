@@ -21,6 +21,7 @@
 
 #include "mesa_common.cuh"
 #include "mesa_internal.h"
+#include "preproc_row.cuh"
 #include "tc_common.cuh"
 
 namespace mesa {
@@ -28,7 +29,7 @@ namespace {
 
 constexpr int kPreWarps = 8;
 constexpr int kTile = 128;                // tokens per CTA
-constexpr int kMaxW = 4;
+constexpr int kMaxW = pre::kMaxW;
 
 // Eight channels of one row: fp32 (two 16-byte loads) or bf16 (one).
 __device__ __forceinline__ void load8(const float* p, float2 (&v)[4]) {
@@ -102,11 +103,7 @@ preprocess_kernel(const E* __restrict__ xq, const E* __restrict__ xk, const floa
     }
     for (int e = tid; e < skip * D; e += 32 * kPreWarps) rows[e] = E(0.f);
     float2 c[kMaxW][4];                               // weights by lag, channel pairs
-#pragma unroll
-    for (int w = 0; w < kMaxW; ++w)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            c[w][j] = w < W ? make_float2(conv[w * D + c0 + 2 * j], conv[w * D + c0 + 2 * j + 1]) : make_float2(0.f, 0.f);
+    pre::load_weights8<D>(conv, W, c0, c);
     const bool landed = tc::mbar_wait(&bar, 0);
     __syncthreads();                                  // zero-filled halo rows visible
     if (!landed) {
@@ -117,26 +114,11 @@ preprocess_kernel(const E* __restrict__ xq, const E* __restrict__ xk, const floa
 #pragma unroll 2
     for (int r = warp * RPS + grp; r < n; r += kRowStride) {
         const E* src = rows + (size_t)(r + kHalo) * D + c0;   // token t0 + r
-        float2 u[4], xs[4];
-        lds8(src, xs);
+        float2 u[4], xs[kMaxW][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) u[j] = __fmul2_rn(c[0][j], xs[j]);
-#pragma unroll
-        for (int w = 1; w < kMaxW; ++w) {
-            lds8(src - (size_t)w * D, xs);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) u[j] = __ffma2_rn(c[w][j], xs[j], u[j]);
-        }
-        float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) ss2 = __ffma2_rn(u[j], u[j], ss2);
-        float ss = ss2.x + ss2.y;
-#pragma unroll
-        for (int off = LPR / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
-        const float inv = 1.f / fmaxf(sqrtf(ss), 1e-6f);
-        const float2 iv = make_float2(inv, inv);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) u[j] = __fmul2_rn(u[j], iv);
+        for (int w = 0; w < kMaxW; ++w) lds8(src - (size_t)w * D, xs[w]);
+        pre::conv8(c, xs, u);
+        pre::norm8<LPR>(u);
         store8(y + (size_t)(t0 + r) * D + c0, u);
     }
 }

@@ -37,6 +37,7 @@
 //                   columns); every dot product is a thread-local sum plus one
 //                   shared-memory exchange across the four column quarters.
 #include "mesa_internal.h"
+#include "preproc_row.cuh"
 #include "tc_layout.cuh"
 
 namespace mesa {
@@ -98,7 +99,11 @@ struct BlkSmem {
     static constexpr int oMisc = oRed + 8192;     // 32 floats
     static constexpr int oBar = oMisc + 128;      // mbarriers: ld (H), s, u, z, g (G), in (rows), v (values)
     static constexpr int oSlot = oBar + 64;
-    static constexpr int bytes = oSlot + 16;
+    static constexpr int oConvK = oSlot + 16;     // fused preprocessing: key and query weights [4][128],
+    static constexpr int oConvQ = oConvK + 2048;
+    static constexpr int oHaloK = oConvQ + 2048;  // and the 3 raw key and query rows before the block
+    static constexpr int oHaloQ = oHaloK + 768;
+    static constexpr int bytes = oHaloQ + 768;
 };
 
 // b[t], t < 128: cumulative sum of log gamma over positions 0..t of the first
@@ -171,7 +176,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
              const float* __restrict__ beta, const float* __restrict__ lambda, int H, int T, int np,
              int cg_steps, float tol, const __half* __restrict__ img, const float* __restrict__ scales,
              float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err,
-             float* __restrict__ x_out, const float* __restrict__ x0) {
+             float* __restrict__ x_out, const float* __restrict__ x0, const float* __restrict__ conv_q,
+             const float* __restrict__ conv_k, int conv_w) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Hs = smem + BlkSmem::oH;
@@ -195,6 +201,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     uint64_t* bar_in = bar_ld + 5;
     uint64_t* bar_v = bar_ld + 6;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + BlkSmem::oSlot);
+    float* sconvK = reinterpret_cast<float*>(smem + BlkSmem::oConvK);
+    float* sconvQ = reinterpret_cast<float*>(smem + BlkSmem::oConvQ);
+    uint8_t* haloK = smem + BlkSmem::oHaloK;
+    uint8_t* haloQ = smem + BlkSmem::oHaloQ;
 
     const int blk = blockIdx.x, bh = blockIdx.y, head = bh % H;
     const int t0 = blk * kBlk;
@@ -231,30 +241,48 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);     // this warp's lane quadrant
     constexpr uint32_t kColU = 0, kColS = 128, kColX = 256, kColR = 384;
 
-    // One round of bulk copies brings everything the setup reads: both state
-    // images, the raw key rows (staged in the P-hat buffer), the raw query rows
-    // (staged in the score buffer) and, for a full aligned block, gamma and beta
-    // (staged in the reduction buffer).
+    // Bulk copies: first what the set-up reads (the raw key rows staged in the
+    // P-hat buffer, the raw query rows staged in the score buffer and, for a
+    // full aligned block, gamma and beta staged in the reduction buffer); the
+    // two state images follow once those have landed, so that they do not
+    // share the memory bandwidth with them (H is first read by the first MMA,
+    // G by the read-out).
     const uint32_t row_bytes = (uint32_t)n * kD * 2;
     const bool gates_bulk = n == kBlk && ((reinterpret_cast<uintptr_t>(gamma + base) |
                                             reinterpret_cast<uintptr_t>(beta + base)) & 15) == 0;
     float* gstage = reinterpret_cast<float*>(red);
+    // Fused input preprocessing (conv_k given): q and k arrive raw, with the
+    // three rows before the block, and are convolved and normalised here.
+    const bool fuse = conv_k != nullptr;
+    const bool halo_rows = fuse && t0 >= pre::kMaxW - 1;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_ld, kImgBytes);
-        bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
-        mbar_arrive_expect_tx(bar_g, kImgBytes);
-        bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
-        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u));
+        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u) + (halo_rows ? 2u * 768u : 0u));
         bulk_g2s(Ps, k + base * kD, row_bytes, bar_in);
         bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
         if (gates_bulk) {
             bulk_g2s(gstage, gamma + base, kBlk * 4, bar_in);
             bulk_g2s(gstage + kBlk, beta + base, kBlk * 4, bar_in);
         }
+        if (halo_rows) {
+            bulk_g2s(haloK, k + (base - 3) * kD, 768, bar_in);
+            bulk_g2s(haloQ, q + (base - 3) * kD, 768, bar_in);
+        }
+    }
+    if (fuse) {
+        pre::stage_weights<kD>(conv_k + (size_t)head * conv_w * kD, conv_w, sconvK);
+        pre::stage_weights<kD>(conv_q + (size_t)head * conv_w * kD, conv_w, sconvQ);
+        if (!halo_rows)                                // rows before the sequence start are zero
+            for (int e = tid; e < 2 * 768 / 16; e += kBlkThreads) reinterpret_cast<uint4*>(haloK)[e] = make_uint4(0, 0, 0, 0);
     }
     const float sH = scales[iH];
     if (tid >= kBlk && tid < kBlk + kD) slam[tid - kBlk] = lambda[(size_t)head * kD + tid - kBlk];
-    if (tid == 0 && !mbar_wait(bar_in, 0)) *abort_flag = 1.f;
+    if (tid == 0) {
+        if (!mbar_wait(bar_in, 0)) *abort_flag = 1.f;
+        mbar_arrive_expect_tx(bar_ld, kImgBytes);
+        bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
+        mbar_arrive_expect_tx(bar_g, kImgBytes);
+        bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
+    }
     __syncthreads();
 
     // gates and beta; the raw key rows (held in registers until the key image
@@ -265,6 +293,18 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         bmax = (tid < n) ? (gates_bulk ? gstage[kBlk + tid] : beta[base + tid]) : 0.f;
         sbeta[tid] = bmax;
     }
+    // a raw piece (row j, channels 8 cc..) of staged rows -> its preprocessed piece
+    auto preprocess_piece = [&](const uint8_t* rows, const uint8_t* halo, const float* sw, int j, int cc,
+                                uint4 raw) -> uint4 {
+        uint4 x[pre::kMaxW];
+        x[0] = raw;
+#pragma unroll
+        for (int wl = 1; wl < pre::kMaxW; ++wl)
+            x[wl] = j >= wl ? *reinterpret_cast<const uint4*>(rows + (j - wl) * 256 + cc * 16)
+                            : *reinterpret_cast<const uint4*>(halo + (3 + j - wl) * 256 + cc * 16);
+        const uint4 y = pre::conv_norm_bf16x8_sw<kD, 16>(sw, cc * 8, x);
+        return j < n ? y : make_uint4(0, 0, 0, 0);
+    };
     uint4 kraw[4];
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
@@ -272,6 +312,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         const int j = cid >> 4, cc = cid & 15;
         kraw[rep] = make_uint4(0, 0, 0, 0);
         if (j < n) kraw[rep] = *reinterpret_cast<const uint4*>(Ps + j * 256 + cc * 16);
+        if (fuse) kraw[rep] = preprocess_piece(Ps, haloK, sconvK, j, cc, kraw[rep]);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[rep]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -287,6 +328,24 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     if (lane == 0) {
         misc[w] = kmax;
         if (w < 4) misc[16 + w] = bmax;
+    }
+    if (fuse) {                                        // queries preprocessed in place in their staging buffer
+        uint4 qp[4];
+#pragma unroll
+        for (int rep = 0; rep < 4; ++rep) {
+            const int cid = tid + kBlkThreads * rep;
+            const int j = cid >> 4, cc = cid & 15;
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (j < n) raw = *reinterpret_cast<const uint4*>(Ws + j * 256 + cc * 16);
+            qp[rep] = preprocess_piece(Ws, haloQ, sconvQ, j, cc, raw);
+        }
+        __syncthreads();                               // every raw query row read
+#pragma unroll
+        for (int rep = 0; rep < 4; ++rep) {
+            const int cid = tid + kBlkThreads * rep;
+            *reinterpret_cast<uint4*>(Ws + (cid >> 4) * 256 + (cid & 15) * 16) = qp[rep];
+        }
+        __syncthreads();
     }
     // CG state: x = 0 and r = q in TMEM, p = q in registers; this thread: token tok, columns col0..col0+31
     float2 p[16];
@@ -421,9 +480,15 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 
     if (tid == 0 && !mbar_wait(bar_ld, 0)) *abort_flag = 1.f;
     uint32_t ph = 0;
+    auto fetch_values = [&]() {                        // raw value rows into the dead H buffer
+        mbar_arrive_expect_tx(bar_v, row_bytes);
+        bulk_g2s(Hs, v + base * kD, row_bytes, bar_v);
+    };
+    const int first_step = x0 ? -1 : 0;
+    int step = first_step;
     // step -1 (warm start only): the matvec of x0; its update leaves x = x0 and
     // turns r = q into r_0 = q - (H_t + Lambda) x0, with p_0 = r_0
-    for (int step = x0 ? -1 : 0; step < cg_steps; ++step) {
+    for (; step < cg_steps; ++step) {
         if (step >= 0) act = act && cg_may_continue(rr, qn, tol);
         fence_proxy_async();
         tc_fence_before();
@@ -453,6 +518,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         wait_mma_each(bar_u, ph & 1, abort_flag);
         wait_mma_each(bar_z, ph & 1, abort_flag);
         ++ph;
+        // with a fixed step count the last U product is known: H is dead from
+        // here, and the read-out's value rows can be on their way during this
+        // step's CUDA-core work
+        if (tid == 0 && tol <= 0.f && step == cg_steps - 1) fetch_values();
 
         // y = s (sH e^b U + sW Z) + lambda p (written over Z); partials p.y, r.y, y.y, r.r
         const float c_u = s * sH * eb, c_z = s * sW;
@@ -543,10 +612,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 
     // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern,
     // with X-hat = x / |x|, V / sV (sV >= max |v|) and the same key and mask images ----
-    if (tid == 0) {            // raw value rows into the dead H buffer, while x is normalised
-        mbar_arrive_expect_tx(bar_v, row_bytes);
-        bulk_g2s(Hs, v + base * kD, row_bytes, bar_v);
-    }
+    // unless the last fixed step already sent them (the loop ran to its end)
+    const bool v_sent = tol <= 0.f && step == cg_steps && cg_steps > first_step;
+    if (tid == 0 && !v_sent) fetch_values();          // while x is normalised
     __syncthreads();                                   // last reduction's readers are done with red[]
     float xs;
     {
@@ -715,7 +783,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
         tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
-            img, scales, a.out, a.iters, err, a.x_out, a.x0);
+            img, scales, a.out, a.iters, err, a.x_out, a.x0, a.conv_q, a.conv_k, a.conv_w);
     }
 #ifdef MESA_DEBUG
     if (inject) {

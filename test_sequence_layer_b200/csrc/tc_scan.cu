@@ -23,6 +23,7 @@
 // before every even chunk is staged in shared memory and stored with one bulk
 // copy.
 #include "mesa_internal.h"
+#include "preproc_row.cuh"
 #include "tc_layout.cuh"
 
 namespace mesa {
@@ -49,10 +50,12 @@ struct ScanSmem {
     static constexpr int oStage = oImg + 2 * kSet;    // staged state image for the bulk store (32 KB)
     static constexpr int oGate = oStage + 32768;  // b[4][64], w[4][64], amax[4][64], kmax[4][64]
     static constexpr int oRed = oGate + 4096;     // 32 floats; [31] is the abort flag
-    static constexpr int oCmax = oRed + 128;      // [2 buffers][16 warps] {max w|a|, max |k|} of a chunk
+    static constexpr int oCmax = oRed + 128;      // [2 buffers] {max w|a|, max |k|} of a chunk (as int bits)
     static constexpr int oBar = oCmax + 256;      // raw[2], mma
     static constexpr int oSlot = oBar + 32;
-    static constexpr int bytes = oSlot + 16;
+    static constexpr int oConv = oSlot + 16;      // key convolution weights [4 lags][128] (fused preprocessing)
+    static constexpr int oHalo = oConv + 2048;    // 2 x the 3 raw key rows before a chunk (fused preprocessing)
+    static constexpr int bytes = oHalo + 2 * 768;
 };
 
 // CTA (m, bh) walks the chunks of sequence bh for m = 0 (H, a = k) or m = 1
@@ -76,7 +79,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
                const float* __restrict__ gamma, const float* __restrict__ beta, int T, int nc,
                const float* __restrict__ H_in, const float* __restrict__ G_in, __half* __restrict__ img,
                float* __restrict__ scales, float* __restrict__ H_out, float* __restrict__ G_out,
-               unsigned* __restrict__ err) {
+               unsigned* __restrict__ err, const float* __restrict__ conv_k, int conv_w, int H) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int m = blockIdx.x, bh = blockIdx.y;
@@ -88,10 +91,16 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     float* amax = sw + 4 * kC;                                          // [4][64]
     float* kmax = amax + 4 * kC;                                        // [4][64]
     float* red = reinterpret_cast<float*>(smem + ScanSmem::oRed);
-    float2* cmax = reinterpret_cast<float2*>(smem + ScanSmem::oCmax);
+    // Chunk maxima, kept as the bit patterns of non-negative floats (which
+    // order like the floats), so each warp folds its maximum in with one
+    // shared-memory atomicMax; buffer cc & 1, cleared after its chunk's images
+    // are written.
+    int* cmax = reinterpret_cast<int*>(smem + ScanSmem::oCmax);
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(smem + ScanSmem::oBar);
     uint64_t* bar_mma = bar_raw + 2;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + ScanSmem::oSlot);
+    float* sconv = reinterpret_cast<float*>(smem + ScanSmem::oConv);
+    uint8_t* halo = smem + ScanSmem::oHalo;           // [2][3 rows][256 B]
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int q4 = w & 3;
@@ -156,6 +165,23 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     // build_store (stage cc-1): sA, sK from cmax, then A = w_j a_j / sA (hi/lo)
     // [j][i] and B = k_j / sK [j][l] into set cc & 1, both MN-major SW128 in two
     // 64-column blocks; returns sA sK, the factor the chunk's product carries.
+    // Fused input preprocessing of the keys (conv_k given): the raw piece of
+    // row j of chunk cc becomes its convolved, normalised bf16 piece. The rows
+    // before it come from the chunk's raw rows or, for its first three rows,
+    // from the halo buffer cc & 1, which holds the previous chunk's last three
+    // raw rows (zero before the sequence start); the chunk's own last three
+    // raw rows go to halo buffer (cc + 1) & 1. Padding rows (j >= n) give zero.
+    auto preprocess_key = [&](int cc, int n, int j, int cc16, const uint8_t* rows, uint4 raw) -> uint4 {
+        uint4 x[pre::kMaxW];
+        x[0] = raw;
+#pragma unroll
+        for (int w = 1; w < pre::kMaxW; ++w)
+            x[w] = j >= w ? *reinterpret_cast<const uint4*>(rows + (j - w) * 256 + cc16 * 16)
+                          : *reinterpret_cast<const uint4*>(halo + (cc & 1) * 768 + (3 + j - w) * 256 + cc16 * 16);
+        if (j >= kC - 3) *reinterpret_cast<uint4*>(halo + ((cc + 1) & 1) * 768 + (j - (kC - 3)) * 256 + cc16 * 16) = raw;
+        const uint4 y = pre::conv_norm_bf16x8_sw<kD, 16>(sconv, cc16 * 8, x);
+        return j < n ? y : make_uint4(0, 0, 0, 0);
+    };
     uint4 ra[2], rk[2];
     auto build_load = [&](int cc) {
         const int n = min(kC, T - cc * kC);
@@ -171,6 +197,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             const int j = cid >> 4, cc16 = cid & 15;
             ra[rep] = make_uint4(0, 0, 0, 0);
             if (j < n) ra[rep] = *reinterpret_cast<const uint4*>(rpa + j * 256 + cc16 * 16);
+            if (conv_k && !m) ra[rep] = preprocess_key(cc, n, j, cc16, rpa, ra[rep]);
             const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ra[rep]);
             float mx = 0.f;
 #pragma unroll
@@ -186,6 +213,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             if (m) {   // key rows: the B operand and the key row maxima for the value-state bound
                 rk[rep] = make_uint4(0, 0, 0, 0);
                 if (j < n) rk[rep] = *reinterpret_cast<const uint4*>(rpk + j * 256 + cc16 * 16);
+                if (conv_k) rk[rep] = preprocess_key(cc, n, j, cc16, rpk, rk[rep]);
                 const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&rk[rep]);
                 kmx = 0.f;
 #pragma unroll
@@ -202,21 +230,18 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         }
         wa = fmaxf(wa, __shfl_xor_sync(0xffffffffu, wa, 16));   // the warp's other row
         wk = fmaxf(wk, __shfl_xor_sync(0xffffffffu, wk, 16));
-        if (lane == 0) cmax[(cc & 1) * 16 + w] = make_float2(wa, wk);
+        if (lane == 0) {
+            atomicMax(cmax + 2 * (cc & 1), __float_as_int(wa));
+            atomicMax(cmax + 2 * (cc & 1) + 1, __float_as_int(wk));
+        }
     };
     auto build_store = [&](int cc) -> float {
         const float* swc = sw + (cc & 3) * kC;
         uint8_t* Ahi = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
         uint8_t* Alo = Ahi + 16384;
         uint8_t* Bk = Ahi + 32768;
-        float wa = 0.f, wk = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float2 c2 = cmax[(cc & 1) * 16 + i];
-            wa = fmaxf(wa, c2.x);
-            wk = fmaxf(wk, c2.y);
-        }
-        const float sA = pow2_ceil(wa), sK = pow2_ceil(wk);
+        const int2 c2 = *reinterpret_cast<const int2*>(cmax + 2 * (cc & 1));
+        const float sA = pow2_ceil(__int_as_float(c2.x)), sK = pow2_ceil(__int_as_float(c2.y));
         const float inv_sA = 1.f / sA, inv_sK = 1.f / sK;       // powers of two: exact
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
@@ -268,6 +293,11 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         mbar_init(bar_mma, 1);
         fence_mbar_init();
         red[31] = 0.f;
+    }
+    if (tid < 4) cmax[tid] = 0;
+    if (conv_k) {                                  // fused preprocessing: weights, zero rows before t = 0
+        pre::stage_weights<kD>(conv_k + (size_t)(bh % H) * conv_w * kD, conv_w, sconv);
+        for (int e = tid; e < 768 / 16; e += kScanThreads) reinterpret_cast<uint4*>(halo)[e] = make_uint4(0, 0, 0, 0);
     }
     if (w == 0) tmem_alloc(slot, 128);
     tc_fence_before();
@@ -337,6 +367,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid < 2) cmax[tid] = 0;               // buffer 0 is free for chunk 2
         if (tid == 0) {
             const size_t ci = image_index(bh, np, 0, m);
             bulk_s2g(img + ci * kImgHalves, stage, kImgBytes);
@@ -394,6 +425,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             break;
         }
         // ---- S <- e^{b_last} S + sA sK Delta ----
+        if (tid < 2) cmax[2 * ((c + 1) & 1) + tid] = 0;     // chunk c+1's images are written: free for c+3
         const float Gam = expf(blast);
         {
             float dv[32];
@@ -458,7 +490,7 @@ cudaError_t tc_scan_launch(const ForwardArgs& a, void* img, float* scales, unsig
     LaunchTimer timer(kKindTcScan, st);
     tc_scan_kernel<<<dim3(2, a.B * a.H), kScanThreads, smem, st>>>(
         static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.T, nc,
-        a.H_in, a.G_in, static_cast<__half*>(img), scales, a.H_out, a.G_out, err);
+        a.H_in, a.G_in, static_cast<__half*>(img), scales, a.H_out, a.G_out, err, a.conv_k, a.conv_w, a.H);
     return cudaGetLastError();
 }
 

@@ -67,6 +67,11 @@ def _load():
     lib.mesa_timing_read.restype = I
     lib.mesa_preprocess.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, P]
     lib.mesa_preprocess.restype = I
+    lib.mesa_forward_preprocessed.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
+                                              P, P, P, Z, P]
+    lib.mesa_forward_preprocessed.restype = I
+    lib.mesa_forward_preprocessed_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.mesa_forward_preprocessed_workspace_size.restype = Z
     lib.mesa_chunk_state_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.mesa_chunk_state_workspace_size.restype = Z
     lib.mesa_chunk_state.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, Z, P]
@@ -301,6 +306,43 @@ def preprocess(q_raw, k_raw, conv_q, conv_k, *, q_out=None, k_out=None, stream=N
                              _dtype_code(q_raw), _ptr(q_out), _ptr(k_out), _stream(stream, q_raw.device))
     _check(rc, "mesa_preprocess")
     return q_out, k_out
+
+
+def forward_preprocessed(q_raw, k_raw, v, gamma, beta, lam, conv_q, conv_k, *, chunk=64, cg_steps=15, tol=0.0,
+                         out=None, return_iters=False, iters=None, H_in=None, G_in=None, return_state=False,
+                         workspace=None, stream=None):
+    """forward() of preprocess(q_raw, k_raw, conv_q, conv_k) in one call
+    (mesa_forward_preprocessed): on the tensor-core shape the scan and the
+    solve convolve and normalise the raw rows as they stage them. Same
+    returns as forward()."""
+    lib = _load()
+    B, H, T, dk = q_raw.shape
+    dv = v.shape[-1]
+    W = conv_q.shape[1]
+    assert conv_q.shape == (H, W, dk) and conv_k.shape == (H, W, dk)
+    code = _dtype_code(q_raw)
+    dev = q_raw.device
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32, device=dev)
+    if return_iters and iters is None:
+        iters = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+    H_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev) if return_state else None
+    G_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev) if return_state else None
+    need = int(lib.mesa_forward_preprocessed_workspace_size(B, H, T, dk, dv, chunk, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.mesa_forward_preprocessed(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(lam),
+                                       _ptr(conv_q), _ptr(conv_k), W, B, H, T, dk, dv, chunk, code, int(cg_steps),
+                                       float(tol), _ptr(out), _ptr(iters), _ptr(H_in), _ptr(G_in), _ptr(H_out),
+                                       _ptr(G_out), _ptr(workspace), ws_bytes, _stream(stream, dev))
+    _check(rc, "mesa_forward_preprocessed")
+    res = (out,)
+    if return_iters:
+        res += (iters,)
+    if return_state:
+        res += (H_out, G_out)
+    return res[0] if len(res) == 1 else res
 
 
 def step(q, k, v, gamma, beta, lam, Hstate, Gstate, *, cg_steps=15, tol=0.0, out=None,

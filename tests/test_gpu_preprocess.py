@@ -99,3 +99,70 @@ def test_preprocess_full_size_sampled(mesa, oracle_mod):
             ref = oracle_mod.preprocess(raw[b:b + 1, h:h + 1].float().cpu().numpy(),
                                         c[h:h + 1].cpu().numpy())
             check(got[b:b + 1, h:h + 1].float().cpu().numpy(), ref, "bf16")
+
+
+# ---------------------------------------------------------------------------
+# mesa_forward_preprocessed: the preprocessing folded into the forward's own
+# staged loads (tensor-core shape) must give exactly the bits of the two-step
+# path, mesa_preprocess followed by mesa_forward.
+# ---------------------------------------------------------------------------
+
+def layer_inputs(B, H, T, d, seed, dtype):
+    w = mi.Workload("pre", B, H, T, d, d, 64, dtype, 15, 0.0, False, seed)
+    x = mi.batch(w)
+    rng = np.random.default_rng(seed + 1)
+    raw_q = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    raw_k = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    return x, raw_q, raw_k
+
+
+@pytest.mark.parametrize("T,W,tol", [(1, 4, 0.0), (3, 4, 0.0), (64, 2, 0.0), (65, 4, 0.0), (130, 3, 0.0),
+                                     (333, 4, 0.0), (700, 1, 0.0), (300, 4, 1e-3)])
+def test_fused_forward_equals_preprocess_then_forward(mesa, T, W, tol):
+    B, H, d = 2, 3, 128
+    x, rq, rk = layer_inputs(B, H, T, d, 90 + T, "bf16")
+    rng = np.random.default_rng(T)
+    cq = torch.from_numpy((rng.standard_normal((H, W, d)) / np.sqrt(W)).astype(np.float32)).cuda()
+    ck = torch.from_numpy((rng.standard_normal((H, W, d)) / np.sqrt(W)).astype(np.float32)).cuda()
+    q_raw, k_raw = on_device(rq, "bf16"), on_device(rk, "bf16")
+    v = on_device(x["v"], "bf16")
+    g, b = torch.from_numpy(x["gamma"]).cuda(), torch.from_numpy(x["beta"]).cuda()
+    lam = torch.from_numpy(x["lam"]).cuda()
+    q, k = mesa.preprocess(q_raw, k_raw, cq, ck)
+    ref, it_ref, H_ref, G_ref = mesa.forward(q, k, v, g, b, lam, chunk=64, cg_steps=30 if tol else 15, tol=tol,
+                                             return_iters=True, return_state=True)
+    out, it, H_o, G_o = mesa.forward_preprocessed(q_raw, k_raw, v, g, b, lam, cq, ck, chunk=64,
+                                                  cg_steps=30 if tol else 15, tol=tol, return_iters=True,
+                                                  return_state=True)
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    assert torch.equal(out, ref) and torch.equal(it, it_ref)
+    assert torch.equal(H_o, H_ref) and torch.equal(G_o, G_ref)
+
+
+@pytest.mark.parametrize("dtype,d,chunk", [("bf16", 128, 64), ("f32", 64, 16), ("bf16", 32, 32)])
+def test_fused_forward_matches_oracle(mesa, oracle_mod, dtype, d, chunk):
+    """Against the oracle's preprocessing followed by its CG forward (the other
+    shapes take the two-step path inside the same entry point)."""
+    B, H, T, W = 1, 2, 200, 4
+    x, rq, rk = layer_inputs(B, H, T, d, 97, dtype)
+    rng = np.random.default_rng(5)
+    cq = (rng.standard_normal((H, W, d)) / 2).astype(np.float32)
+    ck = (rng.standard_normal((H, W, d)) / 2).astype(np.float32)
+    q_raw, k_raw = on_device(rq, dtype), on_device(rk, dtype)
+    v = on_device(x["v"], dtype)
+    out = mesa.forward_preprocessed(q_raw, k_raw, v, torch.from_numpy(x["gamma"]).cuda(),
+                                    torch.from_numpy(x["beta"]).cuda(), torch.from_numpy(x["lam"]).cuda(),
+                                    torch.from_numpy(cq).cuda(), torch.from_numpy(ck).cuda(), chunk=chunk,
+                                    cg_steps=15)
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    # the oracle preprocesses the same raw values; the GPU's q and k are rounded
+    # to the input type after preprocessing, so the oracle sees that rounding too
+    pq = oracle_mod.preprocess(q_raw.float().cpu().numpy(), cq)
+    pk = oracle_mod.preprocess(k_raw.float().cpu().numpy(), ck)
+    if dtype == "bf16":
+        pq, pk = mi.bf16_round(pq.astype(np.float32)), mi.bf16_round(pk.astype(np.float32))
+    ref, _, _, _ = oracle_mod.forward_cg(pq, pk, v.float().cpu().numpy(), x["gamma"], x["beta"], x["lam"], 15)
+    tol = TOL_BF16 if dtype == "bf16" else 1e-4
+    assert rel_err(out.cpu().numpy(), ref) <= tol
