@@ -400,6 +400,98 @@ def run_preprocess(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_fused_preprocess(args, w, world, rank, local):
+    """The forward with the q/k preprocessing folded into its staged loads
+    (mesa_forward_preprocessed) on the workload, from raw q and k (window 4).
+    Also times, on the same inputs, the plain forward of already-preprocessed
+    q and k, and the two-step path (mesa_preprocess, then mesa_forward), so the
+    cost of the preprocessing inside the forward reads off directly."""
+    import torch
+    import torch.distributed as dist
+    from test_sequence_layer_b200 import build as mbuild, mesa
+    mbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    x = mi.device_batch(w, dev, seed_offset=rank)
+    B, H, T, d, C, W = w.B, w.H, w.T, w.dk, w.chunk, 4
+    g = torch.Generator(device=dev).manual_seed(5 + rank)
+    q_raw = torch.randn((B, H, T, d), generator=g, device=dev).to(x["q"].dtype)
+    k_raw = torch.randn((B, H, T, d), generator=g, device=dev).to(x["q"].dtype)
+    cq = torch.randn((H, W, d), generator=g, device=dev) / 2
+    ck = torch.randn((H, W, d), generator=g, device=dev) / 2
+    q_pre, k_pre = torch.empty_like(q_raw), torch.empty_like(k_raw)
+    out = torch.empty((B, H, T, d), device=dev)
+    ws = torch.empty(max(mesa.workspace_size(B, H, T, d, d, C, x["q"].dtype), 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(chunk=C, cg_steps=w.cg_steps, tol=w.tol, out=out, workspace=ws, stream=stream)
+
+    def fused():
+        mesa.forward_preprocessed(q_raw, k_raw, x["v"], x["gamma"], x["beta"], x["lam"], cq, ck, **kw)
+
+    def plain():
+        mesa.forward(q_pre, k_pre, x["v"], x["gamma"], x["beta"], x["lam"], **kw)
+
+    def two_step():
+        mesa.preprocess(q_raw, k_raw, cq, ck, q_out=q_pre, k_out=k_pre, stream=stream)
+        plain()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    mesa.timing_enable(True)
+    mesa.timing_read()
+    ms_two = timed(two_step)            # also leaves q_pre, k_pre for the plain forward
+    k_two = mesa.timing_read()
+    ms_plain = timed(plain)
+    k_plain = mesa.timing_read()
+    ms_fused = timed(fused)
+    kernels = mesa.timing_read()
+    mesa.timing_enable(False)
+    clk = clocks.stop()
+    assert mesa.get_error(stream) == 0
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    tokens = B * H * T
+    per = lambda ks: {k: {"launches": v[0], "total_ms": v[1]} for k, v in ks.items()}    # noqa: E731
+    line = {
+        "metric": "Mesa-layer fwd tokens/s (B*H*T) from raw q, k with the input preprocessing folded into the "
+                  "forward's loads",
+        "value": whole_job_rate(tokens, world, ms_fused), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_fused, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-in/f16-mma/f32-acc" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name + "+fused-preprocess", "B": B, "H": H, "T": T, "d": d, "chunk": C,
+                   "cg_steps": w.cg_steps, "window": W, "l2": "inputs larger than L2"},
+        "fused": {"ms_per_step": ms_fused, "kernels": per(kernels)},
+        "plain_forward": {"ms_per_step": ms_plain, "kernels": per(k_plain)},
+        "preprocess_then_forward": {"ms_per_step": ms_two, "kernels": per(k_two)},
+        "roofline": None, "gpu_launches": sum(v[0] for v in kernels.values()),
+        "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # Useful flops per token of each backward kernel (d, chunk C, N CG steps):
 # a CG matvec or a read-out-shaped product counts 2d^2 + 2d(C+1) (the causal
 # intra-chunk terms j <= t only), a chunk-state update 2 d^2 per matrix.
@@ -684,6 +776,8 @@ def main():
                     help="time mesa_preprocess (q/k convolution + normalisation) on the workload's shape")
     ap.add_argument("--backward", action="store_true",
                     help="time mesa_backward (implicit-differentiation gradients) on the workload's shape")
+    ap.add_argument("--fused-preprocess", action="store_true",
+                    help="time mesa_forward_preprocessed (raw q, k) against the plain and the two-step forward")
     ap.add_argument("--seq-sharded", action="store_true",
                     help="sequence-sharded forward: each rank one slice of T, one all-gather of slice states")
     ap.add_argument("--warm-start", action="store_true",
@@ -712,6 +806,9 @@ def main():
         return
     if args.backward:
         run_backward(args, w, world, rank, local)
+        return
+    if args.fused_preprocess:
+        run_fused_preprocess(args, w, world, rank, local)
         return
     if args.seq_sharded:
         run_seq_sharded(args, w, world, rank, local)
