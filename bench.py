@@ -205,7 +205,7 @@ def run_reference(args, w, rank):
 
 METRIC = "Mesa-layer fwd tokens/s (B*H*T) at T=8192,d=128,15 CG steps; % tensor peak"
 DECODE_METRIC = "Mesa decode tokens/s (sequences x heads per mesa_step), d=128, 15 CG steps; % HBM peak"
-BWD_METRIC = "Mesa-layer bwd tokens/s (B*H*T): implicit-differentiation backward, d=128, 15 CG steps; % fp32 FMA peak"
+BWD_METRIC = "Mesa-layer bwd tokens/s (B*H*T): implicit-differentiation backward, d=128, 15 CG steps; % of the dominant kernel's peak"
 PRE_METRIC = "Mesa input preprocessing tokens/s (q and k: causal depthwise conv, window 4, + L2 norm); % HBM peak"
 
 
@@ -495,10 +495,17 @@ def run_fused_preprocess(args, w, world, rank, local):
 # Useful flops per token of each backward kernel (d, chunk C, N CG steps):
 # a CG matvec or a read-out-shaped product counts 2d^2 + 2d(C+1) (the causal
 # intra-chunk terms j <= t only), a chunk-state update 2 d^2 per matrix.
-def bwd_flops_per_token(d, C, N):
+def bwd_flops_per_token(d, C, N, tc):
     mv = 2 * d * d + 2 * d * (C + 1)
-    return {"simt_scan": 4 * d * d, "simt_cg": N * mv, "bwd_adjoint": (N + 2) * mv,
-            "bwd_rscan": 4 * d * d, "bwd_grad": 8 * d * d + 8 * d * (C + 1)}
+    fl = {"simt_scan": 4 * d * d, "simt_cg": N * mv, "bwd_adjoint": (N + 2) * mv,
+          "bwd_rscan": 4 * d * d, "bwd_grad": 8 * d * d + 8 * d * (C + 1)}
+    if tc:    # tensor-core shape: the forward solve with its read-out, the right-hand sides, adjoint CG + H x
+        fl.update({"tc_scan": 4 * d * d, "tc_cg": (N + 1) * mv, "bwd_rhs": mv, "bwd_adjoint": (N + 1) * mv})
+        del fl["simt_scan"], fl["simt_cg"]
+    return fl
+
+
+BWD_TENSOR_KERNELS = ("tc_scan", "tc_cg", "bwd_rhs", "bwd_adjoint")
 
 
 def fp32_fma_peak_tflops(sm_mhz):
@@ -509,7 +516,9 @@ def fp32_fma_peak_tflops(sm_mhz):
 def run_backward(args, w, world, rank, local):
     """mesa_backward on the workload's shape with device-resident inputs and a
     seeded upstream gradient: forward solve, adjoint solve, reverse scan and
-    gradient kernels, all fp32 on the CUDA cores."""
+    gradient kernels. On the tensor-core shape the forward solve, the adjoint
+    right-hand sides and the adjoint solve run on tcgen05; the reverse scans
+    and gradient kernels are fp32 on the CUDA cores."""
     import torch
     import torch.distributed as dist
     from test_sequence_layer_b200 import build as mbuild, mesa
@@ -560,12 +569,15 @@ def run_backward(args, w, world, rank, local):
     if rank != 0:
         return
     tokens = w.B * w.H * w.T
-    fl = bwd_flops_per_token(w.dk, w.chunk, N)
+    tc = w.dtype == "bf16" and w.dk == 128 and w.dv == 128 and w.chunk == 64
+    fl = bwd_flops_per_token(w.dk, w.chunk, N, tc)
     top = max((k for k in kernels if k in fl), key=lambda k: kernels[k][1])
     launches, kms = kernels[top]
     avg_ms = kms / launches
     achieved = fl[top] * tokens / (avg_ms / 1e3) / 1e12
-    peak = fp32_fma_peak_tflops(1965.0)
+    on_tensor = tc and top in BWD_TENSOR_KERNELS
+    peaks = load_peaks()
+    peak = peaks["bf16_tflops"] if on_tensor else fp32_fma_peak_tflops(1965.0)
     line = {
         "metric": BWD_METRIC, "value": whole_job_rate(tokens, world, ms / args.steps), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -575,9 +587,11 @@ def run_backward(args, w, world, rank, local):
                    "cg_steps": N, "tol": w.tol, "flops_per_token": sum(fl.values()),
                    "l2": "inputs larger than L2 (%.2f GB per step)" % (
                        (3 * x["q"].numel() * x["q"].element_size() + do.numel() * 4) / 1e9)},
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": top, "avg_ms": avg_ms,
-                     "peak_kind": "derived fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz"},
+        "roofline": {"bound": "tensor" if on_tensor else "alu", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "kernel": top, "avg_ms": avg_ms,
+                     "peak_kind": (f"{peaks['_source']} bf16 dense burst (fp16 operands run at the bf16 rate)"
+                                   if on_tensor else
+                                   "derived fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz")},
         "kernels": {k: {"launches": v[0], "total_ms": v[1]} for k, v in kernels.items()},
         "gpu_launches": sum(v[0] for v in kernels.values()),
         "clocks": clk, "e2e": None, "cpu_baseline": None,

@@ -262,8 +262,13 @@ mesa_status mesa_forward_preprocessed(const void* q_raw, const void* k_raw, cons
  * When CG has converged this is the exact gradient of the layer.
  *
  *   q, k, v, gamma, beta, lambda, B, H, T, dk, dv, chunk, dtype, cg_steps,
- *                tol: as in mesa_forward (every supported shape and dtype;
- *                the arithmetic is fp32 on the CUDA cores for every dtype).
+ *                tol: as in mesa_forward (every supported shape and dtype).
+ *                On the tensor-core shape (MESA_BF16, dk = dv = 128,
+ *                chunk = 64) the forward solve, the right-hand sides
+ *                G_t^T dout_t and the adjoint solve run on the tensor cores
+ *                (fp16 operands, fp32 accumulation: the bf16-mode accuracy);
+ *                the reverse gradient scans and every other shape are fp32 on
+ *                the CUDA cores.
  *   dout         float32 [B,H,T,dv].
  *   dq, dk_out   float32 [B,H,T,dk];  dv_out float32 [B,H,T,dv].
  *   dgamma, dbeta float32 [B,H,T].    dlambda float32 [H,dk] (summed over

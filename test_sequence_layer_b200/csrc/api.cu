@@ -70,7 +70,7 @@ mesa_status launch_forward(const ForwardArgs& a, cudaStream_t st) {
 // ---- kernel timing records ----
 const char* const kKindNames[kKindCount] = {"simt_scan", "simt_cg", "decode_step", "tc_scan", "tc_cg",
                                              "preprocess", "bwd_adjoint", "bwd_rscan", "bwd_grad", "bwd_reduce",
-                                             "shard"};
+                                             "shard", "bwd_rhs"};
 struct TimingRec {
     int kind;
     cudaEvent_t start, stop;

@@ -56,7 +56,7 @@ unsigned* error_word_ptr();
 // Kernel kinds for the optional timing records (mesa_timing_enable).
 enum KernelKind : int {
     kKindSimtScan = 0, kKindSimtCg, kKindStep, kKindTcScan, kKindTcCg, kKindPre,
-    kKindBwdAdj, kKindBwdRscan, kKindBwdGrad, kKindBwdReduce, kKindShard, kKindCount
+    kKindBwdAdj, kKindBwdRscan, kKindBwdGrad, kKindBwdReduce, kKindShard, kKindBwdRhs, kKindCount
 };
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
@@ -91,6 +91,12 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st);
 // Chunk-state scan of the tensor-core forward: state images and scales into
 // img / scales (layout in tc_layout.cuh), final states into a.H_out / a.G_out.
 cudaError_t tc_scan_launch(const ForwardArgs& a, void* img, float* scales, unsigned* err, cudaStream_t st);
+// The backward's adjoint solve on the tensor cores, from the images a
+// forward_tc call left at the start of `images_ws`: the right-hand side
+// g_t = G_t^T dout_t (into rhs_buf), then u_t = CG(H_t + Lambda, g_t) into dq
+// and e_t = g_t . x_t - u_t . (H_t x_t) into zt.
+cudaError_t tc_adjoint(const ForwardArgs& f, const void* images_ws, const float* dout, const float* xsol,
+                       float* rhs_buf, float* dq, float* zt, cudaStream_t st);
 #ifdef MESA_DEBUG
 // The next `launches` launches of the tensor-core solve kernel leave out the
 // completion signal of their first Z product (fault injection, debug builds).

@@ -28,10 +28,12 @@
 // Kernels (all fp32, 256 threads, thread layout of simt_chunk.cuh):
 //   the forward solutions x_t: the fp32 scan + CG of simt_forward.cu, or,
 //                     for bf16 inputs at d = 128, C = 64, the tensor-core
-//                     scan and solve (x stored in fp32) next to the fp32 scan
-//                     alone for the chunk states;
+//                     scan and solve (x stored in fp32);
 //   simt_adj_kernel   grid (chunks, B*H): right-hand side G_t^T do_t, the
-//                     adjoint CG, H_t x_t, then dq, e_t and per-chunk dlambda sums;
+//                     adjoint CG, H_t x_t, then dq, e_t and per-chunk dlambda
+//                     sums; for bf16 inputs at d = 128, C = 64 the same on the
+//                     tensor cores instead (tc_adjoint in tc_forward.cu, from
+//                     the forward's state images) and dlambda_part_kernel;
 //   simt_rscan_kernel grid (64 x 64 state tiles, B*H): the reverse chunk scan of
 //                     Hhat_c and Ghat_c;
 //   simt_grad_kernel  grid (chunks, B*H): dk, dv, dbeta and z_t;
@@ -517,6 +519,23 @@ __global__ void __launch_bounds__(256) dgamma_kernel(const float* __restrict__ z
 }
 
 // dlambda[h][i] = sum over batch rows b, then chunks c, of the chunk partials.
+// Per-chunk sums -sum_{t in c} u_ti x_ti of the dlambda partials from u (dq)
+// and x, one block per (chunk, b*h) and one thread per key channel, in token
+// order: the layout simt_adj_kernel writes, for dlambda_kernel.
+__global__ void dlambda_part_kernel(const float* __restrict__ u, const float* __restrict__ x, int T, int chunk,
+                                    int nc, int dk, float* __restrict__ part) {
+    const int c = blockIdx.x, bh = blockIdx.y;
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        const int t0 = c * chunk, t1 = min(T, t0 + chunk);
+        float s = 0.f;
+        for (int t = t0; t < t1; ++t) {
+            const size_t e = ((size_t)bh * T + t) * dk + i;
+            s = fmaf(-u[e], x[e], s);
+        }
+        part[((size_t)bh * nc + c) * dk + i] = s;
+    }
+}
+
 __global__ void dlambda_kernel(const float* __restrict__ part, int B, int H, int nc, int dk,
                                float* __restrict__ dlambda) {
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -540,8 +559,8 @@ BwdLayout bwd_layout(int B, int H, int T, int dk, int dv, int chunk, mesa_dtype 
     const size_t BH = (size_t)B * H;
     const size_t se = nc * ((size_t)dk * dk + (size_t)dv * dk) * sizeof(float);
     BwdLayout l;
-    l.states = 0;
-    l.x = l.states + up(BH * se);
+    l.states = 0;                      // fp32 chunk-start states: the CUDA-core adjoint only
+    l.x = l.states + (tc_supported(dk, dv, chunk, dtype) ? 0 : up(BH * se));
     l.z = l.x + up(BH * T * dk * sizeof(float));
     l.rstates = l.z + up(BH * T * sizeof(float));
     l.part = l.rstates + up(BH * se);
@@ -568,7 +587,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
     float* R = reinterpret_cast<float*>(ws + l.rstates);
     float* part = reinterpret_cast<float*>(ws + l.part);
 
-    // forward: fp32 chunk-start states and the solutions x_t
+    // forward: the solutions x_t (and whatever chunk states the adjoint reads)
     ForwardArgs fa = f;
     fa.out = nullptr;
     fa.iters = nullptr;
@@ -578,23 +597,26 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
     fa.x_out = X;
     cudaError_t e;
     if (tc_supported(f.dk, f.dv, f.chunk, f.dtype)) {
-        // bf16 inputs at d = 128, C = 64: x from the tensor-core solve (the
-        // bf16-mode precision), the fp32 states from the scan alone
+        // bf16 inputs at d = 128, C = 64, all on the tensor cores (the
+        // bf16-mode precision): the scan and solve give x and leave their
+        // fp16 state images in the workspace; the adjoint reads those
+        // images, so no fp32 states are formed. The read-out buffer, which
+        // the backward does not need, holds g_t = G_t^T dout_t.
         ForwardArgs ft = fa;
         ft.workspace = ws + l.tcws;
         ft.ws_bytes = l.oscr - l.tcws;
-        ft.out = reinterpret_cast<float*>(ws + l.oscr);
+        float* scratch = reinterpret_cast<float*>(ws + l.oscr);
+        ft.out = scratch;
         if ((e = forward_tc(ft, st)) != cudaSuccess) return e;
-        fa.scan_only = true;
-        fa.x_out = nullptr;
-    }
-    if ((e = forward_simt(fa, st)) != cudaSuccess) return e;
-
-    using L = CgSmem<D, D, CH>;
-    auto adj = simt_adj_kernel<D, D, CH, Tin>;
-    e = cudaFuncSetAttribute(adj, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
-    if (e != cudaSuccess) return e;
-    {
+        if ((e = tc_adjoint(f, ws + l.tcws, a.dout, X, scratch, a.dq, Z, st)) != cudaSuccess) return e;
+        LaunchTimer timer(kKindBwdReduce, st);
+        dlambda_part_kernel<<<dim3(nc, BH), 128, 0, st>>>(a.dq, X, f.T, CH, nc, D, part);
+    } else {
+        if ((e = forward_simt(fa, st)) != cudaSuccess) return e;
+        using L = CgSmem<D, D, CH>;
+        auto adj = simt_adj_kernel<D, D, CH, Tin>;
+        e = cudaFuncSetAttribute(adj, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+        if (e != cudaSuccess) return e;
         LaunchTimer timer(kKindBwdAdj, st);
         adj<<<dim3(nc, BH), kThreads, L::bytes, st>>>(
             static_cast<const Tin*>(f.k), static_cast<const Tin*>(f.v), f.gamma, f.beta, f.lambda, a.dout, X, f.H,

@@ -103,7 +103,8 @@ struct BlkSmem {
     static constexpr int oConvQ = oConvK + 2048;
     static constexpr int oHaloK = oConvQ + 2048;  // and the 3 raw key and query rows before the block
     static constexpr int oHaloQ = oHaloK + 768;
-    static constexpr int bytes = oHaloQ + 768;
+    static constexpr int oGx = oHaloQ + 768;      // adjoint: g_t . x_t per token [128]
+    static constexpr int bytes = oGx + 512;
 };
 
 // b[t], t < 128: cumulative sum of log gamma over positions 0..t of the first
@@ -170,6 +171,12 @@ __device__ __forceinline__ void issue_k128(uint32_t d, uint32_t a, uint32_t b, u
     }
 }
 
+// kAdj = false: the forward (right-hand side q, read-out o = G x).
+// kAdj = true: the adjoint solve of the backward, (H_t + Lambda) u_t = g_t with
+// g_t = G_t^T dout_t read from `rhs` (fp32, tc_rhs_kernel) under the same CG
+// rule; writes dq_t = u_t and e_t = g_t . x_t - u_t . (H_t x_t), with x_t the
+// forward's solutions (`xsol`) and H_t x_t one more product of the same kind.
+template <bool kAdj>
 __global__ void __launch_bounds__(kBlkThreads, 1)
 tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
              const __nv_bfloat16* __restrict__ v, const float* __restrict__ gamma,
@@ -177,7 +184,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
              int cg_steps, float tol, const __half* __restrict__ img, const float* __restrict__ scales,
              float* __restrict__ out, int32_t* __restrict__ iters, unsigned* __restrict__ err,
              float* __restrict__ x_out, const float* __restrict__ x0, const float* __restrict__ conv_q,
-             const float* __restrict__ conv_k, int conv_w) {
+             const float* __restrict__ conv_k, int conv_w, const float* __restrict__ rhs,
+             const float* __restrict__ xsol, float* __restrict__ dq, float* __restrict__ zt) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Hs = smem + BlkSmem::oH;
@@ -256,9 +264,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     const bool fuse = conv_k != nullptr;
     const bool halo_rows = fuse && t0 >= pre::kMaxW - 1;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u) + (halo_rows ? 2u * 768u : 0u));
+        mbar_arrive_expect_tx(bar_in, (kAdj ? 1u : 2u) * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u) +
+                                          (halo_rows ? 2u * 768u : 0u));
         bulk_g2s(Ps, k + base * kD, row_bytes, bar_in);
-        bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
+        if (!kAdj) bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
         if (gates_bulk) {
             bulk_g2s(gstage, gamma + base, kBlk * 4, bar_in);
             bulk_g2s(gstage + kBlk, beta + base, kBlk * 4, bar_in);
@@ -280,8 +289,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         if (!mbar_wait(bar_in, 0)) *abort_flag = 1.f;
         mbar_arrive_expect_tx(bar_ld, kImgBytes);
         bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
-        mbar_arrive_expect_tx(bar_g, kImgBytes);
-        bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
+        if (!kAdj) {                                   // the adjoint has no read-out
+            mbar_arrive_expect_tx(bar_g, kImgBytes);
+            bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
+        }
     }
     __syncthreads();
 
@@ -348,14 +359,38 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         __syncthreads();
     }
     // CG state: x = 0 and r = q in TMEM, p = q in registers; this thread: token tok, columns col0..col0+31
+    // (the adjoint: r = p = g_t from rhs, and the partial g_t . x_t for e_t)
     float2 p[16];
+    float gx = 0.f;
+    if constexpr (kAdj) {
+        float2 acc = make_float2(0.f, 0.f);
+        if (valid) {
+            const float4* gr = reinterpret_cast<const float4*>(rhs + (base + tok) * kD + col0);
+            const float4* xr = reinterpret_cast<const float4*>(xsol + (base + tok) * kD + col0);
+#pragma unroll 1
+            for (int g = 0; g < 8; ++g) {
+                const float4 f = gr[g], xf = xr[g];
+                acc = __ffma2_rn(make_float2(f.x, f.y), make_float2(xf.x, xf.y), acc);
+                acc = __ffma2_rn(make_float2(f.z, f.w), make_float2(xf.z, xf.w), acc);
+            }
+        }
+        gx = acc.x + acc.y;
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (valid) raw = *reinterpret_cast<const uint4*>(Ws + tok * 256 + (col0 + 8 * g) * 2);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        for (int g = 0; g < 8; ++g) {
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (valid) f = reinterpret_cast<const float4*>(rhs + (base + tok) * kD + col0)[g];
+            p[2 * g] = make_float2(f.x, f.y);
+            p[2 * g + 1] = make_float2(f.z, f.w);
+        }
+    } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) p[4 * g + i] = __bfloat1622float2(b2[i]);
+        for (int g = 0; g < 4; ++g) {
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (valid) raw = *reinterpret_cast<const uint4*>(Ws + tok * 256 + (col0 + 8 * g) * 2);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) p[4 * g + i] = __bfloat1622float2(b2[i]);
+        }
     }
     // r = q; x = x0 (a warm start) or 0. With x0, p = x0 for the extra first
     // step that forms r = q - (H_t + Lambda) x0 (below).
@@ -430,9 +465,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) a = __ffma2_rn(p[i], p[i], a);
-        const float4 d = quarter_sum(make_float4(qq, a.x + a.y, 0.f, 0.f), red, cq, tok);   // barrier publishes seb, Mk
+        const float4 d = quarter_sum(make_float4(qq, a.x + a.y, gx, 0.f), red, cq, tok);   // barrier publishes seb, Mk
         rr = d.x;                                      // |q|^2 = |r|^2
         pp = d.y;                                      // |p|^2 (|x0|^2 for a warm start)
+        if (kAdj && cq == 0) reinterpret_cast<float*>(smem + BlkSmem::oGx)[tok] = d.z;   // adjoint: g_t . x_t
     }
     tmem_wait_st();
     const float qn = sqrtf(rr);
@@ -521,7 +557,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         // with a fixed step count the last U product is known: H is dead from
         // here, and the read-out's value rows can be on their way during this
         // step's CUDA-core work
-        if (tid == 0 && tol <= 0.f && step == cg_steps - 1) fetch_values();
+        if (!kAdj && tid == 0 && tol <= 0.f && step == cg_steps - 1) fetch_values();
 
         // y = s (sH e^b U + sW Z) + lambda p (written over Z); partials p.y, r.y, y.y, r.r
         const float c_u = s * sH * eb, c_z = s * sW;
@@ -610,79 +646,450 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tmem_wait_st();
     }
 
-    // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern,
-    // with X-hat = x / |x|, V / sV (sV >= max |v|) and the same key and mask images ----
-    // unless the last fixed step already sent them (the loop ran to its end)
-    const bool v_sent = tol <= 0.f && step == cg_steps && cg_steps > first_step;
-    if (tid == 0 && !v_sent) fetch_values();          // while x is normalised
-    __syncthreads();                                   // last reduction's readers are done with red[]
-    float xs;
-    {
-        float2 xr[16];
+    if constexpr (kAdj) {
+        // ---- adjoint tail: dq = u, then H_t x_t by one more product with
+        // X-hat = x / s_x, and e_t = g_t . x_t - u_t . (H_t x_t) ----
+        __syncthreads();                               // last reduction's readers are done with red[]
+        float ux_part = 0.f;
+        {
+            float2 xr[16];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            float xv[16];
-            tmem_ld32_x16(tl + kColX + col0 + 16 * h2, xv);
+            for (int g = 0; g < 8; ++g) {
+                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (valid) f = reinterpret_cast<const float4*>(xsol + (base + tok) * kD + col0)[g];
+                xr[2 * g] = make_float2(f.x, f.y);
+                xr[2 * g + 1] = make_float2(f.z, f.w);
+            }
+            float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
+            ux_part = a.x + a.y;
+            const float xx = quarter_sum(make_float4(ux_part, 0.f, 0.f, 0.f), red, cq, tok).x;
+            s = pow2_sqrt_scale(xx);
+            store_row32(Ps, tok, col0, xr, 1.f / s);
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {               // dq = u
+            float uv[16];
+            tmem_ld32_x16(tl + kColX + col0 + 16 * h2, uv);
             tmem_wait_ld();
+            if (valid) {
+                float4* dst = reinterpret_cast<float4*>(dq + (base + tok) * kD + col0 + 16 * h2);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) xr[8 * h2 + i] = make_float2(xv[2 * i], xv[2 * i + 1]);
+                for (int i = 0; i < 4; ++i) dst[i] = make_float4(uv[4 * i], uv[4 * i + 1], uv[4 * i + 2], uv[4 * i + 3]);
+            }
         }
-        if (x_out && valid) {                          // the solutions themselves, when asked for (fp32)
-            float4* dst = reinterpret_cast<float4*>(x_out + (base + tok) * kD + col0);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(xr[2 * i].x, xr[2 * i].y, xr[2 * i + 1].x, xr[2 * i + 1].y);
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        bool ok = *abort_flag == 0.f;
+        if (ok) {
+            if (tid == kIssuer) {
+                issue_S();
+                mma_commit(bar_s);
+                issue_U();
+                mma_commit(bar_u);
+            }
+            wait_mma_each(bar_s, ph & 1, abort_flag);
+            masked_scores();
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            ok = *abort_flag == 0.f;
         }
-        float2 a = make_float2(0.f, 0.f);
+        if (ok) {
+            if (tid == kIssuer) {
+                issue_Z();
+                mma_commit(bar_z);
+            }
+            wait_mma_each(bar_u, ph & 1, abort_flag);
+            wait_mma_each(bar_z, ph & 1, abort_flag);
+            ++ph;
+            // H_t x_t = s_x (sH e^b U + sW Z) (no Lambda term); the partial u . (H_t x_t)
+            const float c_u = s * sH * eb, c_z = s * sW;
+            float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
-        const float xx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;
-        xs = xx > 0.f ? sqrtf(xx) : 1.f;
-        store_row32(Ps, tok, col0, xr, 1.f / xs);
+            for (int h2 = 0; h2 < 4; ++h2) {
+                float uv[8], zv[8], xv[8];
+                tmem_ld32_x8(tl + kColU + col0 + 8 * h2, uv);
+                tmem_ld32_x8(tl + kColS + col0 + 8 * h2, zv);
+                tmem_ld32_x8(tl + kColX + col0 + 8 * h2, xv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float2 hx = __fmul2_rn(make_float2(uv[2 * i], uv[2 * i + 1]), make_float2(c_u, c_u));
+                    hx = __ffma2_rn(make_float2(zv[2 * i], zv[2 * i + 1]), make_float2(c_z, c_z), hx);
+                    a = __ffma2_rn(make_float2(xv[2 * i], xv[2 * i + 1]), hx, a);
+                }
+            }
+            const float uhx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;
+            if (cq == 0 && valid) zt[base + tok] = reinterpret_cast<const float*>(smem + BlkSmem::oGx)[tok] - uhx;
+            if (iters && cq == 0 && valid) iters[base + tok] = it;
+            ok = *abort_flag == 0.f;
+        }
+        if (!ok && tid == kIssuer) {
+            record_error(err, kErrTimeout);
+            // one more bounded chance for every MMA issued so far to drain
+            mma_commit(bar_ld);
+            mbar_wait(bar_ld, 0);
+            mbar_wait(bar_ld, 1);
+        }
+    } else {
+        // ---- read-out: o = e^{b_t} G_c x + (M o X K^T) V, on the same MMA pattern,
+        // with X-hat = x / |x|, V / sV (sV >= max |v|) and the same key and mask images ----
+        // unless the last fixed step already sent them (the loop ran to its end)
+        const bool v_sent = tol <= 0.f && step == cg_steps && cg_steps > first_step;
+        if (tid == 0 && !v_sent) fetch_values();          // while x is normalised
+        __syncthreads();                                   // last reduction's readers are done with red[]
+        float xs;
+        {
+            float2 xr[16];
+    #pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                float xv[16];
+                tmem_ld32_x16(tl + kColX + col0 + 16 * h2, xv);
+                tmem_wait_ld();
+    #pragma unroll
+                for (int i = 0; i < 8; ++i) xr[8 * h2 + i] = make_float2(xv[2 * i], xv[2 * i + 1]);
+            }
+            if (x_out && valid) {                          // the solutions themselves, when asked for (fp32)
+                float4* dst = reinterpret_cast<float4*>(x_out + (base + tok) * kD + col0);
+    #pragma unroll
+                for (int i = 0; i < 8; ++i) dst[i] = make_float4(xr[2 * i].x, xr[2 * i].y, xr[2 * i + 1].x, xr[2 * i + 1].y);
+            }
+            float2 a = make_float2(0.f, 0.f);
+    #pragma unroll
+            for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
+            const float xx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;
+            xs = xx > 0.f ? sqrtf(xx) : 1.f;
+            store_row32(Ps, tok, col0, xr, 1.f / xs);
+        }
+        // values of the block (kept in registers until the key image is free) and max |v|
+        if (!mbar_wait(bar_v, 0)) *abort_flag = 1.f;
+        uint4 vraw[4];
+        float vmax = 0.f;
+    #pragma unroll
+        for (int rep = 0; rep < 4; ++rep) {
+            const int cid = tid + kBlkThreads * rep;
+            const int j = cid >> 4, cc = cid & 15;
+            vraw[rep] = make_uint4(0, 0, 0, 0);
+            if (j < n) vraw[rep] = *reinterpret_cast<const uint4*>(Hs + j * 256 + cc * 16);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[rep]);
+    #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b2[i]);
+                vmax = fmaxf(vmax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+    #pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+        if (lane == 0) misc[w] = vmax;
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();                                   // publishes X-hat and misc
+        tc_fence_after();
+        float vm = misc[0];
+    #pragma unroll
+        for (int i = 1; i < 16; ++i) vm = fmaxf(vm, misc[i]);
+        const float sV = pow2_ceil(vm);
+        const float sG = scales[iG];
+        bool ok = *abort_flag == 0.f;
+        if (ok) {
+            if (tid == kIssuer) {
+                issue_S();                         // S' = X-hat K^T
+                mma_commit(bar_s);
+            }
+            wait_mma_each(bar_s, ph & 1, abort_flag);
+            masked_scores();                       // W' = (M sK^2 / sW) o (X-hat (K / sK)^T)
+            const float inv_sV = 1.f / sV;
+    #pragma unroll
+            for (int rep = 0; rep < 4; ++rep) {    // the key image is dead: values take its place
+                const int cid = tid + kBlkThreads * rep;
+                const int j = cid >> 4, cc = cid & 15;
+                *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
+                    bf16x8_to_f16x8(vraw[rep], inv_sV);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            ok = *abort_flag == 0.f;
+        }
+        if (ok) {
+            if (tid == kIssuer) {
+                if (!mbar_wait(bar_g, 0)) {
+                    *abort_flag = 1.f;
+                    mma_commit(bar_u);
+                    mma_commit(bar_z);
+                } else {
+                    issue_k128(tbase + kColU, smem_addr(Ps), smem_addr(Gs), 16, 16384, 16384, 32, kIdKK);   // U' = X-hat G^T
+                    mma_commit(bar_u);
+                    issue_Z();                     // Z' = W' V
+                    mma_commit(bar_z);
+                }
+            }
+            wait_mma_each(bar_u, ph & 1, abort_flag);
+            wait_mma_each(bar_z, ph & 1, abort_flag);
+            ++ph;
+            __syncthreads();
+            ok = *abort_flag == 0.f;
+        }
+        if (ok) {
+            // G x = xs sG U';  sum_j M_tj (x.k_j) v_j = xs sV sW / sK Z'
+            const float cu = xs * sG * eb, cz = xs * sV * sW / sK;
+    #pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                float uv[16], zv[16];
+                tmem_ld32_x16(tl + kColU + col0 + 16 * h2, uv);
+                tmem_ld32_x16(tl + kColS + col0 + 16 * h2, zv);
+                tmem_wait_ld();
+                if (valid) {
+                    float4* dst = reinterpret_cast<float4*>(out + (base + tok) * kD + col0 + 16 * h2);
+    #pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_float4(fmaf(uv[4 * i], cu, zv[4 * i] * cz), fmaf(uv[4 * i + 1], cu, zv[4 * i + 1] * cz),
+                                             fmaf(uv[4 * i + 2], cu, zv[4 * i + 2] * cz),
+                                             fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
+                }
+            }
+            if (iters && cq == 0 && valid) iters[base + tok] = it;
+        } else if (tid == kIssuer) {
+            record_error(err, kErrTimeout);
+            // one more bounded chance for every MMA issued so far to drain
+            mma_commit(bar_ld);
+            mbar_wait(bar_ld, 0);
+            mbar_wait(bar_ld, 1);
+            mbar_wait(bar_g, 0);
+        }
     }
-    // values of the block (kept in registers until the key image is free) and max |v|
-    if (!mbar_wait(bar_v, 0)) *abort_flag = 1.f;
-    uint4 vraw[4];
-    float vmax = 0.f;
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tbase, 512);
+}
+
+// =====================================================================
+// Right-hand side of the adjoint solve, 128 tokens per CTA
+// =====================================================================
+// g_t = G_t^T dout_t for every token of the block, in the chunk form of the
+// read-out with the roles of the two factors swapped:
+//     g_t = e^{b_t} G_c^T dout_t + sum_{j <= t} M_tj (dout_t . v_j) k_j.
+// Images: D = dout_t / s_t (per-token power of two), V / sV, K / sK, the mask
+// M sK^2 / sW as in the solve, and the G image read MN-major (its rows are
+// the value index). Products: S = D V^T, W = mask o S, U = D G, Z = W K, so
+//     g_t = s_t (sG e^{b_t} U_t + sW sV / sK Z_t).
+__global__ void __launch_bounds__(kBlkThreads, 1)
+tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+              const float* __restrict__ gamma, const float* __restrict__ beta, const float* __restrict__ dout,
+              int T, int np, const __half* __restrict__ img, const float* __restrict__ scales,
+              float* __restrict__ rhs, unsigned* __restrict__ err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* Vr = smem + BlkSmem::oH;             // raw value rows
+    uint8_t* Ks = smem + BlkSmem::oK;             // key image
+    uint8_t* Ds = smem + BlkSmem::oP;             // raw key rows, then the dout image
+    uint8_t* Ws = smem + BlkSmem::oW;             // value image, then the masked scores
+    uint8_t* Gs = smem + BlkSmem::oG;             // value-state image
+    __half* Mk = reinterpret_cast<__half*>(smem + BlkSmem::oM);
+    float* seb = reinterpret_cast<float*>(smem + BlkSmem::oEb);
+    float* sbc = reinterpret_cast<float*>(smem + BlkSmem::oB);
+    float* sbeta = reinterpret_cast<float*>(smem + BlkSmem::oBeta);
+    float4* red = reinterpret_cast<float4*>(smem + BlkSmem::oRed);
+    float* misc = reinterpret_cast<float*>(smem + BlkSmem::oMisc);
+    float* abort_flag = misc + 31;
+    uint64_t* bar_in = reinterpret_cast<uint64_t*>(smem + BlkSmem::oBar);
+    uint64_t* bar_g = bar_in + 1;
+    uint64_t* bar_s = bar_in + 2;
+    uint64_t* bar_u = bar_in + 3;
+    uint64_t* bar_z = bar_in + 4;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + BlkSmem::oSlot);
+
+    const int blk = blockIdx.x, bh = blockIdx.y;
+    const int t0 = blk * kBlk;
+    const int n = min(kBlk, T - t0);
+    const size_t base = (size_t)bh * T + t0;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int q4 = w & 3, cq = w >> 2;
+    const int tok = 32 * q4 + lane;
+    const bool valid = tok < n;
+    constexpr int kIssuer = 256;
+    const int col0 = 32 * cq;
+    const size_t iG = image_index(bh, np, blk, 1);
+
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_g, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_u, 1);
+        mbar_init(bar_z, 1);
+        fence_mbar_init();
+        *abort_flag = 0.f;
+        misc[20] = 0.f;                                // max |v| (as int bits, atomicMax)
+    }
+    if (w == 0) tmem_alloc(slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *slot;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
+    constexpr uint32_t kColU = 0, kColS = 128;
+
+    const uint32_t row_bytes = (uint32_t)n * kD * 2;
+    float* gstage = reinterpret_cast<float*>(red);
+    const bool gates_bulk = n == kBlk && ((reinterpret_cast<uintptr_t>(gamma + base) |
+                                            reinterpret_cast<uintptr_t>(beta + base)) & 15) == 0;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u));
+        bulk_g2s(Ds, k + base * kD, row_bytes, bar_in);
+        bulk_g2s(Vr, v + base * kD, row_bytes, bar_in);
+        if (gates_bulk) {
+            bulk_g2s(gstage, gamma + base, kBlk * 4, bar_in);
+            bulk_g2s(gstage + kBlk, beta + base, kBlk * 4, bar_in);
+        }
+        mbar_arrive_expect_tx(bar_g, kImgBytes);
+        bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
+    }
+    // this thread's token row of dout (32 columns, fp32) while the copies run
+    float2 dd[16];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) f = reinterpret_cast<const float4*>(dout + (base + tok) * kD + col0)[g];
+        dd[2 * g] = make_float2(f.x, f.y);
+        dd[2 * g + 1] = make_float2(f.z, f.w);
+    }
+    if (tid == 0 && !mbar_wait(bar_in, 0)) *abort_flag = 1.f;
+    __syncthreads();
+
+    // gates, beta, the raw key and value rows and their maxima
+    if (w == 0) warp_gate_cumsum128(gates_bulk ? gstage : gamma + base, n, sbc);
+    float bmax = 0.f, kmax = 0.f, vmax = 0.f;
+    if (tid < kBlk) {
+        bmax = (tid < n) ? (gates_bulk ? gstage[kBlk + tid] : beta[base + tid]) : 0.f;
+        sbeta[tid] = bmax;
+    }
+    uint4 kraw[4], vraw[4];
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
         const int cid = tid + kBlkThreads * rep;
         const int j = cid >> 4, cc = cid & 15;
-        vraw[rep] = make_uint4(0, 0, 0, 0);
-        if (j < n) vraw[rep] = *reinterpret_cast<const uint4*>(Hs + j * 256 + cc * 16);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[rep]);
+        kraw[rep] = vraw[rep] = make_uint4(0, 0, 0, 0);
+        if (j < n) {
+            kraw[rep] = *reinterpret_cast<const uint4*>(Ds + j * 256 + cc * 16);
+            vraw[rep] = *reinterpret_cast<const uint4*>(Vr + j * 256 + cc * 16);
+        }
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[rep]);
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[rep]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(b2[i]);
-            vmax = fmaxf(vmax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            const float2 fk = __bfloat1622float2(k2[i]), fv = __bfloat1622float2(v2[i]);
+            kmax = fmaxf(kmax, fmaxf(fabsf(fk.x), fabsf(fk.y)));
+            vmax = fmaxf(vmax, fmaxf(fabsf(fv.x), fabsf(fv.y)));
         }
     }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
-    if (lane == 0) misc[w] = vmax;
+    for (int off = 16; off >= 1; off >>= 1) {
+        kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    }
+    if (lane == 0) {
+        misc[w] = kmax;
+        if (w < 4) misc[16 + w] = bmax;
+        atomicMax(reinterpret_cast<int*>(misc + 20), __float_as_int(vmax));
+    }
+    __syncthreads();                                   // maxima visible; raw key rows read
+    float sK, sW, sV;
+    {
+        float km = misc[0], bm = misc[16];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) km = fmaxf(km, misc[i]);
+#pragma unroll
+        for (int i = 17; i < 20; ++i) bm = fmaxf(bm, misc[i]);
+        sK = pow2_ceil(km);
+        sW = pow2_ceil(bm * sK * sK);
+        sV = pow2_ceil(misc[20]);
+        const float inv_sK = 1.f / sK, inv_sV = 1.f / sV;
+#pragma unroll
+        for (int rep = 0; rep < 4; ++rep) {            // key image K / sK and value image V / sV (K-major)
+            const int cid = tid + kBlkThreads * rep;
+            const int j = cid >> 4, cc = cid & 15;
+            const uint32_t off = (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4);
+            *reinterpret_cast<uint4*>(Ks + off) = bf16x8_to_f16x8(kraw[rep], inv_sK);
+            *reinterpret_cast<uint4*>(Ws + off) = bf16x8_to_f16x8(vraw[rep], inv_sV);
+        }
+    }
+    if (tid < kBlk) seb[tid] = expf(sbc[tid]);
+    {
+        const float msc = sK * sK / sW;
+        for (int e = tid; e < kBlk * kBlk / 2; e += kBlkThreads) {
+            const int tt = e >> 6, j = 2 * (e & 63);
+            float m0 = 0.f, m1 = 0.f;
+            if (tt < n) {
+                const float bt = sbc[tt];
+                if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * msc;
+                if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * msc;
+            }
+            *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
+        }
+    }
+    // the dout image D = dout_t / s_t (the raw key rows in this buffer are consumed)
+    float sd;
+    {
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = __ffma2_rn(dd[i], dd[i], a);
+        const float dn = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;   // publishes seb, Mk
+        sd = pow2_sqrt_scale(dn);
+        store_row32(Ds, tok, col0, dd, 1.f / sd);
+    }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();                                   // publishes X-hat and misc
+    __syncthreads();
     tc_fence_after();
-    float vm = misc[0];
-#pragma unroll
-    for (int i = 1; i < 16; ++i) vm = fmaxf(vm, misc[i]);
-    const float sV = pow2_ceil(vm);
-    const float sG = scales[iG];
+
+    constexpr uint32_t kIdKK = idesc_f16(128, 128, false, false);
+    constexpr uint32_t kIdKM = idesc_f16(128, 128, false, true);
     bool ok = *abort_flag == 0.f;
     if (ok) {
         if (tid == kIssuer) {
-            issue_S();                         // S' = X-hat K^T
+            issue_k128(tbase + kColS, smem_addr(Ds), smem_addr(Ws), 16, 16384, 16384, 32, kIdKK);   // S = D V^T
             mma_commit(bar_s);
+            if (!mbar_wait(bar_g, 0)) {
+                *abort_flag = 1.f;
+            } else {
+                issue_k128(tbase + kColU, smem_addr(Ds), smem_addr(Gs), 16384, 16384, 8192, 2048, kIdKM);   // U = D G
+            }
+            mma_commit(bar_u);
         }
-        wait_mma_each(bar_s, ph & 1, abort_flag);
-        masked_scores();                       // W' = (M sK^2 / sW) o (X-hat (K / sK)^T)
-        const float inv_sV = 1.f / sV;
+        wait_mma_each(bar_s, 0, abort_flag);
+        // masked scores over the value image (S is complete, so V is dead); the
+        // quarter of tokens 0..63 against keys 64..127 is written as zeros
+        {
+            const bool zero_blk = q4 < 2 && cq >= 2;
+            const __half* mrow = Mk + tok * BlkSmem::kMS + col0;
+            float2 wv[16];
 #pragma unroll
-        for (int rep = 0; rep < 4; ++rep) {    // the key image is dead: values take its place
-            const int cid = tid + kBlkThreads * rep;
-            const int j = cid >> 4, cc = cid & 15;
-            *reinterpret_cast<uint4*>(Ks + (cc >> 3) * 16384 + j * 128 + (((cc & 7) ^ (j & 7)) << 4)) =
-                bf16x8_to_f16x8(vraw[rep], inv_sV);
+            for (int h2 = 0; h2 < 2; ++h2) {
+                float sv[16];
+                if (!zero_blk) {
+                    tmem_ld32_x16(tl + kColS + col0 + 16 * h2, sv);
+                    tmem_wait_ld();
+                }
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    const uint4 m8 = *reinterpret_cast<const uint4*>(mrow + 16 * h2 + 8 * g);
+                    const __half2* m2 = reinterpret_cast<const __half2*>(&m8);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = 4 * g + i;
+                        wv[8 * h2 + c] = zero_blk ? make_float2(0.f, 0.f)
+                                                  : __fmul2_rn(__half22float2(m2[i]), make_float2(sv[2 * c], sv[2 * c + 1]));
+                    }
+                }
+            }
+            store_row32(Ws, tok, col0, wv, 1.f);
         }
         fence_proxy_async();
         tc_fence_before();
@@ -692,26 +1099,17 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     }
     if (ok) {
         if (tid == kIssuer) {
-            if (!mbar_wait(bar_g, 0)) {
-                *abort_flag = 1.f;
-                mma_commit(bar_u);
-                mma_commit(bar_z);
-            } else {
-                issue_k128(tbase + kColU, smem_addr(Ps), smem_addr(Gs), 16, 16384, 16384, 32, kIdKK);   // U' = X-hat G^T
-                mma_commit(bar_u);
-                issue_Z();                     // Z' = W' V
-                mma_commit(bar_z);
-            }
+            issue_k128(tbase + kColS, smem_addr(Ws), smem_addr(Ks), 16384, 16384, 8192, 2048, kIdKM);   // Z = W K
+            mma_commit(bar_z);
         }
-        wait_mma_each(bar_u, ph & 1, abort_flag);
-        wait_mma_each(bar_z, ph & 1, abort_flag);
-        ++ph;
+        wait_mma_each(bar_u, 0, abort_flag);
+        wait_mma_each(bar_z, 0, abort_flag);
         __syncthreads();
         ok = *abort_flag == 0.f;
     }
     if (ok) {
-        // G x = xs sG U';  sum_j M_tj (x.k_j) v_j = xs sV sW / sK Z'
-        const float cu = xs * sG * eb, cz = xs * sV * sW / sK;
+        const float sG = scales[iG];
+        const float cu = sd * sG * seb[tok], cz = sd * sW * sV / sK;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
             float uv[16], zv[16];
@@ -719,7 +1117,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             tmem_ld32_x16(tl + kColS + col0 + 16 * h2, zv);
             tmem_wait_ld();
             if (valid) {
-                float4* dst = reinterpret_cast<float4*>(out + (base + tok) * kD + col0 + 16 * h2);
+                float4* dst = reinterpret_cast<float4*>(rhs + (base + tok) * kD + col0 + 16 * h2);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dst[i] = make_float4(fmaf(uv[4 * i], cu, zv[4 * i] * cz), fmaf(uv[4 * i + 1], cu, zv[4 * i + 1] * cz),
@@ -727,18 +1125,15 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
                                          fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
             }
         }
-        if (iters && cq == 0 && valid) iters[base + tok] = it;
     } else if (tid == kIssuer) {
         record_error(err, kErrTimeout);
-        // one more bounded chance for every MMA issued so far to drain
-        mma_commit(bar_ld);
-        mbar_wait(bar_ld, 0);
-        mbar_wait(bar_ld, 1);
+        mma_commit(bar_in);                            // one more bounded chance for the MMAs to drain
+        mbar_wait(bar_in, 1);
         mbar_wait(bar_g, 0);
     }
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tbase, 512);
+    if (w == 0) tmem_dealloc(tbase, 256);
 }
 
 }  // namespace
@@ -767,7 +1162,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     const int cg_smem = BlkSmem::bytes + 1024;
     cudaError_t e = tc_scan_launch(a, img, scales, err, st);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_cg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cg_smem);
+    e = cudaFuncSetAttribute(tc_cg_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, cg_smem);
     if (e != cudaSuccess) return e;
 #ifdef MESA_DEBUG
     static const int kOne = 1, kZero = 0;
@@ -780,10 +1175,11 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
 #endif
     {
         LaunchTimer timer(kKindTcCg, st);
-        tc_cg_kernel<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
+        tc_cg_kernel<false><<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
-            img, scales, a.out, a.iters, err, a.x_out, a.x0, a.conv_q, a.conv_k, a.conv_w);
+            img, scales, a.out, a.iters, err, a.x_out, a.x0, a.conv_q, a.conv_k, a.conv_w, nullptr, nullptr,
+            nullptr, nullptr);
     }
 #ifdef MESA_DEBUG
     if (inject) {
@@ -792,6 +1188,39 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
         return cudaMemcpyToSymbolAsync(g_debug_skip_commit, &kZero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
     }
 #endif
+    return cudaGetLastError();
+}
+
+// The adjoint solve of the backward on the tensor-core path, from the state
+// images and scales a forward_tc call over the same inputs left in
+// `images_ws`: g = G_t^T dout into rhs_buf, then u and e_t.
+cudaError_t tc_adjoint(const ForwardArgs& f, const void* images_ws, const float* dout, const float* xsol,
+                       float* rhs_buf, float* dq, float* zt, cudaStream_t st) {
+    const int nc = (f.T + kC - 1) / kC, np = (nc + 1) / 2;
+    const int BH = f.B * f.H;
+    const __half* img = reinterpret_cast<const __half*>(images_ws);
+    const float* scales =
+        reinterpret_cast<const float*>(static_cast<const char*>(images_ws) + tc_images_bytes(f.B, f.H, f.T));
+    unsigned* err = error_word_ptr();
+    const int smem = BlkSmem::bytes + 1024;
+    cudaError_t e = cudaFuncSetAttribute(tc_rhs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_cg_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    {
+        LaunchTimer timer(kKindBwdRhs, st);
+        tc_rhs_kernel<<<dim3(np, BH), kBlkThreads, smem, st>>>(
+            static_cast<const __nv_bfloat16*>(f.k), static_cast<const __nv_bfloat16*>(f.v), f.gamma, f.beta, dout,
+            f.T, np, img, scales, rhs_buf, err);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        LaunchTimer timer(kKindBwdAdj, st);
+        tc_cg_kernel<true><<<dim3(np, BH), kBlkThreads, smem, st>>>(
+            nullptr, static_cast<const __nv_bfloat16*>(f.k), static_cast<const __nv_bfloat16*>(f.v), f.gamma,
+            f.beta, f.lambda, f.H, f.T, np, f.cg_steps, f.tol, img, scales, nullptr, nullptr, err, nullptr, nullptr,
+            nullptr, nullptr, 0, rhs_buf, xsol, dq, zt);
+    }
     return cudaGetLastError();
 }
 

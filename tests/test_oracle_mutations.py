@@ -61,6 +61,11 @@ MUTANTS = {
     "backward dbeta without the value statistics": (
         "for (int j = 0; j < dk; ++j) db += vt[i] * Gbar[(size_t)i * dk + j] * kt[j];",
         "for (int j = 0; j < dk; ++j) db += 0.0 * vt[i] * Gbar[(size_t)i * dk + j] * kt[j];"),
+    "warm forward starts every token from the sequence's first guess": (
+        "x0 ? x0 + bt * dk : NULL", "x0 ? x0 + (size_t)bh * T * dk : NULL"),
+    "warm forward returns the guesses as the solutions": (
+        "if (x_out) memcpy(x_out + bt * dk, x, sizeof(double) * (size_t)dk);",
+        "if (x_out) memcpy(x_out + bt * dk, x0 ? x0 + bt * dk : x, sizeof(double) * (size_t)dk);"),
     "backward dlambda from one batch row only": ("for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * dk + i];",
                                                  "for (int b = 0; b < 1; ++b) s += part[((size_t)b * H + h) * dk + i];"),
 }
@@ -111,6 +116,8 @@ PIN_SUBSET = [
     lambda o: pins.test_preprocess_causal_and_scale_invariant(o),
     lambda o: pins.test_warm_cg_equals_shifted_cold_cg(o),
     lambda o: pins.test_warm_cg_from_the_solution_stops_at_once(o),
+    lambda o: pins.test_warm_forward_is_the_shifted_cold_solve_per_token(o),
+    lambda o: pins.test_warm_forward_from_the_exact_solutions(o),
     lambda o: pins.test_backward_matches_finite_differences_of_the_exact_layer(o),
     lambda o: pins.test_backward_one_step_closed_form(o),
     lambda o: pins.test_backward_respects_the_beta_lambda_scale_invariance(o),
