@@ -104,8 +104,86 @@ struct BlkSmem {
     static constexpr int oHaloK = oConvQ + 2048;  // and the 3 raw key and query rows before the block
     static constexpr int oHaloQ = oHaloK + 768;
     static constexpr int oGx = oHaloQ + 768;      // adjoint: g_t . x_t per token [128]
-    static constexpr int bytes = oGx + 512;
+    static constexpr int oEcol = oGx + 512;       // decay mask column factors [128]
+    static constexpr int bytes = oEcol + 512;
 };
+
+// Decay mask M_tj sK^2 / sW = msc beta_j e^{b_t - b_j} for j <= t < n, zero
+// elsewhere, fp16 in Mk (row stride kMS). Part 1 takes the 16-column group
+// that holds each row's diagonal, from one exponential per entry, and leaves
+// the column factors ecol[j] = beta_j e^{b_r - b_j} (r = the last column of
+// j's group) for part 2, which fills every other group. Part 1 needs b (sbc)
+// and beta in shared memory; part 2 needs ecol, so a CTA barrier separates
+// the two. One item per (row, column pair) or (row, group); rows run fastest
+// across a warp, so the shared loads broadcast and the stores hit distinct banks.
+static_assert(kBlkThreads == 512 && kBlk == 128, "decay mask items assume 512 threads over 128 rows");
+
+__device__ __forceinline__ void decay_mask_diag(__half* Mk, const float* sbc, const float* sbeta, float* ecol, int n,
+                                                float msc, int tid) {
+#pragma unroll
+    for (int rep = 0; rep < 2; ++rep) {
+        const int e = tid + kBlkThreads * rep;         // row tt, pair e / 128 of its diagonal group
+        const int tt = e & (kBlk - 1), j = (tt & ~15) + 2 * (e >> 7);
+        float m0 = 0.f, m1 = 0.f;
+        if (tt < n) {
+            const float bt = sbc[tt];
+            if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * msc;
+            if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * msc;
+        }
+        *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
+    }
+    if (tid < kBlk) ecol[tid] = sbeta[tid] * __expf(sbc[tid | 15] - sbc[tid]);
+}
+
+// Part 2: left of the diagonal group, e^{b_t - b_j} = e^{b_t - b_r} e^{b_r - b_j}
+// with j <= r < t. For 0 < gamma <= 1 both exponents are <= 0: neither factor
+// overflows, and neither underflows unless their product does.
+__device__ __forceinline__ void decay_mask_rest(__half* Mk, const float* sbc, const float* ecol, int n, float msc,
+                                                int tid) {
+#pragma unroll
+    for (int rep = 0; rep < 2; ++rep) {
+        const int e = tid + kBlkThreads * rep;         // row tt, 16-column group g
+        const int tt = e & (kBlk - 1), g = e >> 7;
+        if (g == (tt >> 4)) continue;                  // part 1's group
+        uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0;
+        if (tt < n && g < (tt >> 4)) {
+            const float f = msc * __expf(sbc[tt] - sbc[16 * g + 15]);
+            const float4* ec = reinterpret_cast<const float4*>(ecol + 16 * g);
+            const float4 c0 = ec[0], c1 = ec[1], c2 = ec[2], c3 = ec[3];
+            h0 = make_uint4(pack_half2(f * c0.x, f * c0.y), pack_half2(f * c0.z, f * c0.w),
+                            pack_half2(f * c1.x, f * c1.y), pack_half2(f * c1.z, f * c1.w));
+            h1 = make_uint4(pack_half2(f * c2.x, f * c2.y), pack_half2(f * c2.z, f * c2.w),
+                            pack_half2(f * c3.x, f * c3.y), pack_half2(f * c3.z, f * c3.w));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(Mk + tt * BlkSmem::kMS + 16 * g);
+        dst[0] = h0;
+        dst[1] = h1;
+    }
+}
+
+// Output rows go out through a staging tile in shared memory: each thread
+// holds one token's 32 columns, so direct stores would touch 32 rows per warp
+// instruction. The tile's rows are padded by 16 bytes, so a warp's 32
+// consecutive rows fall in distinct banks; a warp then writes whole 512-byte rows.
+constexpr int kOutPitch = kD * 4 + 16;
+static_assert(kBlk * kOutPitch <= BlkSmem::oG, "output staging must fit the four 32 KB images before G");
+
+__device__ __forceinline__ void stage_out16(uint8_t* stage, int tok, int col, const float (&uv)[16],
+                                            const float (&zv)[16], float cu, float cz) {
+    float4* dst = reinterpret_cast<float4*>(stage + tok * kOutPitch + col * 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        dst[i] = make_float4(fmaf(uv[4 * i], cu, zv[4 * i] * cz), fmaf(uv[4 * i + 1], cu, zv[4 * i + 1] * cz),
+                             fmaf(uv[4 * i + 2], cu, zv[4 * i + 2] * cz), fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
+}
+
+// Rows 0..n-1 of the staging tile to dst (row-major, kD floats a row); warp w
+// takes rows w, w + 16, ...
+__device__ __forceinline__ void write_staged_rows(const uint8_t* stage, float* dst, int n, int w, int lane) {
+    for (int r = w; r < n; r += kBlkThreads / 32)
+        reinterpret_cast<float4*>(dst + (size_t)r * kD)[lane] =
+            *reinterpret_cast<const float4*>(stage + r * kOutPitch + 16 * lane);
+}
 
 // b[t], t < 128: cumulative sum of log gamma over positions 0..t of the first
 // n positions, held constant past n. One warp, four positions per lane.
@@ -198,6 +276,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     float* seb = reinterpret_cast<float*>(smem + BlkSmem::oEb);
     float* sbc = reinterpret_cast<float*>(smem + BlkSmem::oB);
     float* sbeta = reinterpret_cast<float*>(smem + BlkSmem::oBeta);
+    float* ecol = reinterpret_cast<float*>(smem + BlkSmem::oEcol);
     float4* red = reinterpret_cast<float4*>(smem + BlkSmem::oRed);
     float* misc = reinterpret_cast<float*>(smem + BlkSmem::oMisc);
     float* abort_flag = misc + 31;
@@ -383,11 +462,25 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             p[2 * g + 1] = make_float2(f.z, f.w);
         }
     } else {
+        // The staged rows are 256 bytes apart, one per lane: lane l reads its
+        // four 16-byte pieces starting from piece l mod 4, so that a
+        // quarter-warp's eight reads fall in four bank groups, not one; the
+        // pieces are then rotated back into order.
+        const int rot = lane & 3;
+        uint4 raw[4];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-            uint4 raw = make_uint4(0, 0, 0, 0);
-            if (valid) raw = *reinterpret_cast<const uint4*>(Ws + tok * 256 + (col0 + 8 * g) * 2);
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            raw[g] = make_uint4(0, 0, 0, 0);
+            if (valid) raw[g] = *reinterpret_cast<const uint4*>(Ws + tok * 256 + col0 * 2 + 16 * ((g + rot) & 3));
+        }
+        uint4 t[4];                                    // piece c = raw[(c - rot) mod 4]
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t[c] = (rot & 1) ? raw[(c + 3) & 3] : raw[c];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) raw[c] = (rot & 2) ? t[(c + 2) & 3] : t[c];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[g]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) p[4 * g + i] = __bfloat1622float2(b2[i]);
         }
@@ -444,22 +537,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     if (tid < kBlk) seb[tid] = expf(sbc[tid]);
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) reinterpret_cast<uint4*>(Ws)[tid + kBlkThreads * rep] = make_uint4(0, 0, 0, 0);
-    {
-        // M_tj sK^2 / sW for j <= t (at most 1), as fp16 pairs. The exponent b_t - b_j
-        // is <= 0; the fast exponential's few-ulp error is far below the fp16 rounding
-        // that follows.
-        const float msc = sK * sK / sW;                // powers of two: exact
-        for (int e = tid; e < kBlk * kBlk / 2; e += kBlkThreads) {
-            const int tt = e >> 6, j = 2 * (e & 63);
-            float m0 = 0.f, m1 = 0.f;
-            if (tt < n) {
-                const float bt = sbc[tt];
-                if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * msc;
-                if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * msc;
-            }
-            *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
-        }
-    }
+    // M_tj sK^2 / sW (at most 1), part 1. The exponents are <= 0; the fast
+    // exponential's few-ulp error is far below the fp16 rounding that follows.
+    const float msc = sK * sK / sW;                    // powers of two: exact
+    decay_mask_diag(Mk, sbc, sbeta, ecol, n, msc, tid);
     float rr, pp;
     {
         float2 a = make_float2(0.f, 0.f);
@@ -470,6 +551,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         pp = d.y;                                      // |p|^2 (|x0|^2 for a warm start)
         if (kAdj && cq == 0) reinterpret_cast<float*>(smem + BlkSmem::oGx)[tok] = d.z;   // adjoint: g_t . x_t
     }
+    decay_mask_rest(Mk, sbc, ecol, n, msc, tid);       // published by the first step's barrier
     tmem_wait_st();
     const float qn = sqrtf(rr);
     bool act = valid;
@@ -840,21 +922,16 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             // G x = xs sG U';  sum_j M_tj (x.k_j) v_j = xs sV sW / sK Z'
             const float cu = xs * sG * eb, cz = xs * sV * sW / sK;
     #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
+            for (int h2 = 0; h2 < 2; ++h2) {           // every image is dead: the staging tile takes their place
                 float uv[16], zv[16];
                 tmem_ld32_x16(tl + kColU + col0 + 16 * h2, uv);
                 tmem_ld32_x16(tl + kColS + col0 + 16 * h2, zv);
                 tmem_wait_ld();
-                if (valid) {
-                    float4* dst = reinterpret_cast<float4*>(out + (base + tok) * kD + col0 + 16 * h2);
-    #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_float4(fmaf(uv[4 * i], cu, zv[4 * i] * cz), fmaf(uv[4 * i + 1], cu, zv[4 * i + 1] * cz),
-                                             fmaf(uv[4 * i + 2], cu, zv[4 * i + 2] * cz),
-                                             fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
-                }
+                stage_out16(smem, tok, col0 + 16 * h2, uv, zv, cu, cz);
             }
             if (iters && cq == 0 && valid) iters[base + tok] = it;
+            __syncthreads();
+            write_staged_rows(smem, out + base * kD, n, w, lane);
         } else if (tid == kIssuer) {
             record_error(err, kErrTimeout);
             // one more bounded chance for every MMA issued so far to drain
@@ -895,6 +972,7 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
     float* seb = reinterpret_cast<float*>(smem + BlkSmem::oEb);
     float* sbc = reinterpret_cast<float*>(smem + BlkSmem::oB);
     float* sbeta = reinterpret_cast<float*>(smem + BlkSmem::oBeta);
+    float* ecol = reinterpret_cast<float*>(smem + BlkSmem::oEcol);
     float4* red = reinterpret_cast<float4*>(smem + BlkSmem::oRed);
     float* misc = reinterpret_cast<float*>(smem + BlkSmem::oMisc);
     float* abort_flag = misc + 31;
@@ -1021,19 +1099,8 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
         }
     }
     if (tid < kBlk) seb[tid] = expf(sbc[tid]);
-    {
-        const float msc = sK * sK / sW;
-        for (int e = tid; e < kBlk * kBlk / 2; e += kBlkThreads) {
-            const int tt = e >> 6, j = 2 * (e & 63);
-            float m0 = 0.f, m1 = 0.f;
-            if (tt < n) {
-                const float bt = sbc[tt];
-                if (j <= tt) m0 = sbeta[j] * __expf(bt - sbc[j]) * msc;
-                if (j + 1 <= tt) m1 = sbeta[j + 1] * __expf(bt - sbc[j + 1]) * msc;
-            }
-            *reinterpret_cast<__half2*>(Mk + tt * BlkSmem::kMS + j) = __floats2half2_rn(m0, m1);
-        }
-    }
+    const float msc = sK * sK / sW;
+    decay_mask_diag(Mk, sbc, sbeta, ecol, n, msc, tid);
     // the dout image D = dout_t / s_t (the raw key rows in this buffer are consumed)
     float sd;
     {
@@ -1044,6 +1111,7 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
         sd = pow2_sqrt_scale(dn);
         store_row32(Ds, tok, col0, dd, 1.f / sd);
     }
+    decay_mask_rest(Mk, sbc, ecol, n, msc, tid);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -1116,15 +1184,10 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
             tmem_ld32_x16(tl + kColU + col0 + 16 * h2, uv);
             tmem_ld32_x16(tl + kColS + col0 + 16 * h2, zv);
             tmem_wait_ld();
-            if (valid) {
-                float4* dst = reinterpret_cast<float4*>(rhs + (base + tok) * kD + col0 + 16 * h2);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_float4(fmaf(uv[4 * i], cu, zv[4 * i] * cz), fmaf(uv[4 * i + 1], cu, zv[4 * i + 1] * cz),
-                                         fmaf(uv[4 * i + 2], cu, zv[4 * i + 2] * cz),
-                                         fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
-            }
+            stage_out16(smem, tok, col0 + 16 * h2, uv, zv, cu, cz);
         }
+        __syncthreads();
+        write_staged_rows(smem, rhs + base * kD, n, w, lane);
     } else if (tid == kIssuer) {
         record_error(err, kErrTimeout);
         mma_commit(bar_in);                            // one more bounded chance for the MMAs to drain
