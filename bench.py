@@ -54,11 +54,13 @@ def load_peaks():
 # Reported only while the kernel source still hashes to the captured version;
 # otherwise the field is null.
 MEASURED_TRAFFIC = {
-    "tc_cg": {"src_sha16": "15b41b6ab47e1ee9", "files": ("tc_forward.cu", "tc_layout.cuh", "tc_common.cuh"),
-              "bytes_per_token": (337.732352e6 + 107.899904e6) / 262144},
-    "tc_scan": {"src_sha16": "a21be8747fd3bf82", "files": ("tc_scan.cu", "tc_layout.cuh", "tc_common.cuh"),
-                "bytes_per_token": (136.371456e6 + 95.315456e6) / 262144},
-    "preprocess": {"src_sha16": "084d9e828774199c", "files": ("preprocess.cu",),
+    "tc_cg": {"src_sha16": "3f13d97d69d93404",
+              "files": ("tc_forward.cu", "tc_layout.cuh", "tc_common.cuh", "preproc_row.cuh"),
+              "bytes_per_token": (338.047488e6 + 109.416704e6) / 262144},
+    "tc_scan": {"src_sha16": "49f7da0aa07e356c",
+                "files": ("tc_scan.cu", "tc_layout.cuh", "tc_common.cuh", "preproc_row.cuh"),
+                "bytes_per_token": (136.399616e6 + 92.17664e6) / 262144},
+    "preprocess": {"src_sha16": "084d9e828774199c", "files": ("preprocess.cu", "preproc_row.cuh"),
                    "bytes_per_token": (537.019904e6 + 489.792512e6) / 1048576},
     "decode_step": {"src_sha16": "2d83b99e92f2442f", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
 }
