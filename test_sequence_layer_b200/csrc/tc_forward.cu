@@ -177,12 +177,37 @@ __device__ __forceinline__ void stage_out16(uint8_t* stage, int tok, int col, co
                              fmaf(uv[4 * i + 2], cu, zv[4 * i + 2] * cz), fmaf(uv[4 * i + 3], cu, zv[4 * i + 3] * cz));
 }
 
+__device__ __forceinline__ void stage_copy16(uint8_t* stage, int tok, int col, const float (&v)[16]) {
+    float4* dst = reinterpret_cast<float4*>(stage + tok * kOutPitch + col * 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+// This thread's 32 columns of TMEM columns [c0, c0 + 128) (fp32) into the
+// staging tile, then, after a CTA barrier, rows 0..n-1 of the tile to dst.
+// Every thread of the CTA calls it; the tile's previous readers must be done.
+__device__ __forceinline__ void tmem_rows_out(uint8_t* stage, uint32_t tl, uint32_t c0, int tok, int col0,
+                                              float* dst, int n, int w, int lane);
+
 // Rows 0..n-1 of the staging tile to dst (row-major, kD floats a row); warp w
 // takes rows w, w + 16, ...
 __device__ __forceinline__ void write_staged_rows(const uint8_t* stage, float* dst, int n, int w, int lane) {
     for (int r = w; r < n; r += kBlkThreads / 32)
         reinterpret_cast<float4*>(dst + (size_t)r * kD)[lane] =
             *reinterpret_cast<const float4*>(stage + r * kOutPitch + 16 * lane);
+}
+
+__device__ __forceinline__ void tmem_rows_out(uint8_t* stage, uint32_t tl, uint32_t c0, int tok, int col0,
+                                              float* dst, int n, int w, int lane) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        float v[16];
+        tmem_ld32_x16(tl + c0 + col0 + 16 * h2, v);
+        tmem_wait_ld();
+        stage_copy16(stage, tok, col0 + 16 * h2, v);
+    }
+    __syncthreads();
+    write_staged_rows(stage, dst, n, w, lane);
 }
 
 // b[t], t < 128: cumulative sum of log gamma over positions 0..t of the first
@@ -254,7 +279,10 @@ __device__ __forceinline__ void issue_k128(uint32_t d, uint32_t a, uint32_t b, u
 // g_t = G_t^T dout_t read from `rhs` (fp32, tc_rhs_kernel) under the same CG
 // rule; writes dq_t = u_t and e_t = g_t . x_t - u_t . (H_t x_t), with x_t the
 // forward's solutions (`xsol`) and H_t x_t one more product of the same kind.
-template <bool kAdj>
+// kAdj: the backward's adjoint solve (no read-out); kXout: the forward also
+// stores its solutions x in x_out (a separate instantiation keeps that path's
+// registers out of the plain forward).
+template <bool kAdj, bool kXout>
 __global__ void __launch_bounds__(kBlkThreads, 1)
 tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
              const __nv_bfloat16* __restrict__ v, const float* __restrict__ gamma,
@@ -750,17 +778,6 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             s = pow2_sqrt_scale(xx);
             store_row32(Ps, tok, col0, xr, 1.f / s);
         }
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {               // dq = u
-            float uv[16];
-            tmem_ld32_x16(tl + kColX + col0 + 16 * h2, uv);
-            tmem_wait_ld();
-            if (valid) {
-                float4* dst = reinterpret_cast<float4*>(dq + (base + tok) * kD + col0 + 16 * h2);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_float4(uv[4 * i], uv[4 * i + 1], uv[4 * i + 2], uv[4 * i + 3]);
-            }
-        }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -809,6 +826,8 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             const float uhx = quarter_sum(make_float4(a.x + a.y, 0.f, 0.f, 0.f), red, cq, tok).x;
             if (cq == 0 && valid) zt[base + tok] = reinterpret_cast<const float*>(smem + BlkSmem::oGx)[tok] - uhx;
             if (iters && cq == 0 && valid) iters[base + tok] = it;
+            // dq = u, still in the x columns of TMEM, through the staging tile (every image is dead)
+            tmem_rows_out(smem, tl, kColX, tok, col0, dq + base * kD, n, w, lane);
             ok = *abort_flag == 0.f;
         }
         if (!ok && tid == kIssuer) {
@@ -835,11 +854,6 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
                 tmem_wait_ld();
     #pragma unroll
                 for (int i = 0; i < 8; ++i) xr[8 * h2 + i] = make_float2(xv[2 * i], xv[2 * i + 1]);
-            }
-            if (x_out && valid) {                          // the solutions themselves, when asked for (fp32)
-                float4* dst = reinterpret_cast<float4*>(x_out + (base + tok) * kD + col0);
-    #pragma unroll
-                for (int i = 0; i < 8; ++i) dst[i] = make_float4(xr[2 * i].x, xr[2 * i].y, xr[2 * i + 1].x, xr[2 * i + 1].y);
             }
             float2 a = make_float2(0.f, 0.f);
     #pragma unroll
@@ -932,6 +946,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
             if (iters && cq == 0 && valid) iters[base + tok] = it;
             __syncthreads();
             write_staged_rows(smem, out + base * kD, n, w, lane);
+            if (kXout && x_out) {                          // the solutions themselves (fp32), x still in TMEM
+                __syncthreads();                           // the tile's rows are read
+                tmem_rows_out(smem, tl, kColX, tok, col0, x_out + base * kD, n, w, lane);
+            }
         } else if (tid == kIssuer) {
             record_error(err, kErrTimeout);
             // one more bounded chance for every MMA issued so far to drain
@@ -1225,7 +1243,8 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
     const int cg_smem = BlkSmem::bytes + 1024;
     cudaError_t e = tc_scan_launch(a, img, scales, err, st);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_cg_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, cg_smem);
+    auto kern = a.x_out ? tc_cg_kernel<false, true> : tc_cg_kernel<false, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, cg_smem);
     if (e != cudaSuccess) return e;
 #ifdef MESA_DEBUG
     static const int kOne = 1, kZero = 0;
@@ -1238,7 +1257,7 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st) {
 #endif
     {
         LaunchTimer timer(kKindTcCg, st);
-        tc_cg_kernel<false><<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
+        kern<<<dim3((nc + 1) / 2, BH), kBlkThreads, cg_smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.lambda, a.H, a.T, (nc + 1) / 2, a.cg_steps, a.tol,
             img, scales, a.out, a.iters, err, a.x_out, a.x0, a.conv_q, a.conv_k, a.conv_w, nullptr, nullptr,
@@ -1268,7 +1287,7 @@ cudaError_t tc_adjoint(const ForwardArgs& f, const void* images_ws, const float*
     const int smem = BlkSmem::bytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(tc_rhs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_cg_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(tc_cg_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     {
         LaunchTimer timer(kKindBwdRhs, st);
@@ -1279,7 +1298,7 @@ cudaError_t tc_adjoint(const ForwardArgs& f, const void* images_ws, const float*
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
         LaunchTimer timer(kKindBwdAdj, st);
-        tc_cg_kernel<true><<<dim3(np, BH), kBlkThreads, smem, st>>>(
+        tc_cg_kernel<true, false><<<dim3(np, BH), kBlkThreads, smem, st>>>(
             nullptr, static_cast<const __nv_bfloat16*>(f.k), static_cast<const __nv_bfloat16*>(f.v), f.gamma,
             f.beta, f.lambda, f.H, f.T, np, f.cg_steps, f.tol, img, scales, nullptr, nullptr, err, nullptr, nullptr,
             nullptr, nullptr, 0, rhs_buf, xsol, dq, zt);
