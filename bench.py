@@ -54,15 +54,16 @@ def load_peaks():
 # Reported only while the kernel source still hashes to the captured version;
 # otherwise the field is null.
 MEASURED_TRAFFIC = {
-    "tc_cg": {"src_sha16": "3f13d97d69d93404",
+    "tc_cg": {"src_sha16": "4cc94ae76b14144e",
               "files": ("tc_forward.cu", "tc_layout.cuh", "tc_common.cuh", "preproc_row.cuh"),
-              "bytes_per_token": (338.047488e6 + 109.416704e6) / 262144},
+              "bytes_per_token": (337.759488e6 + 108.347904e6) / 262144},
     "tc_scan": {"src_sha16": "49f7da0aa07e356c",
                 "files": ("tc_scan.cu", "tc_layout.cuh", "tc_common.cuh", "preproc_row.cuh"),
-                "bytes_per_token": (136.399616e6 + 92.17664e6) / 262144},
-    "preprocess": {"src_sha16": "084d9e828774199c", "files": ("preprocess.cu", "preproc_row.cuh"),
-                   "bytes_per_token": (537.019904e6 + 489.792512e6) / 1048576},
-    "decode_step": {"src_sha16": "2d83b99e92f2442f", "files": ("decode.cu",), "bytes_per_token": (543.244032e6 + 478.658816e6) / 4096},
+                "bytes_per_token": (136.559872e6 + 92.076544e6) / 262144},
+    "preprocess": {"src_sha16": "49bdcb4b9d87fc99", "files": ("preprocess.cu", "preproc_row.cuh"),
+                   "bytes_per_token": (536.979456e6 + 489.550848e6) / 1048576},
+    "decode_step": {"src_sha16": "fc551aaaf910efd1", "files": ("decode.cu", "tc_common.cuh"),
+                    "bytes_per_token": (543.23328e6 + 480.29056e6) / 4096},
 }
 
 

@@ -57,6 +57,32 @@ def test_steps_match_oracle(mesa, oracle_mod, d, tol):
     assert mesa.get_error() == 0
 
 
+def test_every_head_of_a_wide_batch(mesa, oracle_mod):
+    """More heads than the step kernel has CTAs (two per SM), and a count that
+    is not a multiple of them: the CTAs walk the heads, so every head, the
+    last ones included, is checked against the oracle over a few steps."""
+    H = 17
+    B = 2 * torch.cuda.get_device_properties(0).multi_processor_count // H + 2     # 323 heads on 148 SMs
+    w = mi.Workload("walk", B, H, 12, 32, 32, 16, "f32", 15, 0.0, False, 77)
+    x = mi.batch(w)
+    t0 = 8
+    _, _, Hs, Gs = oracle_mod.forward_cg(*(x[n][:, :, :t0] for n in ("q", "k", "v", "gamma", "beta")), x["lam"], 15)
+    Hg, Gg = cuda(Hs), cuda(Gs)
+    lam = cuda(x["lam"])
+    for t in range(t0, w.T):
+        ref, _, Hs, Gs = oracle_mod.step(*(x[n][:, :, t] for n in ("q", "k", "v", "gamma", "beta")), x["lam"],
+                                         Hs, Gs, 15, 0.0)
+        out = mesa.step(*(cuda(x[n][:, :, t]) for n in ("q", "k", "v", "gamma", "beta")), lam, Hg, Gg, cg_steps=15)
+        torch.cuda.synchronize()
+        o = out.cpu().numpy()
+        for b in range(B):                             # every head on its own
+            for h in range(H):
+                assert rel_err(o[b, h], ref[b, h]) <= TOL_F32, (t, b, h)
+    assert np.allclose(Hg.cpu().numpy(), Hs, rtol=1e-4, atol=1e-5)
+    assert np.allclose(Gg.cpu().numpy(), Gs, rtol=1e-4, atol=1e-5)
+    assert mesa.get_error() == 0
+
+
 def test_decode_equals_forward_on_gpu(mesa):
     """T single steps from a zero state reproduce the chunkwise forward (fp32)."""
     w = mi.Workload("t", 1, 4, 48, 64, 64, 16, "f32", 12, 0.0, False, 5)
