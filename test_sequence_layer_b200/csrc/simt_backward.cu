@@ -218,8 +218,11 @@ simt_adj_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const floa
 // of sequence bh from the last to the first for one tile of Hhat (rows from
 // u) or Ghat (rows from dL/do), columns from x. Writes, per chunk c, the state
 // carried in from the tokens after it.
+// Four CTAs per SM (at most 64 registers a thread): with 2 x (d / 64)^2 tiles
+// per sequence the grid is 1024 CTAs at d = 128, B x H = 128, which then runs
+// in two waves of 592 instead of three of 444.
 template <int DK, int DV, int CH>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, const float* __restrict__ xsol,
                   const float* __restrict__ gamma, int T, int nc, float* __restrict__ rstates) {
     static_assert(DK == DV, "dk == dv");
