@@ -405,9 +405,9 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     const float* Hh = rstates + ((size_t)bh * nc + c) * SE;
     const float* Gh = Hh + (size_t)DK * DK;
 
-#pragma unroll 16
+#pragma unroll 32
     for (int e = tid; e < DV * DK; e += kThreads) sR[(e / DK) * DP + e % DK] = Gh[e];
-#pragma unroll 8
+#pragma unroll 16
     for (int e = tid; e < CH * DK; e += kThreads) {
         const int t = e / DK, d = e % DK;
         const bool ok = t < n;
@@ -458,9 +458,9 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     __syncthreads();                                   // done with Ghat, the dL/do rows and the scores
 
     // ---- key statistics: Hbar_s k_s and Hbar_s^T k_s (-> dk, dbeta) ----
-#pragma unroll 16
+#pragma unroll 32
     for (int e = tid; e < DK * DK; e += kThreads) sR[(e / DK) * DP + e % DK] = Hh[e];
-#pragma unroll 8
+#pragma unroll 16
     for (int e = tid; e < CH * DK; e += kThreads) {
         const int t = e / DK, d = e % DK;
         sD[t * DP + d] = (t < n) ? u[(base + t) * DK + d] : 0.f;
