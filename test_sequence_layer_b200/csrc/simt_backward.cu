@@ -292,7 +292,8 @@ struct GradSmem {
     static constexpr int oX = oV + CH * DP;            // forward solutions x   [CH][DP]
     static constexpr int oD = oX + CH * DP;            // dL/do rows, later u   [CH][DP]
     static constexpr int oW = oD + CH * DP;            // reversed masked scores [CH][CHP]
-    static constexpr int oB = oW + CH * CHP;           // b_t                   [CH]
+    static constexpr int oW1 = oW + CH * CHP;          // N_st (k_s . x_t), kept for the second half [CH][CHP]
+    static constexpr int oB = oW1 + CH * CHP;          // b_t                   [CH]
     static constexpr int oBeta = oB + CH;              // beta_t                [CH]
     static constexpr int total = oBeta + CH;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
@@ -394,6 +395,7 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     float* sX = smem + G::oX;
     float* sD = smem + G::oD;
     float* sW = smem + G::oW;
+    float* sW1 = smem + G::oW1;
     float* sB = smem + G::oB;
     float* sBeta = smem + G::oBeta;
 
@@ -425,11 +427,11 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
 
     float acc[TP][IP], stt[TP][IP], dk_acc[TP][IP], dbt[TP];
     // ---- value statistics: Gbar_s k_s (-> dv) and Gbar_s^T v_s (-> dk) ----
-    rev_scores<DK, CH>(sK, sX, sB, n, sW);             // N_st (k_s . x_t)
+    rev_scores<DK, CH>(sK, sX, sB, n, sW1);            // N_st (k_s . x_t), used again below
     __syncthreads();
     zero2<CH, IP>(acc);
     zero2<CH, IP>(stt);
-    add_wr<DK, CH>(sW, sD, acc);
+    add_wr<DK, CH>(sW1, sD, acc);
     add_state<DK, CH, false>(sK, sR, stt);
 #pragma unroll
     for (int a = 0; a < TP; ++a) {
@@ -465,12 +467,10 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
         const int t = e / DK, d = e % DK;
         sD[t * DP + d] = (t < n) ? u[(base + t) * DK + d] : 0.f;
     }
-    __syncthreads();
-    rev_scores<DK, CH>(sK, sX, sB, n, sW);             // N_st (k_s . x_t)
-    __syncthreads();
+    __syncthreads();                                   // Hhat and the u rows are in place
     zero2<CH, IP>(acc);
     zero2<CH, IP>(stt);
-    add_wr<DK, CH>(sW, sD, acc);
+    add_wr<DK, CH>(sW1, sD, acc);                      // the same N_st (k_s . x_t) as the first half
     add_state<DK, CH, false>(sK, sR, stt);
 #pragma unroll
     for (int a = 0; a < TP; ++a) {
