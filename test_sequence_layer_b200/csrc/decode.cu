@@ -238,12 +238,15 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
             const float yi = matvec_row(pc, pi);
             const float pAp = block_sum(pi * yi, contrib, red, par, warp, lane);   // also ends the reads of sr
             if (!cg_curvature_ok(pAp)) break;
-            const float alpha = rr / pAp;
+            // alpha and rho feed recurrences that CG corrects: the fast
+            // division (a few ulp) suffices and is off the chain's critical
+            // path sooner than the IEEE one
+            const float alpha = __fdividef(rr, pAp);
             xi = fmaf(alpha, pi, xi);
             r_i = fmaf(-alpha, yi, r_i);
             if (contrib) sr[ri] = r_i;
             const float rr_new = block_sum(r_i * r_i, contrib, red, par, warp, lane);   // publishes sr
-            const float rho = rr_new / rr;
+            const float rho = __fdividef(rr_new, rr);
             pi = fmaf(rho, pi, r_i);
 #pragma unroll
             for (int c = 0; c < CPL; ++c) pc[c] = col_ok ? fmaf(rho, pc[c], sr[col0 + c]) : 0.f;
