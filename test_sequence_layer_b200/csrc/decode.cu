@@ -77,18 +77,21 @@ __device__ __forceinline__ int row_of_lane(int lane) {
 // red holds two kWarps-slot buffers used alternately (par flips per call):
 // the barrier of the call in between orders a buffer's readers before its
 // next writers, so each call needs one barrier.
+// The contributing lanes are those whose lane index is a multiple of DUP, so
+// the butterfly stops at offset DUP: lane 0 then holds the warp's sum. The 8
+// warp sums are read as two float4 (red is 16-byte aligned) and added as a tree.
+template <int DUP>
 __device__ __forceinline__ float block_sum(float v, bool contrib, float* red, int& par, int warp, int lane) {
+    static_assert(kWarps == 8, "two float4 of warp sums");
     float s = contrib ? v : 0.f;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    for (int off = 16; off >= DUP; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     float* rb = red + par * kWarps;
     if (lane == 0) rb[warp] = s;
     __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) tot += rb[w];
+    const float4 a = *reinterpret_cast<const float4*>(rb), b = *reinterpret_cast<const float4*>(rb + 4);
     par ^= 1;
-    return tot;
+    return ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
 }
 
 template <int D>
@@ -215,7 +218,7 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
 #pragma unroll
         for (int c = 0; c < CPL; ++c) pc[c] = col_ok ? sp[col0 + c] : 0.f;
         float xi = 0.f, r_i = q_i;
-        const float qq = block_sum(q_i * q_i, contrib, red, par, warp, lane);   // its barrier ends the reads of q
+        const float qq = block_sum<DUP>(q_i * q_i, contrib, red, par, warp, lane);   // its barrier ends the reads of q
         const float qn = sqrtf(qq);
         float rr = qq;
         if (xs) {                                           // r0 = q - (H + Lambda) x0
@@ -227,7 +230,7 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
             for (int c = 0; c < CPL; ++c) xc0[c] = col_ok ? sp[col0 + c] : 0.f;
             r_i = q_i - matvec_row(xc0, xi);
             if (contrib) sr[ri] = r_i;
-            rr = block_sum(r_i * r_i, contrib, red, par, warp, lane);          // publishes r0 in sr
+            rr = block_sum<DUP>(r_i * r_i, contrib, red, par, warp, lane);          // publishes r0 in sr
 #pragma unroll
             for (int c = 0; c < CPL; ++c) pc[c] = col_ok ? sr[col0 + c] : 0.f;   // p0 = r0
         }
@@ -236,7 +239,7 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
         for (int s = 0; s < cg_steps; ++s) {
             if (!cg_may_continue(rr, qn, tol)) break;   // block-uniform
             const float yi = matvec_row(pc, pi);
-            const float pAp = block_sum(pi * yi, contrib, red, par, warp, lane);   // also ends the reads of sr
+            const float pAp = block_sum<DUP>(pi * yi, contrib, red, par, warp, lane);   // also ends the reads of sr
             if (!cg_curvature_ok(pAp)) break;
             // alpha and rho feed recurrences that CG corrects: the fast
             // division (a few ulp) suffices and is off the chain's critical
@@ -245,7 +248,7 @@ step_kernel(const float* __restrict__ q, const float* __restrict__ k, const floa
             xi = fmaf(alpha, pi, xi);
             r_i = fmaf(-alpha, yi, r_i);
             if (contrib) sr[ri] = r_i;
-            const float rr_new = block_sum(r_i * r_i, contrib, red, par, warp, lane);   // publishes sr
+            const float rr_new = block_sum<DUP>(r_i * r_i, contrib, red, par, warp, lane);   // publishes sr
             const float rho = __fdividef(rr_new, rr);
             pi = fmaf(rho, pi, r_i);
 #pragma unroll
