@@ -62,8 +62,8 @@ MEASURED_TRAFFIC = {
                 "bytes_per_token": (136.559872e6 + 92.076544e6) / 262144},
     "preprocess": {"src_sha16": "49bdcb4b9d87fc99", "files": ("preprocess.cu", "preproc_row.cuh"),
                    "bytes_per_token": (536.979456e6 + 489.550848e6) / 1048576},
-    "decode_step": {"src_sha16": "fc551aaaf910efd1", "files": ("decode.cu", "tc_common.cuh"),
-                    "bytes_per_token": (543.23328e6 + 480.29056e6) / 4096},
+    "decode_step": {"src_sha16": "6e6713cd01e91c39", "files": ("decode.cu", "tc_common.cuh"),
+                    "bytes_per_token": (543.233792e6 + 478.705664e6) / 4096},
 }
 
 
