@@ -285,15 +285,17 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
 
 template <int D, int CH>
 struct GradSmem {
-    static constexpr int DP = D + 1, CHP = CH + 1;
+    // rows 16-byte aligned (vector loads along a row) and 16 bytes apart in
+    // the banks, so eight threads reading one 16-byte piece of eight
+    // consecutive rows hit distinct banks
+    static constexpr int DP = D + 4, CHP = CH + 1;
     static constexpr int oR = 0;                       // Ghat_c, later Hhat_c  [D][DP]
     static constexpr int oK = oR + D * DP;             // keys                  [CH][DP]
     static constexpr int oV = oK + CH * DP;            // values                [CH][DP]
     static constexpr int oX = oV + CH * DP;            // forward solutions x   [CH][DP]
     static constexpr int oD = oX + CH * DP;            // dL/do rows, later u   [CH][DP]
     static constexpr int oW = oD + CH * DP;            // reversed masked scores [CH][CHP]
-    static constexpr int oW1 = oW + CH * CHP;          // N_st (k_s . x_t), kept for the second half [CH][CHP]
-    static constexpr int oB = oW1 + CH * CHP;          // b_t                   [CH]
+    static constexpr int oB = oW + CH * CHP;           // b_t                   [CH]
     static constexpr int oBeta = oB + CH;              // beta_t                [CH]
     static constexpr int total = oBeta + CH;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
@@ -302,24 +304,29 @@ struct GradSmem {
 // W_st = e^{b_t - b_s} (a_s . c_t) for s <= t < n, else 0 (rows s, columns t).
 template <int D, int CH>
 __device__ __forceinline__ void rev_scores(const float* sA, const float* sC, const float* sB, int n, float* sW) {
-    constexpr int TP = CH / 16, JP = CH / 16, DP = D + 1, CHP = CH + 1;
+    constexpr int TP = CH / 16, JP = CH / 16, DP = GradSmem<D, CH>::DP, CHP = CH + 1;
     const int tt = threadIdx.x >> 4, ti = threadIdx.x & 15;
     float s[TP][JP];
 #pragma unroll
     for (int a = 0; a < TP; ++a)
 #pragma unroll
         for (int b = 0; b < JP; ++b) s[a][b] = 0.f;
-#pragma unroll 4
-    for (int kk = 0; kk < D; ++kk) {
-        float av[TP], cv[JP];
+#pragma unroll 2
+    for (int kk = 0; kk < D; kk += 4) {                // four k at a time, in order
+        float4 av[TP], cv[JP];
 #pragma unroll
-        for (int a = 0; a < TP; ++a) av[a] = sA[(tt + 16 * a) * DP + kk];
+        for (int a = 0; a < TP; ++a) av[a] = *reinterpret_cast<const float4*>(sA + (tt + 16 * a) * DP + kk);
 #pragma unroll
-        for (int b = 0; b < JP; ++b) cv[b] = sC[(ti + 16 * b) * DP + kk];
+        for (int b = 0; b < JP; ++b) cv[b] = *reinterpret_cast<const float4*>(sC + (ti + 16 * b) * DP + kk);
 #pragma unroll
         for (int a = 0; a < TP; ++a)
 #pragma unroll
-            for (int b = 0; b < JP; ++b) s[a][b] = fmaf(av[a], cv[b], s[a][b]);
+            for (int b = 0; b < JP; ++b) {
+                s[a][b] = fmaf(av[a].x, cv[b].x, s[a][b]);
+                s[a][b] = fmaf(av[a].y, cv[b].y, s[a][b]);
+                s[a][b] = fmaf(av[a].z, cv[b].z, s[a][b]);
+                s[a][b] = fmaf(av[a].w, cv[b].w, s[a][b]);
+            }
     }
 #pragma unroll
     for (int a = 0; a < TP; ++a)
@@ -333,7 +340,7 @@ __device__ __forceinline__ void rev_scores(const float* sA, const float* sC, con
 // acc[s][o] += sum_t W_st R_t[o]   (rows s = tt + 16 a, columns o = ti + 16 b)
 template <int D, int CH>
 __device__ __forceinline__ void add_wr(const float* sW, const float* sR, float (&acc)[CH / 16][D / 16]) {
-    constexpr int TP = CH / 16, IP = D / 16, DP = D + 1, CHP = CH + 1;
+    constexpr int TP = CH / 16, IP = D / 16, DP = GradSmem<D, CH>::DP, CHP = CH + 1;
     const int tt = threadIdx.x >> 4, ti = threadIdx.x & 15;
 #pragma unroll 4
     for (int t = 0; t < CH; ++t) {
@@ -352,19 +359,39 @@ __device__ __forceinline__ void add_wr(const float* sW, const float* sR, float (
 // acc[s][o] += sum_r A_s[r] M[o][r] (COL = false) or A_s[r] M[r][o] (COL = true)
 template <int D, int CH, bool COL>
 __device__ __forceinline__ void add_state(const float* sA, const float* sM, float (&acc)[CH / 16][D / 16]) {
-    constexpr int TP = CH / 16, IP = D / 16, DP = D + 1;
+    constexpr int TP = CH / 16, IP = D / 16, DP = GradSmem<D, CH>::DP;
     const int tt = threadIdx.x >> 4, ti = threadIdx.x & 15;
-#pragma unroll 4
-    for (int r = 0; r < D; ++r) {
-        float av[TP], mv[IP];
+#pragma unroll 1
+    for (int r = 0; r < D; r += 4) {                   // four r at a time, in order
+        float4 av[TP];
 #pragma unroll
-        for (int a = 0; a < TP; ++a) av[a] = sA[(tt + 16 * a) * DP + r];
+        for (int a = 0; a < TP; ++a) av[a] = *reinterpret_cast<const float4*>(sA + (tt + 16 * a) * DP + r);
+        if constexpr (COL) {                           // rows of M: one float per column, per r
 #pragma unroll
-        for (int b = 0; b < IP; ++b) mv[b] = COL ? sM[r * DP + ti + 16 * b] : sM[(ti + 16 * b) * DP + r];
+            for (int j = 0; j < 4; ++j) {
+                float mv[IP];
 #pragma unroll
-        for (int a = 0; a < TP; ++a)
+                for (int b = 0; b < IP; ++b) mv[b] = sM[(r + j) * DP + ti + 16 * b];
 #pragma unroll
-            for (int b = 0; b < IP; ++b) acc[a][b] = fmaf(av[a], mv[b], acc[a][b]);
+                for (int a = 0; a < TP; ++a) {
+                    const float aj = j == 0 ? av[a].x : j == 1 ? av[a].y : j == 2 ? av[a].z : av[a].w;
+#pragma unroll
+                    for (int b = 0; b < IP; ++b) acc[a][b] = fmaf(aj, mv[b], acc[a][b]);
+                }
+            }
+        } else {                                       // columns of M: four r per vector load
+#pragma unroll
+            for (int b = 0; b < IP; ++b) {
+                const float4 m4 = *reinterpret_cast<const float4*>(sM + (ti + 16 * b) * DP + r);
+#pragma unroll
+                for (int a = 0; a < TP; ++a) {
+                    acc[a][b] = fmaf(av[a].x, m4.x, acc[a][b]);
+                    acc[a][b] = fmaf(av[a].y, m4.y, acc[a][b]);
+                    acc[a][b] = fmaf(av[a].z, m4.z, acc[a][b]);
+                    acc[a][b] = fmaf(av[a].w, m4.w, acc[a][b]);
+                }
+            }
+        }
     }
 }
 
@@ -395,7 +422,6 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     float* sX = smem + G::oX;
     float* sD = smem + G::oD;
     float* sW = smem + G::oW;
-    float* sW1 = smem + G::oW1;
     float* sB = smem + G::oB;
     float* sBeta = smem + G::oBeta;
 
@@ -427,11 +453,11 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
 
     float acc[TP][IP], stt[TP][IP], dk_acc[TP][IP], dbt[TP];
     // ---- value statistics: Gbar_s k_s (-> dv) and Gbar_s^T v_s (-> dk) ----
-    rev_scores<DK, CH>(sK, sX, sB, n, sW1);            // N_st (k_s . x_t), used again below
+    rev_scores<DK, CH>(sK, sX, sB, n, sW);             // N_st (k_s . x_t)
     __syncthreads();
     zero2<CH, IP>(acc);
     zero2<CH, IP>(stt);
-    add_wr<DK, CH>(sW1, sD, acc);
+    add_wr<DK, CH>(sW, sD, acc);
     add_state<DK, CH, false>(sK, sR, stt);
 #pragma unroll
     for (int a = 0; a < TP; ++a) {
@@ -467,10 +493,12 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
         const int t = e / DK, d = e % DK;
         sD[t * DP + d] = (t < n) ? u[(base + t) * DK + d] : 0.f;
     }
-    __syncthreads();                                   // Hhat and the u rows are in place
+    __syncthreads();
+    rev_scores<DK, CH>(sK, sX, sB, n, sW);             // N_st (k_s . x_t)
+    __syncthreads();
     zero2<CH, IP>(acc);
     zero2<CH, IP>(stt);
-    add_wr<DK, CH>(sW1, sD, acc);                      // the same N_st (k_s . x_t) as the first half
+    add_wr<DK, CH>(sW, sD, acc);
     add_state<DK, CH, false>(sK, sR, stt);
 #pragma unroll
     for (int a = 0; a < TP; ++a) {
