@@ -283,19 +283,31 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
     }
 }
 
+// Shared tiles of the gradient kernel: rows of D floats, no padding. The
+// tiles read down their columns (the state, x and the dL/do / u rows) are
+// swizzled: the 16-byte piece j of row rho sits at piece j ^ (rho & SWM), so
+// eight threads reading one piece of eight consecutive rows hit distinct
+// banks, and a thread reads four consecutive elements of a row at once.
+template <int D>
+struct GradSwz {
+    static constexpr int SWM = (D / 4 < 8 ? D / 4 : 8) - 1;
+    // element (row, col)
+    static __device__ __forceinline__ int at(int row, int col) {
+        return row * D + ((((col >> 2) ^ (row & SWM))) << 2) + (col & 3);
+    }
+};
+
 template <int D, int CH>
 struct GradSmem {
-    // rows 16-byte aligned (vector loads along a row) and 16 bytes apart in
-    // the banks, so eight threads reading one 16-byte piece of eight
-    // consecutive rows hit distinct banks
-    static constexpr int DP = D + 4, CHP = CH + 1;
-    static constexpr int oR = 0;                       // Ghat_c, later Hhat_c  [D][DP]
-    static constexpr int oK = oR + D * DP;             // keys                  [CH][DP]
-    static constexpr int oV = oK + CH * DP;            // values                [CH][DP]
-    static constexpr int oX = oV + CH * DP;            // forward solutions x   [CH][DP]
-    static constexpr int oD = oX + CH * DP;            // dL/do rows, later u   [CH][DP]
+    static constexpr int DP = D, CHP = CH + 1;
+    static constexpr int oR = 0;                       // Ghat_c, later Hhat_c  [D][D] swizzled
+    static constexpr int oK = oR + D * DP;             // keys                  [CH][D]
+    static constexpr int oV = oK + CH * DP;            // values                [CH][D]
+    static constexpr int oX = oV + CH * DP;            // forward solutions x   [CH][D] swizzled
+    static constexpr int oD = oX + CH * DP;            // dL/do rows, later u   [CH][D] swizzled
     static constexpr int oW = oD + CH * DP;            // reversed masked scores [CH][CHP]
-    static constexpr int oB = oW + CH * CHP;           // b_t                   [CH]
+    static constexpr int oW1 = oW + CH * CHP;          // N_st (k_s . x_t), kept for the second half [CH][CHP]
+    static constexpr int oB = oW1 + CH * CHP;          // b_t                   [CH]
     static constexpr int oBeta = oB + CH;              // beta_t                [CH]
     static constexpr int total = oBeta + CH;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
@@ -317,7 +329,8 @@ __device__ __forceinline__ void rev_scores(const float* sA, const float* sC, con
 #pragma unroll
         for (int a = 0; a < TP; ++a) av[a] = *reinterpret_cast<const float4*>(sA + (tt + 16 * a) * DP + kk);
 #pragma unroll
-        for (int b = 0; b < JP; ++b) cv[b] = *reinterpret_cast<const float4*>(sC + (ti + 16 * b) * DP + kk);
+        for (int b = 0; b < JP; ++b)                   // sC swizzled; (ti + 16 b) & SWM = ti & SWM
+            cv[b] = *reinterpret_cast<const float4*>(sC + (ti + 16 * b) * DP + (((kk >> 2) ^ (ti & GradSwz<D>::SWM)) << 2));
 #pragma unroll
         for (int a = 0; a < TP; ++a)
 #pragma unroll
@@ -347,8 +360,12 @@ __device__ __forceinline__ void add_wr(const float* sW, const float* sR, float (
         float wv[TP], rv[IP];
 #pragma unroll
         for (int a = 0; a < TP; ++a) wv[a] = sW[(tt + 16 * a) * CHP + t];
+        // sR swizzled: column ti + 16 b of row t (the swizzle flips bit 0 of b
+        // when bit 2 of t & SWM is set, and the low piece bits by t & 3)
+        const int x = t & GradSwz<D>::SWM, flip = (x >> 2) << 4;
+        const float* rrow = sR + t * DP + (((ti >> 2) ^ (x & 3)) << 2) + (ti & 3);
 #pragma unroll
-        for (int b = 0; b < IP; ++b) rv[b] = sR[t * DP + ti + 16 * b];
+        for (int b = 0; b < IP; ++b) rv[b] = rrow[16 * b + ((b & 1) ? -flip : flip)];
 #pragma unroll
         for (int a = 0; a < TP; ++a)
 #pragma unroll
@@ -370,8 +387,10 @@ __device__ __forceinline__ void add_state(const float* sA, const float* sM, floa
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float mv[IP];
+                const int x = (r + j) & GradSwz<D>::SWM, flip = (x >> 2) << 4;
+                const float* mrow = sM + (r + j) * DP + (((ti >> 2) ^ (x & 3)) << 2) + (ti & 3);
 #pragma unroll
-                for (int b = 0; b < IP; ++b) mv[b] = sM[(r + j) * DP + ti + 16 * b];
+                for (int b = 0; b < IP; ++b) mv[b] = mrow[16 * b + ((b & 1) ? -flip : flip)];
 #pragma unroll
                 for (int a = 0; a < TP; ++a) {
                     const float aj = j == 0 ? av[a].x : j == 1 ? av[a].y : j == 2 ? av[a].z : av[a].w;
@@ -382,7 +401,8 @@ __device__ __forceinline__ void add_state(const float* sA, const float* sM, floa
         } else {                                       // columns of M: four r per vector load
 #pragma unroll
             for (int b = 0; b < IP; ++b) {
-                const float4 m4 = *reinterpret_cast<const float4*>(sM + (ti + 16 * b) * DP + r);
+                const float4 m4 =
+                    *reinterpret_cast<const float4*>(sM + (ti + 16 * b) * DP + (((r >> 2) ^ (ti & GradSwz<D>::SWM)) << 2));
 #pragma unroll
                 for (int a = 0; a < TP; ++a) {
                     acc[a][b] = fmaf(av[a].x, m4.x, acc[a][b]);
@@ -422,8 +442,10 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     float* sX = smem + G::oX;
     float* sD = smem + G::oD;
     float* sW = smem + G::oW;
+    float* sW1 = smem + G::oW1;
     float* sB = smem + G::oB;
     float* sBeta = smem + G::oBeta;
+    using Z = GradSwz<DK>;                             // layout of sR, sX and sD
 
     const int c = blockIdx.x, bh = blockIdx.y;
     const int t0 = c * CH;
@@ -434,15 +456,15 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     const float* Gh = Hh + (size_t)DK * DK;
 
 #pragma unroll 32
-    for (int e = tid; e < DV * DK; e += kThreads) sR[(e / DK) * DP + e % DK] = Gh[e];
+    for (int e = tid; e < DV * DK; e += kThreads) sR[Z::at(e / DK, e % DK)] = Gh[e];
 #pragma unroll 16
     for (int e = tid; e < CH * DK; e += kThreads) {
         const int t = e / DK, d = e % DK;
         const bool ok = t < n;
         sK[t * DP + d] = ok ? ld_in(k, (base + t) * DK + d) : 0.f;
         sV[t * DP + d] = ok ? ld_in(v, (base + t) * DV + d) : 0.f;
-        sX[t * DP + d] = ok ? xsol[(base + t) * DK + d] : 0.f;
-        sD[t * DP + d] = ok ? dout[(base + t) * DV + d] : 0.f;
+        sX[Z::at(t, d)] = ok ? xsol[(base + t) * DK + d] : 0.f;
+        sD[Z::at(t, d)] = ok ? dout[(base + t) * DV + d] : 0.f;
     }
     chunk_log_cumsum<CH>(gamma, base, n, sB);
     for (int t = tid; t < CH; t += kThreads) sBeta[t] = (t < n) ? beta[base + t] : 0.f;
@@ -453,11 +475,11 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
 
     float acc[TP][IP], stt[TP][IP], dk_acc[TP][IP], dbt[TP];
     // ---- value statistics: Gbar_s k_s (-> dv) and Gbar_s^T v_s (-> dk) ----
-    rev_scores<DK, CH>(sK, sX, sB, n, sW);             // N_st (k_s . x_t)
+    rev_scores<DK, CH>(sK, sX, sB, n, sW1);            // N_st (k_s . x_t), used again below
     __syncthreads();
     zero2<CH, IP>(acc);
     zero2<CH, IP>(stt);
-    add_wr<DK, CH>(sW, sD, acc);
+    add_wr<DK, CH>(sW1, sD, acc);
     add_state<DK, CH, false>(sK, sR, stt);
 #pragma unroll
     for (int a = 0; a < TP; ++a) {
@@ -487,18 +509,16 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
 
     // ---- key statistics: Hbar_s k_s and Hbar_s^T k_s (-> dk, dbeta) ----
 #pragma unroll 32
-    for (int e = tid; e < DK * DK; e += kThreads) sR[(e / DK) * DP + e % DK] = Hh[e];
+    for (int e = tid; e < DK * DK; e += kThreads) sR[Z::at(e / DK, e % DK)] = Hh[e];
 #pragma unroll 16
     for (int e = tid; e < CH * DK; e += kThreads) {
         const int t = e / DK, d = e % DK;
-        sD[t * DP + d] = (t < n) ? u[(base + t) * DK + d] : 0.f;
+        sD[Z::at(t, d)] = (t < n) ? u[(base + t) * DK + d] : 0.f;
     }
-    __syncthreads();
-    rev_scores<DK, CH>(sK, sX, sB, n, sW);             // N_st (k_s . x_t)
-    __syncthreads();
+    __syncthreads();                                   // Hhat and the u rows are in place
     zero2<CH, IP>(acc);
     zero2<CH, IP>(stt);
-    add_wr<DK, CH>(sW, sD, acc);
+    add_wr<DK, CH>(sW1, sD, acc);                      // the same N_st (k_s . x_t) as the first half
     add_state<DK, CH, false>(sK, sR, stt);
 #pragma unroll
     for (int a = 0; a < TP; ++a) {
