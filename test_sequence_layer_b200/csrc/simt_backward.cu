@@ -288,12 +288,25 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
 // swizzled: the 16-byte piece j of row rho sits at piece j ^ (rho & SWM), so
 // eight threads reading one piece of eight consecutive rows hit distinct
 // banks, and a thread reads four consecutive elements of a row at once.
+// Four consecutive input elements (16-byte aligned for float, 8-byte for bf16), widened to float.
+__device__ __forceinline__ float4 ld_in4(const float* p, size_t i) { return *reinterpret_cast<const float4*>(p + i); }
+__device__ __forceinline__ float4 ld_in4(const __nv_bfloat16* p, size_t i) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p + i);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
 template <int D>
 struct GradSwz {
     static constexpr int SWM = (D / 4 < 8 ? D / 4 : 8) - 1;
     // element (row, col)
     static __device__ __forceinline__ int at(int row, int col) {
         return row * D + ((((col >> 2) ^ (row & SWM))) << 2) + (col & 3);
+    }
+    // the 16-byte piece j of row `row`
+    static __device__ __forceinline__ float4* piece(float* tile, int row, int j) {
+        return reinterpret_cast<float4*>(tile + row * D + ((j ^ (row & SWM)) << 2));
     }
 };
 
@@ -455,16 +468,21 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     const float* Hh = rstates + ((size_t)bh * nc + c) * SE;
     const float* Gh = Hh + (size_t)DK * DK;
 
-#pragma unroll 32
-    for (int e = tid; e < DV * DK; e += kThreads) sR[Z::at(e / DK, e % DK)] = Gh[e];
-#pragma unroll 16
-    for (int e = tid; e < CH * DK; e += kThreads) {
-        const int t = e / DK, d = e % DK;
+    // 16-byte pieces: the state, then the rows (zero past n)
+    constexpr int PR = DK / 4;                         // pieces per row
+#pragma unroll 8
+    for (int e = tid; e < DV * PR; e += kThreads)
+        *Z::piece(sR, e / PR, e % PR) = *reinterpret_cast<const float4*>(Gh + 4 * (size_t)e);
+#pragma unroll 4
+    for (int e = tid; e < CH * PR; e += kThreads) {
+        const int t = e / PR, j = e % PR;
         const bool ok = t < n;
-        sK[t * DP + d] = ok ? ld_in(k, (base + t) * DK + d) : 0.f;
-        sV[t * DP + d] = ok ? ld_in(v, (base + t) * DV + d) : 0.f;
-        sX[Z::at(t, d)] = ok ? xsol[(base + t) * DK + d] : 0.f;
-        sD[Z::at(t, d)] = ok ? dout[(base + t) * DV + d] : 0.f;
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+        const size_t g = (base + t) * DK + 4 * j;
+        *reinterpret_cast<float4*>(sK + t * DP + 4 * j) = ok ? ld_in4(k, g) : zero;
+        *reinterpret_cast<float4*>(sV + t * DP + 4 * j) = ok ? ld_in4(v, g) : zero;
+        *Z::piece(sX, t, j) = ok ? *reinterpret_cast<const float4*>(xsol + g) : zero;
+        *Z::piece(sD, t, j) = ok ? *reinterpret_cast<const float4*>(dout + g) : zero;
     }
     chunk_log_cumsum<CH>(gamma, base, n, sB);
     for (int t = tid; t < CH; t += kThreads) sBeta[t] = (t < n) ? beta[base + t] : 0.f;
@@ -508,12 +526,14 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     __syncthreads();                                   // done with Ghat, the dL/do rows and the scores
 
     // ---- key statistics: Hbar_s k_s and Hbar_s^T k_s (-> dk, dbeta) ----
-#pragma unroll 32
-    for (int e = tid; e < DK * DK; e += kThreads) sR[Z::at(e / DK, e % DK)] = Hh[e];
-#pragma unroll 16
-    for (int e = tid; e < CH * DK; e += kThreads) {
-        const int t = e / DK, d = e % DK;
-        sD[Z::at(t, d)] = (t < n) ? u[(base + t) * DK + d] : 0.f;
+#pragma unroll 8
+    for (int e = tid; e < DK * PR; e += kThreads)
+        *Z::piece(sR, e / PR, e % PR) = *reinterpret_cast<const float4*>(Hh + 4 * (size_t)e);
+#pragma unroll 4
+    for (int e = tid; e < CH * PR; e += kThreads) {
+        const int t = e / PR, j = e % PR;
+        *Z::piece(sD, t, j) = (t < n) ? *reinterpret_cast<const float4*>(u + (base + t) * DK + 4 * j)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();                                   // Hhat and the u rows are in place
     zero2<CH, IP>(acc);
