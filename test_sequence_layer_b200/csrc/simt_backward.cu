@@ -470,10 +470,10 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
 
     // 16-byte pieces: the state, then the rows (zero past n)
     constexpr int PR = DK / 4;                         // pieces per row
-#pragma unroll 8
+#pragma unroll 16
     for (int e = tid; e < DV * PR; e += kThreads)
         *Z::piece(sR, e / PR, e % PR) = *reinterpret_cast<const float4*>(Gh + 4 * (size_t)e);
-#pragma unroll 4
+#pragma unroll 8
     for (int e = tid; e < CH * PR; e += kThreads) {
         const int t = e / PR, j = e % PR;
         const bool ok = t < n;
@@ -526,10 +526,10 @@ simt_grad_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, const flo
     __syncthreads();                                   // done with Ghat, the dL/do rows and the scores
 
     // ---- key statistics: Hbar_s k_s and Hbar_s^T k_s (-> dk, dbeta) ----
-#pragma unroll 8
+#pragma unroll 16
     for (int e = tid; e < DK * PR; e += kThreads)
         *Z::piece(sR, e / PR, e % PR) = *reinterpret_cast<const float4*>(Hh + 4 * (size_t)e);
-#pragma unroll 4
+#pragma unroll 8
     for (int e = tid; e < CH * PR; e += kThreads) {
         const int t = e / PR, j = e % PR;
         *Z::piece(sD, t, j) = (t < n) ? *reinterpret_cast<const float4*>(u + (base + t) * DK + 4 * j)
