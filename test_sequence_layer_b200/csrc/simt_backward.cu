@@ -265,11 +265,17 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
         for (int t = threadIdx.x; t < CH; t += kThreads) sw[t] = (t < n) ? expf(sb[t]) : 0.f;
         __syncthreads();
 #pragma unroll 4
-        for (int idx = threadIdx.x; idx < CH * TL; idx += kThreads) {
-            const int t = idx / TL, col = idx % TL;
-            const bool ok = t < n;
-            sA[t * TS + col] = ok ? sw[t] * A[(base + t) * DK + trow + col] : 0.f;
-            sX[t * TS + col] = ok ? xsol[(base + t) * DK + tcol + col] : 0.f;
+        for (int idx = threadIdx.x; idx < CH * TL / 4; idx += kThreads) {   // 16-byte pieces (TL, TS multiples of 4)
+            const int t = idx / (TL / 4), col = 4 * (idx % (TL / 4));
+            float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), x4 = a4;
+            if (t < n) {
+                const float wt = sw[t];
+                a4 = *reinterpret_cast<const float4*>(A + (base + t) * DK + trow + col);
+                a4 = make_float4(wt * a4.x, wt * a4.y, wt * a4.z, wt * a4.w);
+                x4 = *reinterpret_cast<const float4*>(xsol + (base + t) * DK + tcol + col);
+            }
+            *reinterpret_cast<float4*>(sA + t * TS + col) = a4;
+            *reinterpret_cast<float4*>(sX + t * TS + col) = x4;
         }
         __syncthreads();
         const float Gam = expf(blast);
