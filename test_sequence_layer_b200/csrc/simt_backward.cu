@@ -252,6 +252,19 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int c = 0; c < R; ++c) S[r][c] = 0.f;
+    // warp 0 holds the gammas of the next chunk (positions 2 lane, 2 lane + 1;
+    // 1 past the sequence end), loaded a chunk ahead so their latency hides
+    // under the current chunk's copies and products
+    const int lane = threadIdx.x & 31;
+    const bool gw = threadIdx.x < 32;
+    float g0 = 1.f, g1 = 1.f;
+    auto load_gates = [&](int cc) {
+        const int nn = min(CH, T - cc * CH);
+        const size_t gb = (size_t)bh * T + (size_t)cc * CH;
+        g0 = 2 * lane < nn ? gamma[gb + 2 * lane] : 1.f;
+        g1 = 2 * lane + 1 < nn ? gamma[gb + 2 * lane + 1] : 1.f;
+    };
+    if (gw && nc > 0) load_gates(nc - 1);
     for (int c = nc - 1; c >= 0; --c) {
         const int t0 = c * CH;
         const int n = min(CH, T - t0);
@@ -259,7 +272,20 @@ simt_rscan_kernel(const float* __restrict__ dout, const float* __restrict__ u, c
         float* dst = rstates + ((size_t)bh * nc + c) * SE + mat_off;
 #pragma unroll
         for (int r = 0; r < R; ++r) store_n<R>(dst + (size_t)(i0 + r) * DK + j0, S[r]);
-        chunk_log_cumsum<CH>(gamma, base, n, sb);
+        if (gw) {                                      // b = the in-chunk log-cumsum of gamma
+            const float l0 = logf(g0), l1 = logf(g1);
+            const float pair = l0 + l1;
+            float incl = pair;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            const float excl = incl - pair;
+            if (2 * lane < CH) sb[2 * lane] = excl + l0;
+            if (2 * lane + 1 < CH) sb[2 * lane + 1] = excl + l0 + l1;
+            if (c > 0) load_gates(c - 1);
+        }
         __syncthreads();
         const float blast = sb[CH - 1];
         for (int t = threadIdx.x; t < CH; t += kThreads) sw[t] = (t < n) ? expf(sb[t]) : 0.f;
