@@ -370,11 +370,21 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     // three rows before the block, and are convolved and normalised here.
     const bool fuse = conv_k != nullptr;
     const bool halo_rows = fuse && t0 >= pre::kMaxW - 1;
+    // The adjoint has no query rows and no read-out: its right-hand sides g_t
+    // and the forward solutions x_t (fp32 rows) are staged instead, g in the
+    // score and G buffers (64 KB, both free until the first masked scores)
+    // and x in the H and key buffers (the H image follows once x is read).
+    const uint32_t frow_bytes = (uint32_t)n * kD * 4;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_in, (kAdj ? 1u : 2u) * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u) +
-                                          (halo_rows ? 2u * 768u : 0u));
+        mbar_arrive_expect_tx(bar_in, (kAdj ? row_bytes + 2u * frow_bytes : 2u * row_bytes) +
+                                          (gates_bulk ? 2u * kBlk * 4u : 0u) + (halo_rows ? 2u * 768u : 0u));
         bulk_g2s(Ps, k + base * kD, row_bytes, bar_in);
-        if (!kAdj) bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
+        if (!kAdj) {
+            bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
+        } else {
+            bulk_g2s(Ws, rhs + base * kD, frow_bytes, bar_in);
+            bulk_g2s(Hs, xsol + base * kD, frow_bytes, bar_in);
+        }
         if (gates_bulk) {
             bulk_g2s(gstage, gamma + base, kBlk * 4, bar_in);
             bulk_g2s(gstage + kBlk, beta + base, kBlk * 4, bar_in);
@@ -394,10 +404,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     if (tid >= kBlk && tid < kBlk + kD) slam[tid - kBlk] = lambda[(size_t)head * kD + tid - kBlk];
     if (tid == 0) {
         if (!mbar_wait(bar_in, 0)) *abort_flag = 1.f;
-        mbar_arrive_expect_tx(bar_ld, kImgBytes);
-        bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
-        if (!kAdj) {                                   // the adjoint has no read-out
-            mbar_arrive_expect_tx(bar_g, kImgBytes);
+        if (!kAdj) {                                   // (the adjoint's H image follows its staged x rows)
+            mbar_arrive_expect_tx(bar_ld, kImgBytes);
+            bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
+            mbar_arrive_expect_tx(bar_g, kImgBytes);   // the adjoint has no read-out
             bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
         }
     }
@@ -470,25 +480,23 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     float2 p[16];
     float gx = 0.f;
     if constexpr (kAdj) {
+        // this token's g_t and x_t columns from the staged rows (one row per lane)
+        const float4* gr = reinterpret_cast<const float4*>(Ws) + tok * (kD / 4) + col0 / 4;
+        const float4* xr = reinterpret_cast<const float4*>(Hs) + tok * (kD / 4) + col0 / 4;
         float2 acc = make_float2(0.f, 0.f);
-        if (valid) {
-            const float4* gr = reinterpret_cast<const float4*>(rhs + (base + tok) * kD + col0);
-            const float4* xr = reinterpret_cast<const float4*>(xsol + (base + tok) * kD + col0);
-#pragma unroll 1
-            for (int g = 0; g < 8; ++g) {
-                const float4 f = gr[g], xf = xr[g];
-                acc = __ffma2_rn(make_float2(f.x, f.y), make_float2(xf.x, xf.y), acc);
-                acc = __ffma2_rn(make_float2(f.z, f.w), make_float2(xf.z, xf.w), acc);
-            }
-        }
-        gx = acc.x + acc.y;
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
-            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (valid) f = reinterpret_cast<const float4*>(rhs + (base + tok) * kD + col0)[g];
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f), xf = f;
+            if (valid) {
+                f = gr[g];
+                xf = xr[g];
+            }
+            acc = __ffma2_rn(make_float2(f.x, f.y), make_float2(xf.x, xf.y), acc);
+            acc = __ffma2_rn(make_float2(f.z, f.w), make_float2(xf.z, xf.w), acc);
             p[2 * g] = make_float2(f.x, f.y);
             p[2 * g + 1] = make_float2(f.z, f.w);
         }
+        gx = acc.x + acc.y;
     } else {
         // The staged rows are 256 bytes apart, one per lane: lane l reads its
         // four 16-byte pieces starting from piece l mod 4, so that a
@@ -543,6 +551,11 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
     }
     __syncthreads();                                   // gates, beta, maxima visible; staged rows consumed
+    if (kAdj && tid == 0) {                            // the H image, now that the staged x rows are read
+        fence_proxy_async();
+        mbar_arrive_expect_tx(bar_ld, kImgBytes);
+        bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
+    }
     // key scale sK >= max |k| and mask scale sW >= max_j beta_j sK^2 (powers of two)
     float sK, sW;
     {
