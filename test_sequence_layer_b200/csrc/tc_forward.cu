@@ -643,6 +643,10 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         mbar_arrive_expect_tx(bar_v, row_bytes);
         bulk_g2s(Hs, v + base * kD, row_bytes, bar_v);
     };
+    auto fetch_xsol = [&]() {                          // adjoint: the x_t rows (fp32) into the score and G buffers
+        mbar_arrive_expect_tx(bar_v, frow_bytes);
+        bulk_g2s(Ws, xsol + base * kD, frow_bytes, bar_v);
+    };
     const int first_step = x0 ? -1 : 0;
     int step = first_step;
     // step -1 (warm start only): the matvec of x0; its update leaves x = x0 and
@@ -681,6 +685,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         // here, and the read-out's value rows can be on their way during this
         // step's CUDA-core work
         if (!kAdj && tid == 0 && tol <= 0.f && step == cg_steps - 1) fetch_values();
+        // the adjoint's tail re-reads x_t: with a fixed step count its rows can
+        // be on their way into the score and G buffers (dead from here)
+        if (kAdj && tid == 0 && tol <= 0.f && step == cg_steps - 1) fetch_xsol();
 
         // y = s (sH e^b U + sW Z) + lambda p (written over Z); partials p.y, r.y, y.y, r.r
         const float c_u = s * sH * eb, c_z = s * sW;
@@ -772,14 +779,20 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     if constexpr (kAdj) {
         // ---- adjoint tail: dq = u, then H_t x_t by one more product with
         // X-hat = x / s_x, and e_t = g_t . x_t - u_t . (H_t x_t) ----
-        __syncthreads();                               // last reduction's readers are done with red[]
+        // the x_t rows: sent during the last fixed step, else now (the
+        // masked scores are dead once the loop has ended)
+        const bool x_sent = tol <= 0.f && step == cg_steps && cg_steps > first_step;
+        if (tid == 0 && !x_sent) fetch_xsol();
+        if (tid == 0 && !mbar_wait(bar_v, 0)) *abort_flag = 1.f;
+        __syncthreads();                               // x rows landed; last reduction's readers are done with red[]
         float ux_part = 0.f;
         {
             float2 xr[16];
+            const float4* xrow = reinterpret_cast<const float4*>(Ws) + tok * (kD / 4) + col0 / 4;
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
                 float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (valid) f = reinterpret_cast<const float4*>(xsol + (base + tok) * kD + col0)[g];
+                if (valid) f = xrow[g];
                 xr[2 * g] = make_float2(f.x, f.y);
                 xr[2 * g + 1] = make_float2(f.z, f.w);
             }
@@ -787,9 +800,13 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
             for (int i = 0; i < 16; ++i) a = __ffma2_rn(xr[i], xr[i], a);
             ux_part = a.x + a.y;
-            const float xx = quarter_sum(make_float4(ux_part, 0.f, 0.f, 0.f), red, cq, tok).x;
+            const float xx = quarter_sum(make_float4(ux_part, 0.f, 0.f, 0.f), red, cq, tok).x;   // every x row read
             s = pow2_sqrt_scale(xx);
             store_row32(Ps, tok, col0, xr, 1.f / s);
+            // the staged rows overwrote the score image's quarter above the
+            // diagonal (tokens 0..63, keys 64..127), which the masked scores
+            // never rewrite: zero it again (8 KB, one 16-byte piece a thread)
+            reinterpret_cast<uint4*>(Ws + 16384)[tid] = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async();
         tc_fence_before();
