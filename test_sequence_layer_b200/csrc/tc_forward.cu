@@ -374,13 +374,17 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     // and the forward solutions x_t (fp32 rows) are staged instead, g in the
     // score and G buffers (64 KB, both free until the first masked scores)
     // and x in the H and key buffers (the H image follows once x is read).
+    // A warm-started forward (the instantiation that stores its solutions)
+    // stages its x0 rows (fp32) in the H and key buffers the same way.
     const uint32_t frow_bytes = (uint32_t)n * kD * 4;
+    const bool x0_staged = kXout && !kAdj && x0 != nullptr;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_in, (kAdj ? row_bytes + 2u * frow_bytes : 2u * row_bytes) +
+        mbar_arrive_expect_tx(bar_in, (kAdj ? row_bytes + 2u * frow_bytes : 2u * row_bytes + (x0_staged ? frow_bytes : 0u)) +
                                           (gates_bulk ? 2u * kBlk * 4u : 0u) + (halo_rows ? 2u * 768u : 0u));
         bulk_g2s(Ps, k + base * kD, row_bytes, bar_in);
         if (!kAdj) {
             bulk_g2s(Ws, q + base * kD, row_bytes, bar_in);
+            if (x0_staged) bulk_g2s(Hs, x0 + base * kD, frow_bytes, bar_in);
         } else {
             bulk_g2s(Ws, rhs + base * kD, frow_bytes, bar_in);
             bulk_g2s(Hs, xsol + base * kD, frow_bytes, bar_in);
@@ -404,10 +408,12 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     if (tid >= kBlk && tid < kBlk + kD) slam[tid - kBlk] = lambda[(size_t)head * kD + tid - kBlk];
     if (tid == 0) {
         if (!mbar_wait(bar_in, 0)) *abort_flag = 1.f;
-        if (!kAdj) {                                   // (the adjoint's H image follows its staged x rows)
+        if (!kAdj && !x0_staged) {                     // (else the H image follows the staged fp32 rows)
             mbar_arrive_expect_tx(bar_ld, kImgBytes);
             bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
-            mbar_arrive_expect_tx(bar_g, kImgBytes);   // the adjoint has no read-out
+        }
+        if (!kAdj) {                                   // the adjoint has no read-out
+            mbar_arrive_expect_tx(bar_g, kImgBytes);
             bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
         }
     }
@@ -534,8 +540,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
     for (int h2 = 0; h2 < 4; ++h2) {
         float z[8], rv[8];
         float4 xa = make_float4(0.f, 0.f, 0.f, 0.f), xb = xa;
-        if (x0 && valid) {
-            const float4* src = reinterpret_cast<const float4*>(x0 + (base + tok) * kD + col0 + 8 * h2);
+        if (x0 && valid) {                             // this token's x0 columns: staged rows, else global memory
+            const float4* src = x0_staged ? reinterpret_cast<const float4*>(Hs) + tok * (kD / 4) + (col0 + 8 * h2) / 4
+                                          : reinterpret_cast<const float4*>(x0 + (base + tok) * kD + col0 + 8 * h2);
             xa = src[0];
             xb = src[1];
         }
@@ -551,7 +558,7 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
         tmem_st32_x8(tl + kColR + col0 + 8 * h2, rv);
     }
     __syncthreads();                                   // gates, beta, maxima visible; staged rows consumed
-    if (kAdj && tid == 0) {                            // the H image, now that the staged x rows are read
+    if ((kAdj || x0_staged) && tid == 0) {             // the H image, now that the staged fp32 rows are read
         fence_proxy_async();
         mbar_arrive_expect_tx(bar_ld, kImgBytes);
         bulk_g2s(Hs, img + iH * kImgHalves, kImgBytes, bar_ld);
