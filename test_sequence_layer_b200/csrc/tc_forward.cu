@@ -1072,10 +1072,16 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
     float* gstage = reinterpret_cast<float*>(red);
     const bool gates_bulk = n == kBlk && ((reinterpret_cast<uintptr_t>(gamma + base) |
                                             reinterpret_cast<uintptr_t>(beta + base)) & 15) == 0;
+    // the dout rows (fp32) are staged too: tokens 0..63 in the key-image
+    // buffer and 64..127 in the score buffer, both free until the images are
+    // written after the maxima
+    const int n_lo = n < 64 ? n : 64, n_hi = n - n_lo;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (gates_bulk ? 2u * kBlk * 4u : 0u));
+        mbar_arrive_expect_tx(bar_in, 2 * row_bytes + (uint32_t)n * kD * 4 + (gates_bulk ? 2u * kBlk * 4u : 0u));
         bulk_g2s(Ds, k + base * kD, row_bytes, bar_in);
         bulk_g2s(Vr, v + base * kD, row_bytes, bar_in);
+        bulk_g2s(Ks, dout + base * kD, (uint32_t)n_lo * kD * 4, bar_in);
+        if (n_hi > 0) bulk_g2s(Ws, dout + (base + 64) * kD, (uint32_t)n_hi * kD * 4, bar_in);
         if (gates_bulk) {
             bulk_g2s(gstage, gamma + base, kBlk * 4, bar_in);
             bulk_g2s(gstage + kBlk, beta + base, kBlk * 4, bar_in);
@@ -1083,17 +1089,20 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
         mbar_arrive_expect_tx(bar_g, kImgBytes);
         bulk_g2s(Gs, img + iG * kImgHalves, kImgBytes, bar_g);
     }
-    // this thread's token row of dout (32 columns, fp32) while the copies run
-    float2 dd[16];
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) f = reinterpret_cast<const float4*>(dout + (base + tok) * kD + col0)[g];
-        dd[2 * g] = make_float2(f.x, f.y);
-        dd[2 * g + 1] = make_float2(f.z, f.w);
-    }
     if (tid == 0 && !mbar_wait(bar_in, 0)) *abort_flag = 1.f;
     __syncthreads();
+    // this thread's token row of dout (32 columns, fp32), from the staged rows
+    float2 dd[16];
+    {
+        const float4* drow = reinterpret_cast<const float4*>(tok < 64 ? Ks : Ws) + (tok & 63) * (kD / 4) + col0 / 4;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (valid) f = drow[g];
+            dd[2 * g] = make_float2(f.x, f.y);
+            dd[2 * g + 1] = make_float2(f.z, f.w);
+        }
+    }
 
     // gates, beta, the raw key and value rows and their maxima
     if (w == 0) warp_gate_cumsum128(gates_bulk ? gstage : gamma + base, n, sbc);
