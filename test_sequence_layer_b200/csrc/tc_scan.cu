@@ -63,9 +63,12 @@ struct ScanSmem {
 static_assert(ScanSmem::oImg % 1024 == 0 && ScanSmem::kSet % 1024 == 0, "SW128 images need 1 KB alignment");
 static_assert(ScanSmem::oCmax % 16 == 0 && ScanSmem::oBar % 8 == 0, "vector and barrier alignment");
 
-// Tensor memory of a CTA (512 columns): the chunk products of H and G, then
-// the running states of H and G, 128 columns each.
-constexpr uint32_t kColAccH = 0, kColAccG = 128, kColStH = 256, kColStG = 384;
+// Tensor memory of a CTA carrying kNM states (kNM = 2: H and G; kNM = 1: the
+// one blockIdx.y names): the chunk product of state slot i in columns
+// 128 i .. 128 i + 127, the running state of slot i in 128 (kNM + i) .. .
+__host__ __device__ constexpr uint32_t col_acc(int i) { return 128u * (uint32_t)i; }
+template <int kNM>
+__device__ constexpr uint32_t col_state(int i) { return 128u * (uint32_t)(kNM + i); }
 constexpr int kAbort = 32;
 
 // The bf16 piece x times f, split into fp16 hi and lo parts (x f = hi + lo to
@@ -119,14 +122,18 @@ __device__ __forceinline__ float absmax8(uint4 raw) {
     return mx;
 }
 
-// CTA bh walks the chunks of sequence bh. Warp w serves TMEM lane quadrant
-// w % 4 (state rows 32 (w % 4) .. + 31, one per thread) and the 32 columns
-// 32 (w / 4) .. + 31 of both states. Per chunk, with w_j = beta_j e^{b_last - b_j},
+// CTA bh walks the chunks of sequence bh, for both states (kNM = 2) or for
+// state blockIdx.y (kNM = 1: H for 0, G for 1; twice the CTAs, each chunk
+// about 0.7 of the time, which pays while 2 B H CTAs fit on the SMs at once).
+// Warp w serves TMEM lane quadrant w % 4 (state rows 32 (w % 4) .. + 31, one
+// per thread) and the 32 columns 32 (w / 4) .. + 31 of each state. Per
+// chunk, with w_j = beta_j e^{b_last - b_j},
 //     H <- e^{b_last} H + sAH sK sum_j (w_j k_j / sAH) (k_j / sK)^T
 //     G <- e^{b_last} G + sAG sK sum_j (w_j v_j / sAG) (k_j / sK)^T
 // where each sum is one M = 128, N = 128, K = 64 product over the chunk's
 // tokens, issued for the hi and the lo fp16 parts of the left factor; the
 // two products share the key image.
+template <int kNM>
 __global__ void __launch_bounds__(kScanThreads, 1)
 tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                const float* __restrict__ gamma, const float* __restrict__ beta, int T, int nc,
@@ -136,6 +143,8 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int bh = blockIdx.x;
+    const int m0 = kNM == 2 ? 0 : (int)blockIdx.y;     // state of slot 0 (0: H, 1: G)
+    const bool with_h = kNM == 2 || m0 == 0, with_g = kNM == 2 || m0 == 1;   // with_g: v rows are needed
     uint8_t* rawK = smem + ScanSmem::oRawK;
     uint8_t* rawV = smem + ScanSmem::oRawV;
     float* sb = reinterpret_cast<float*>(smem + ScanSmem::oGate);      // [4][64]
@@ -161,16 +170,16 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     const size_t seq = (size_t)bh * T;
     const int np = (nc + 1) >> 1;
 
-    // Rows of chunk cc (k and v) into the row buffers (thread 0). One copy is
+    // Rows of chunk cc (k, and v for G) into the row buffers (thread 0). One copy is
     // in flight at a time: the next is issued once every thread has read the
     // rows of the previous one, so the barrier's phase parity is cc & 1.
     int prefetched = 0;
     auto prefetch = [&](int cc) {
         const int nn = min(kC, T - cc * kC);
         const uint32_t bytes = (uint32_t)nn * kD * 2;
-        mbar_arrive_expect_tx(bar_raw, 2 * bytes);
+        mbar_arrive_expect_tx(bar_raw, with_g ? 2 * bytes : bytes);
         bulk_g2s(rawK, k + (seq + (size_t)cc * kC) * kD, bytes, bar_raw);
-        bulk_g2s(rawV, v + (seq + (size_t)cc * kC) * kD, bytes, bar_raw);
+        if (with_g) bulk_g2s(rawV, v + (seq + (size_t)cc * kC) * kD, bytes, bar_raw);
         prefetched = cc + 1;
     };
     auto wait_rows = [&](int cc) {                // every thread: chunk cc's rows have landed
@@ -249,7 +258,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             rv[rep] = make_uint4(0, 0, 0, 0);
             if (j < n) {
                 rk[rep] = *reinterpret_cast<const uint4*>(rawK + j * 256 + cc16 * 16);
-                rv[rep] = *reinterpret_cast<const uint4*>(rawV + j * 256 + cc16 * 16);
+                if (with_g) rv[rep] = *reinterpret_cast<const uint4*>(rawV + j * 256 + cc16 * 16);
             }
             if (conv_k) rk[rep] = preprocess_key(cc, n, j, cc16, rk[rep]);
             float mk = absmax8(rk[rep]), mv = absmax8(rv[rep]);
@@ -289,12 +298,16 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             const int j = cid >> 4, cc16 = cid & 15;
             const uint32_t off = (uint32_t)((cc16 >> 3) * 8192 + j * 128 + (((cc16 & 7) ^ (j & 7)) << 4));
             uint4 hi, lo;
-            split_hilo(rk[rep], swc[j] * iAH, hi, lo);
-            *reinterpret_cast<uint4*>(set + off) = hi;
-            *reinterpret_cast<uint4*>(set + 16384 + off) = lo;
-            split_hilo(rv[rep], swc[j] * iAG, hi, lo);
-            *reinterpret_cast<uint4*>(set + ScanSmem::oAG + off) = hi;
-            *reinterpret_cast<uint4*>(set + ScanSmem::oAG + 16384 + off) = lo;
+            if (with_h) {
+                split_hilo(rk[rep], swc[j] * iAH, hi, lo);
+                *reinterpret_cast<uint4*>(set + off) = hi;
+                *reinterpret_cast<uint4*>(set + 16384 + off) = lo;
+            }
+            if (with_g) {
+                split_hilo(rv[rep], swc[j] * iAG, hi, lo);
+                *reinterpret_cast<uint4*>(set + ScanSmem::oAG + off) = hi;
+                *reinterpret_cast<uint4*>(set + ScanSmem::oAG + 16384 + off) = lo;
+            }
             *reinterpret_cast<uint4*>(set + ScanSmem::oB + off) = bf16x8_to_f16x8(rk[rep], iK);
         }
         return make_float2(sAH * sK, sAG * sK);
@@ -338,7 +351,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         pre::stage_weights<kD>(conv_k + (size_t)(bh % H) * conv_w * kD, conv_w, sconv);
         for (int e = tid; e < 768 / 16; e += kScanThreads) reinterpret_cast<uint4*>(halo)[e] = make_uint4(0, 0, 0, 0);
     }
-    if (w == 0) tmem_alloc(slot, 512);
+    if (w == 0) tmem_alloc(slot, 256 * kNM);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -349,7 +362,8 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     // The initial states (zero without H_in / G_in) into tensor memory, and
     // max |S_in| over each matrix for the entry bounds.
 #pragma unroll
-    for (int mm = 0; mm < 2; ++mm) {
+    for (int i = 0; i < kNM; ++i) {
+        const int mm = m0 + i;
         const float* init = mm ? G_in : H_in;
         float* fin = mm ? G_out : H_out;
         float mx = 0.f;
@@ -373,11 +387,11 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
 #pragma unroll
                 for (int i = 0; i < 4; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
             }
-            tmem_st32_x16(tl + (mm ? kColStG : kColStH) + 16 * h, S);
+            tmem_st32_x16(tl + col_state<kNM>(i) + 16 * h, S);
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        if (lane == 0) red[16 * mm + w] = mx;
+        if (lane == 0) red[16 * i + w] = mx;
     }
     tmem_wait_st();
     if (w == 1) {                                  // gates of chunks 0..2, gamma and beta of chunk 3
@@ -390,26 +404,27 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     tc_fence_before();
     __syncthreads();                              // gates and the bounds' partials visible
     tc_fence_after();
-    float bH = red[0], bG = red[16];
+    float bnd[kNM];                               // entry bounds of the slots' states
 #pragma unroll
-    for (int i = 1; i < 16; ++i) {
-        bH = fmaxf(bH, red[i]);
-        bG = fmaxf(bG, red[16 + i]);
+    for (int i = 0; i < kNM; ++i) {
+        bnd[i] = red[16 * i];
+#pragma unroll
+        for (int e = 1; e < 16; ++e) bnd[i] = fmaxf(bnd[i], red[16 * i + e]);
     }
     bool ok = red[kAbort] == 0.f;
 
     constexpr uint32_t kIdesc = idesc_f16(128, 128, true, true);
-    auto issue_mma = [&](int cc) {                // thread 0: the chunk's 2 x 8 K steps (hi, then lo) into TMEM
+    auto issue_mma = [&](int cc) {                // thread 0: the chunk's kNM x 8 K steps (hi, then lo) into TMEM
         const uint8_t* set = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
         const uint64_t dB = sdesc(smem_addr(set + ScanSmem::oB), 8192, 1024);
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm) {
-            const uint8_t* A = set + mm * ScanSmem::oAG;
+        for (int i = 0; i < kNM; ++i) {
+            const uint8_t* A = set + (m0 + i) * ScanSmem::oAG;
             const uint64_t dAhi = sdesc(smem_addr(A), 8192, 1024), dAlo = sdesc(smem_addr(A + 16384), 8192, 1024);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t ko = ((ks & 3) * 2048) >> 4;
-                mma_f16(tbase + (mm ? kColAccG : kColAccH), (ks < 4 ? dAhi : dAlo) + ko, dB + ko, kIdesc,
+                mma_f16(tbase + col_acc(i), (ks < 4 ? dAhi : dAlo) + ko, dB + ko, kIdesc,
                         ks > 0 ? 1u : 0u);
             }
         }
@@ -419,25 +434,22 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     float2 ds_cur = make_float2(1.f, 1.f), ds_next = ds_cur;   // sA sK of the chunk in the MMA, of the next chunk
     if (ok && nc > 0) {
         // the states before chunk 0 (block 0's images), chunk 0's operands, chunk 1's rows
-        const float sH0 = pow2_ceil(bH), sG0 = pow2_ceil(bG);
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm) {
-            const size_t ci = image_index(bh, np, 0, mm);
-            const float inv = 1.f / (mm ? sG0 : sH0);
+        for (int i = 0; i < kNM; ++i) {
+            const size_t ci = image_index(bh, np, 0, m0 + i);
+            const float inv = 1.f / pow2_ceil(bnd[i]);
             uint4 U[4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float S[16];
-                tmem_ld32_x16(tl + (mm ? kColStG : kColStH) + 16 * h, S);
+                tmem_ld32_x16(tl + col_state<kNM>(i) + 16 * h, S);
                 tmem_wait_ld();
                 pack_units16(U, h, S, inv);
             }
             write_units(ci, U);
         }
-        if (tid == 0) {
-            scales[image_index(bh, np, 0, 0)] = sH0;
-            scales[image_index(bh, np, 0, 1)] = sG0;
-        }
+        if (tid == 0)
+            for (int i = 0; i < kNM; ++i) scales[image_index(bh, np, 0, m0 + i)] = pow2_ceil(bnd[i]);
         wait_rows(0);
         build_load(0);
         __syncthreads();                          // chunk 0's maxima; its rows are read
@@ -484,8 +496,8 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
                 addG += __shfl_xor_sync(0xffffffffu, addG, off);
             }
             const float eb = expf(blast);
-            bH = fmaf(eb, bH, addH);
-            bG = fmaf(eb, bG, addG);
+#pragma unroll
+            for (int i = 0; i < kNM; ++i) bnd[i] = fmaf(eb, bnd[i], m0 + i ? addG : addH);
         }
         const bool emit = c + 1 < nc && ((c + 1) & 1) == 0;
         if (tid == 0) {
@@ -511,17 +523,18 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         const float Gam = expf(blast);
         const bool last = c + 1 == nc;
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm) {
+        for (int i = 0; i < kNM; ++i) {
+            const int mm = m0 + i;
             const float ds = mm ? ds_cur.y : ds_cur.x;
-            const float inv = 1.f / pow2_ceil(mm ? bG : bH);
+            const float inv = 1.f / pow2_ceil(bnd[i]);
             const size_t ci = image_index(bh, np, (c + 1) >> 1, mm);
             float* fin = mm ? G_out : H_out;
             uint4 U[4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float dv[16], S[16];
-                tmem_ld32_x16(tl + (mm ? kColAccG : kColAccH) + 16 * h, dv);
-                tmem_ld32_x16(tl + (mm ? kColStG : kColStH) + 16 * h, S);
+                tmem_ld32_x16(tl + col_acc(i) + 16 * h, dv);
+                tmem_ld32_x16(tl + col_state<kNM>(i) + 16 * h, S);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) S[i] = fmaf(Gam, S[i], ds * dv[i]);
@@ -533,7 +546,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
                             d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
                     }
                 } else {
-                    tmem_st32_x16(tl + (mm ? kColStG : kColStH) + 16 * h, S);
+                    tmem_st32_x16(tl + col_state<kNM>(i) + 16 * h, S);
                     if (emit) pack_units16(U, h, S, inv);
                 }
             }
@@ -546,10 +559,8 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         __syncthreads();                          // products read; chunk c+1's images written
         tc_fence_after();
         if (tid == 0) {
-            if (emit) {
-                scales[image_index(bh, np, (c + 1) >> 1, 0)] = pow2_ceil(bH);
-                scales[image_index(bh, np, (c + 1) >> 1, 1)] = pow2_ceil(bG);
-            }
+            if (emit)
+                for (int i = 0; i < kNM; ++i) scales[image_index(bh, np, (c + 1) >> 1, m0 + i)] = pow2_ceil(bnd[i]);
             issue_mma(c + 1);
             ++mma_issued;
         }
@@ -563,18 +574,28 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     }
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tbase, 512);
+    if (w == 0) tmem_dealloc(tbase, 256 * kNM);
 }
 
 }  // namespace
 
+// One CTA per state and sequence while all 2 B H of them fit on the SMs at
+// once (a chain of chunks is then as short as it gets); one CTA per sequence
+// carrying both states otherwise (half the CTAs, each chunk ~1.45 times as long).
 cudaError_t tc_scan_launch(const ForwardArgs& a, void* img, float* scales, unsigned* err, cudaStream_t st) {
     const int nc = (a.T + kC - 1) / kC;
     const int smem = ScanSmem::bytes + 1024;
-    const cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long seqs = (long long)a.B * a.H;
+    const bool split = 2 * seqs <= sms;
+    auto kern = split ? tc_scan_kernel<1> : tc_scan_kernel<2>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     LaunchTimer timer(kKindTcScan, st);
-    tc_scan_kernel<<<a.B * a.H, kScanThreads, smem, st>>>(
+    kern<<<dim3((unsigned)seqs, split ? 2 : 1), kScanThreads, smem, st>>>(
         static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.gamma, a.beta, a.T, nc,
         a.H_in, a.G_in, static_cast<__half*>(img), scales, a.H_out, a.G_out, err, a.conv_k, a.conv_w, a.H);
     return cudaGetLastError();
