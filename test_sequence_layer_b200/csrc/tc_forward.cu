@@ -88,7 +88,7 @@ struct BlkSmem {
     static constexpr int oK = 32768;              // key image [128 j][128 k] (32 KB); later values
     static constexpr int oP = 65536;              // P-hat image [128 t][128 k] (32 KB); later X-hat
     static constexpr int oW = 98304;              // masked scores [128 t][128 j] (32 KB)
-    static constexpr int oG = 131072;             // value-state image [128 i][128 k] (32 KB), fetched at start
+    static constexpr int oG = 131072;             // value-state image [128 l][128 i] (G transposed, 32 KB), fetched at start
     static constexpr int kMS = 136;               // mask row stride in halves (conflict-free 16-byte rows)
     static constexpr int oM = 163840;             // decay mask M sK^2 / sW, fp16 [128 t][128 j], stride kMS
     static constexpr int oLam = oM + kBlk * kMS * 2;   // lambda [128]
@@ -957,7 +957,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
                     mma_commit(bar_u);
                     mma_commit(bar_z);
                 } else {
-                    issue_k128(tbase + kColU, smem_addr(Ps), smem_addr(Gs), 16, 16384, 16384, 32, kIdKK);   // U' = X-hat G^T
+                    // U' = X-hat G^T: the image holds G transposed (row l, column i), the
+                    // right operand MN-major like the key image
+                    issue_k128(tbase + kColU, smem_addr(Ps), smem_addr(Gs), 16384, 16384, 8192, 2048, kIdKM);
                     mma_commit(bar_u);
                     issue_Z();                     // Z' = W' V
                     mma_commit(bar_z);
@@ -1008,8 +1010,9 @@ tc_cg_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 // read-out with the roles of the two factors swapped:
 //     g_t = e^{b_t} G_c^T dout_t + sum_{j <= t} M_tj (dout_t . v_j) k_j.
 // Images: D = dout_t / s_t (per-token power of two), V / sV, K / sK, the mask
-// M sK^2 / sW as in the solve, and the G image read MN-major (its rows are
-// the value index). Products: S = D V^T, W = mask o S, U = D G, Z = W K, so
+// M sK^2 / sW as in the solve, and the G image read K-major (it holds G
+// transposed: its rows are the key index l). Products: S = D V^T,
+// W = mask o S, U = D G, Z = W K, so
 //     g_t = s_t (sG e^{b_t} U_t + sW sV / sK Z_t).
 __global__ void __launch_bounds__(kBlkThreads, 1)
 tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -1191,7 +1194,8 @@ tc_rhs_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
             if (!mbar_wait(bar_g, 0)) {
                 *abort_flag = 1.f;
             } else {
-                issue_k128(tbase + kColU, smem_addr(Ds), smem_addr(Gs), 16384, 16384, 8192, 2048, kIdKM);   // U = D G
+                // U = D G: the image's rows are G's columns l, so it is read K-major
+                issue_k128(tbase + kColU, smem_addr(Ds), smem_addr(Gs), 16, 16384, 16384, 32, kIdKK);
             }
             mma_commit(bar_u);
         }

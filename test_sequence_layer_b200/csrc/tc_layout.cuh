@@ -2,9 +2,10 @@
 // tensor-core solve (tc_forward.cu) share: the head size and chunk length
 // they are built for, the fp16 state-image format and the scaling helpers.
 //
-// State image: the state before a 128-token block of one sequence (H or G,
-// 128 x 128, rows i, columns l) as fp16 values divided by a power-of-two
-// scale s >= 1 stored beside it. Two 64-column blocks of 16 KB; row i of a
+// State image: the state before a 128-token block of one sequence as fp16
+// values divided by a power-of-two scale s >= 1 stored beside it: H with
+// rows i and columns l, G transposed (row l, column i holds G[i][l]), both
+// 128 x 128. Two 64-column blocks of 16 KB; row i of a
 // block is 128 bytes whose 16-byte units (8 columns each) are permuted by
 // XOR with (i & 7): the K-major 128-byte-swizzle layout that tcgen05.mma
 // reads, so the solve loads an image with one bulk copy. Images of sequence

@@ -11,10 +11,10 @@
 // before every 128-token block of the solve is written as a scaled fp16 image
 // (format in tc_layout.cuh), plus the final states.
 //
-// Numerics: per chunk, w_j k_j / sAH and w_j v_j / sAG are split into fp16
-// hi/lo pairs and multiplied by the fp16 keys k_j / sK on the tensor cores
-// with fp32 accumulation, so each chunk's sum carries ~22-bit products into
-// the fp32 running states. sAH, sAG and sK are the powers of two at or above
+// Numerics: per chunk, the fp16 keys k_j / sK multiply w_j k_j / sAH and
+// w_j v_j / sAG, split into fp16 hi/lo pairs, on the tensor cores with fp32
+// accumulation, so each chunk's sum carries ~22-bit products into the fp32
+// running states. sAH, sAG and sK are the powers of two at or above
 // the chunk's largest |w_j k_j|, |w_j v_j| and |k_j| entries, so every operand
 // lies in [-1, 1] whatever the size of beta, k or v; a state takes sA sK
 // times its sum.
@@ -47,10 +47,10 @@ constexpr int kScanThreads = 512;
 struct ScanSmem {
     static constexpr int oRawK = 0;               // [64][128] bf16 rows of k (16 KB)
     static constexpr int oRawV = 16384;           // [64][128] bf16 rows of v (16 KB)
-    static constexpr int oImg = 32768;            // 2 operand sets, MN-major SW128, 16 KB each:
-    static constexpr int kSet = 81920;            //   {AH hi, AH lo, AG hi, AG lo, B}
-    static constexpr int oAG = 32768;             // offsets in a set
-    static constexpr int oB = 65536;
+    static constexpr int oImg = 32768;            // 2 operand sets, MN-major SW128, 16 KB per image:
+    static constexpr int kSet = 81920;            //   {W hi of slot 0, 1; W lo of slot 0, 1; K}
+    static constexpr int oLo = 32768;             // offsets in a set (W hi of slot i at 16384 i)
+    static constexpr int oK = 65536;
     static constexpr int oGate = oImg + 2 * kSet; // b[4][64], w[4][64], kmax[4][64], vmax[4][64]
     static constexpr int oRed = oGate + 4096;     // 64 floats: warp partials of H [0, 16) and G [16, 32); [32] abort
     static constexpr int oCmax = oRed + 256;      // [2 buffers][4] {max w|k|, max w|v|, max |k|, -} (int bits)
@@ -130,9 +130,12 @@ __device__ __forceinline__ float absmax8(uint4 raw) {
 // chunk, with w_j = beta_j e^{b_last - b_j},
 //     H <- e^{b_last} H + sAH sK sum_j (w_j k_j / sAH) (k_j / sK)^T
 //     G <- e^{b_last} G + sAG sK sum_j (w_j v_j / sAG) (k_j / sK)^T
-// where each sum is one M = 128, N = 128, K = 64 product over the chunk's
-// tokens, issued for the hi and the lo fp16 parts of the left factor; the
-// two products share the key image.
+// Both sums are one product over the chunk's tokens with the keys as the
+// left factor: D[l][n] = sum_j (k_j[l] / sK) W_j[n], with W_j = [w_j k_j / sAH |
+// w_j v_j / sAG] (N = 256; N = 128 with one state), issued for the hi and the
+// lo fp16 parts of W. Row l of D holds H[l][.] and G[.][l]: tensor memory
+// carries G transposed, and so do its images (row l, column i hold G[i][l])
+// and the reads and writes of G_in and G_out.
 template <int kNM>
 __global__ void __launch_bounds__(kScanThreads, 1)
 tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -222,10 +225,10 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     // v rows into registers, the row maxima of |k| and |v| into buffer cc & 3
     // (for the state bounds) and this warp's maxima of w_j |k_j|, w_j |v_j|
     // and |k_j| into cmax buffer cc & 1 (for the chunk's operand scales).
-    // build_store (stage cc-1): the scales from cmax, then AH = w_j k_j / sAH
-    // and AG = w_j v_j / sAG (hi/lo) [j][i] and B = k_j / sK [j][l] into set
-    // cc & 1, all MN-major SW128 in two 64-column blocks; returns (sAH sK,
-    // sAG sK), the factors the chunk's products carry.
+    // build_store (stage cc-1): the scales from cmax, then w_j k_j / sAH and
+    // w_j v_j / sAG (hi/lo) [j][i] and K = k_j / sK [j][l] into set cc & 1,
+    // all MN-major SW128 in 64-column blocks; returns (sAH sK, sAG sK), the
+    // factors the chunk's products carry.
     // Fused input preprocessing of the keys (conv_k given): the raw piece of
     // row j of chunk cc becomes its convolved, normalised bf16 piece. The rows
     // before it come from the chunk's raw rows or, for its first three rows,
@@ -298,17 +301,17 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             const int j = cid >> 4, cc16 = cid & 15;
             const uint32_t off = (uint32_t)((cc16 >> 3) * 8192 + j * 128 + (((cc16 & 7) ^ (j & 7)) << 4));
             uint4 hi, lo;
-            if (with_h) {
+            if (with_h) {                          // slot 0
                 split_hilo(rk[rep], swc[j] * iAH, hi, lo);
                 *reinterpret_cast<uint4*>(set + off) = hi;
-                *reinterpret_cast<uint4*>(set + 16384 + off) = lo;
+                *reinterpret_cast<uint4*>(set + ScanSmem::oLo + off) = lo;
             }
-            if (with_g) {
+            if (with_g) {                          // slot kNM - 1
                 split_hilo(rv[rep], swc[j] * iAG, hi, lo);
-                *reinterpret_cast<uint4*>(set + ScanSmem::oAG + off) = hi;
-                *reinterpret_cast<uint4*>(set + ScanSmem::oAG + 16384 + off) = lo;
+                *reinterpret_cast<uint4*>(set + 16384 * (kNM - 1) + off) = hi;
+                *reinterpret_cast<uint4*>(set + ScanSmem::oLo + 16384 * (kNM - 1) + off) = lo;
             }
-            *reinterpret_cast<uint4*>(set + ScanSmem::oB + off) = bf16x8_to_f16x8(rk[rep], iK);
+            *reinterpret_cast<uint4*>(set + ScanSmem::oK + off) = bf16x8_to_f16x8(rk[rep], iK);
         }
         return make_float2(sAH * sK, sAG * sK);
     };
@@ -337,6 +340,36 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         for (int s = 0; s < 4; ++s) {
             const int r = 32 * q4 + (lane & ~3) + s;
             *reinterpret_cast<uint4*>(blk + r * 128 + ((u ^ (r & 7)) << 4)) = U[s];
+        }
+    };
+
+    // 16 entries of a state as this thread holds them (TMEM lane `row`,
+    // columns col0 + 16 h ..): H[row][col] for H (mm = 0), G[col][row] for G,
+    // which tensor memory carries transposed; the G accesses are coalesced
+    // across the warp's consecutive rows.
+    auto load16 = [&](const float* src, int mm, int h, float (&S)[16]) {
+        const float* base = src + (size_t)bh * kD * kD;
+        if (mm == 0) {
+            const float4* s4 = reinterpret_cast<const float4*>(base + (size_t)row * kD + col0 + 16 * h);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 f = s4[i];
+                S[4 * i] = f.x; S[4 * i + 1] = f.y; S[4 * i + 2] = f.z; S[4 * i + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) S[i] = base[(size_t)(col0 + 16 * h + i) * kD + row];
+        }
+    };
+    auto store16 = [&](float* dst, int mm, int h, const float (&S)[16]) {
+        float* base = dst + (size_t)bh * kD * kD;
+        if (mm == 0) {
+            float4* d4 = reinterpret_cast<float4*>(base + (size_t)row * kD + col0 + 16 * h);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) base[(size_t)(col0 + 16 * h + i) * kD + row] = S[i];
         }
     };
 
@@ -372,21 +405,10 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
             float S[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) S[i] = 0.f;
-            if (init) {
-                const float4* src = reinterpret_cast<const float4*>(init + ((size_t)bh * kD + row) * kD + col0 + 16 * h);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 f = src[i];
-                    S[4 * i] = f.x; S[4 * i + 1] = f.y; S[4 * i + 2] = f.z; S[4 * i + 3] = f.w;
-                }
-            }
+            if (init) load16(init, mm, h, S);
 #pragma unroll
             for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(S[i]));
-            if (nc == 0 && fin) {                 // no tokens: the final state is the initial one
-                float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0 + 16 * h);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
-            }
+            if (nc == 0 && fin) store16(fin, mm, h, S);    // no tokens: the final state is the initial one
             tmem_st32_x16(tl + col_state<kNM>(i) + 16 * h, S);
         }
 #pragma unroll
@@ -413,20 +435,15 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
     }
     bool ok = red[kAbort] == 0.f;
 
-    constexpr uint32_t kIdesc = idesc_f16(128, 128, true, true);
-    auto issue_mma = [&](int cc) {                // thread 0: the chunk's kNM x 8 K steps (hi, then lo) into TMEM
+    constexpr uint32_t kIdesc = idesc_f16(128, 128 * kNM, true, true);
+    auto issue_mma = [&](int cc) {                // thread 0: the chunk's 8 K steps (W hi, then W lo) into TMEM
         const uint8_t* set = smem + ScanSmem::oImg + (cc & 1) * ScanSmem::kSet;
-        const uint64_t dB = sdesc(smem_addr(set + ScanSmem::oB), 8192, 1024);
+        const uint64_t dA = sdesc(smem_addr(set + ScanSmem::oK), 8192, 1024);
+        const uint64_t dBhi = sdesc(smem_addr(set), 8192, 1024), dBlo = sdesc(smem_addr(set + ScanSmem::oLo), 8192, 1024);
 #pragma unroll
-        for (int i = 0; i < kNM; ++i) {
-            const uint8_t* A = set + (m0 + i) * ScanSmem::oAG;
-            const uint64_t dAhi = sdesc(smem_addr(A), 8192, 1024), dAlo = sdesc(smem_addr(A + 16384), 8192, 1024);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t ko = ((ks & 3) * 2048) >> 4;
-                mma_f16(tbase + col_acc(i), (ks < 4 ? dAhi : dAlo) + ko, dB + ko, kIdesc,
-                        ks > 0 ? 1u : 0u);
-            }
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t ko = ((ks & 3) * 2048) >> 4;
+            mma_f16(tbase + col_acc(0), dA + ko, (ks < 4 ? dBhi : dBlo) + ko, kIdesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(bar_mma);
     };
@@ -539,12 +556,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
 #pragma unroll
                 for (int i = 0; i < 16; ++i) S[i] = fmaf(Gam, S[i], ds * dv[i]);
                 if (last) {
-                    if (fin) {
-                        float4* d4 = reinterpret_cast<float4*>(fin + ((size_t)bh * kD + row) * kD + col0 + 16 * h);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            d4[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
-                    }
+                    if (fin) store16(fin, mm, h, S);
                 } else {
                     tmem_st32_x16(tl + col_state<kNM>(i) + 16 * h, S);
                     if (emit) pack_units16(U, h, S, inv);
