@@ -6,10 +6,11 @@
 // "Parallelisation" paragraph: the states carried from chunk to chunk obey
 //     H_{c+1} = e^{b_last} H_c + K^T diag(w) K,   G_{c+1} = e^{b_last} G_c + V^T diag(w) K,
 // with b_t the in-chunk log-cumsum of gamma and w_j = beta_j e^{b_last-b_j}.
-// One CTA walks the chunks of one sequence and carries both states: they
-// live in tensor memory as fp32 beside the two chunk products, and the state
-// before every 128-token block of the solve is written as a scaled fp16 image
-// (format in tc_layout.cuh), plus the final states.
+// One CTA walks the chunks of one sequence and carries both states (or, for
+// small batches, one CTA per state and sequence): they live in tensor memory
+// as fp32 beside the chunk products, and the state before every 128-token
+// block of the solve is written as a scaled fp16 image (format in
+// tc_layout.cuh), plus the final states.
 //
 // Numerics: per chunk, the fp16 keys k_j / sK multiply w_j k_j / sAH and
 // w_j v_j / sAG, split into fp16 hi/lo pairs, on the tensor cores with fp32
@@ -134,8 +135,9 @@ __device__ __forceinline__ float absmax8(uint4 raw) {
 // left factor: D[l][n] = sum_j (k_j[l] / sK) W_j[n], with W_j = [w_j k_j / sAH |
 // w_j v_j / sAG] (N = 256; N = 128 with one state), issued for the hi and the
 // lo fp16 parts of W. Row l of D holds H[l][.] and G[.][l]: tensor memory
-// carries G transposed, and so do its images (row l, column i hold G[i][l])
-// and the reads and writes of G_in and G_out.
+// carries G transposed, and so do its images (row l, column i hold G[i][l]);
+// G_in and G_out keep the [i][l] layout of the interface and are read and
+// written down their columns.
 template <int kNM>
 __global__ void __launch_bounds__(kScanThreads, 1)
 tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,

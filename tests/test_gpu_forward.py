@@ -115,6 +115,35 @@ def test_state_in_and_out(mesa, oracle_mod, dtype, d, chunk):
     assert rel_err(out.cpu().numpy(), ref) <= tol
 
 
+def test_state_in_and_out_wide_batch(mesa, oracle_mod):
+    """A batch of 96 sequences: more than half the SM count, so the tensor-core
+    scan carries both states in one CTA per sequence (G transposed in tensor
+    memory, in its images and in the reads of G_in and writes of G_out).
+    The smaller batches above use one CTA per state."""
+    w = rand_workload(128, 64, "bf16", 100, B=6, H=16, N=4, seed=11)
+    x = mi.batch(w)
+    t0 = 37
+    pre = {n: x[n][:, :, :t0] for n in ("q", "k", "v", "gamma", "beta")}
+    post = {n: x[n][:, :, t0:] for n in ("q", "k", "v", "gamma", "beta")}
+    _, _, H1, G1 = oracle_mod.forward_cg(*(pre[n] for n in ("q", "k", "v", "gamma", "beta")), x["lam"], 4)
+    ref, _, Hf, Gf = oracle_mod.forward_cg(*(post[n] for n in ("q", "k", "v", "gamma", "beta")), x["lam"], 4,
+                                           H0=H1, G0=G1)
+    dpre = to_dev(dict(pre, lam=x["lam"]), "bf16")
+    dpost = to_dev(dict(post, lam=x["lam"]), "bf16")
+    _, Hg, Gg = mesa.forward(dpre["q"], dpre["k"], dpre["v"], dpre["gamma"], dpre["beta"], dpre["lam"],
+                             chunk=64, cg_steps=4, return_state=True)
+    out, Hg2, Gg2 = mesa.forward(dpost["q"], dpost["k"], dpost["v"], dpost["gamma"], dpost["beta"], dpost["lam"],
+                                 chunk=64, cg_steps=4, H_in=Hg, G_in=Gg, return_state=True)
+    torch.cuda.synchronize()
+    assert mesa.get_error() == 0
+    assert np.allclose(Hg.cpu().numpy(), H1, rtol=1e-5, atol=1e-5)
+    assert np.allclose(Gg.cpu().numpy(), G1, rtol=1e-5, atol=1e-5)
+    assert np.allclose(Hg2.cpu().numpy(), Hf, rtol=1e-5, atol=1e-5)
+    assert np.allclose(Gg2.cpu().numpy(), Gf, rtol=1e-5, atol=1e-5)
+    got = out.cpu().numpy()
+    assert rel_err(got, ref) <= TOL_BF16, err_report(got, ref)
+
+
 def test_empty_sequence_copies_state(mesa):
     B, H, d = 2, 3, 16
     z = torch.zeros((B, H, 0, d), device="cuda")
