@@ -116,10 +116,13 @@ def layer_inputs(B, H, T, d, seed, dtype):
     return x, raw_q, raw_k
 
 
-@pytest.mark.parametrize("T,W,tol", [(1, 4, 0.0), (3, 4, 0.0), (64, 2, 0.0), (65, 4, 0.0), (130, 3, 0.0),
-                                     (333, 4, 0.0), (700, 1, 0.0), (300, 4, 1e-3)])
-def test_fused_forward_equals_preprocess_then_forward(mesa, T, W, tol):
-    B, H, d = 2, 3, 128
+@pytest.mark.parametrize("B,H,T,W,tol", [(2, 3, 1, 4, 0.0), (2, 3, 3, 4, 0.0), (2, 3, 64, 2, 0.0), (2, 3, 65, 4, 0.0),
+                                         (2, 3, 130, 3, 0.0), (2, 3, 333, 4, 0.0), (2, 3, 700, 1, 0.0),
+                                         (2, 3, 300, 4, 1e-3),
+                                         # 96 sequences: the scan carries both states in one CTA per sequence
+                                         (6, 16, 200, 4, 0.0), (6, 16, 150, 3, 1e-3)])
+def test_fused_forward_equals_preprocess_then_forward(mesa, B, H, T, W, tol):
+    d = 128
     x, rq, rk = layer_inputs(B, H, T, d, 90 + T, "bf16")
     rng = np.random.default_rng(T)
     cq = torch.from_numpy((rng.standard_normal((H, W, d)) / np.sqrt(W)).astype(np.float32)).cuda()
