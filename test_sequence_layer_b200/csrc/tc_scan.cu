@@ -406,10 +406,10 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
         for (int h = 0; h < 2; ++h) {
             float S[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) S[i] = 0.f;
+            for (int e = 0; e < 16; ++e) S[e] = 0.f;
             if (init) load16(init, mm, h, S);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(S[i]));
+            for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(S[e]));
             if (nc == 0 && fin) store16(fin, mm, h, S);    // no tokens: the final state is the initial one
             tmem_st32_x16(tl + col_state<kNM>(i) + 16 * h, S);
         }
@@ -556,7 +556,7 @@ tc_scan_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restr
                 tmem_ld32_x16(tl + col_state<kNM>(i) + 16 * h, S);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) S[i] = fmaf(Gam, S[i], ds * dv[i]);
+                for (int e = 0; e < 16; ++e) S[e] = fmaf(Gam, S[e], ds * dv[e]);
                 if (last) {
                     if (fin) store16(fin, mm, h, S);
                 } else {
