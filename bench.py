@@ -57,9 +57,9 @@ MEASURED_TRAFFIC = {
     "tc_cg": {"src_sha16": "e4bafe8b775e8e79",
               "files": ("tc_forward.cu", "tc_layout.cuh", "tc_common.cuh", "preproc_row.cuh"),
               "bytes_per_token": (337.756672e6 + 109.066752e6) / 262144},
-    "tc_scan": {"src_sha16": "d4fbf3eb303e3798",
+    "tc_scan": {"src_sha16": "7e35aa166da95c08",
                 "files": ("tc_scan.cu", "tc_layout.cuh", "tc_common.cuh", "preproc_row.cuh"),
-                "bytes_per_token": (136.396800e6 + 91.947520e6) / 262144},
+                "bytes_per_token": (136.395520e6 + 91.302400e6) / 262144},
     "preprocess": {"src_sha16": "49bdcb4b9d87fc99", "files": ("preprocess.cu", "preproc_row.cuh"),
                    "bytes_per_token": (536.979456e6 + 489.550848e6) / 1048576},
     "decode_step": {"src_sha16": "6e6713cd01e91c39", "files": ("decode.cu", "tc_common.cuh"),
