@@ -91,6 +91,11 @@ cudaError_t forward_tc(const ForwardArgs& a, cudaStream_t st);
 // Chunk-state scan of the tensor-core forward: state images and scales into
 // img / scales (layout in tc_layout.cuh), final states into a.H_out / a.G_out.
 cudaError_t tc_scan_launch(const ForwardArgs& a, void* img, float* scales, unsigned* err, cudaStream_t st);
+// The backward's reverse chunk scan of the gradient states on the tensor
+// cores (d = 128, C = 64): per chunk the fp32 states carried in from the
+// tokens after it, [B*H][chunks][Hhat, Ghat][128][128].
+cudaError_t tc_rscan_launch(const float* dout, const float* u, const float* xsol, const float* gamma, int B, int H,
+                            int T, float* rstates, unsigned* err, cudaStream_t st);
 // The backward's adjoint solve on the tensor cores, from the images a
 // forward_tc call left at the start of `images_ws`: the right-hand side
 // g_t = G_t^T dout_t (into rhs_buf), then u_t = CG(H_t + Lambda, g_t) into dq

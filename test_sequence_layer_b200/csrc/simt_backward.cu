@@ -731,9 +731,13 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
             f.T, nc, f.cg_steps, f.tol, states, a.dq, Z, part);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    constexpr int TL = D < 64 ? D : 64;
-    constexpr int tiles = 2 * (D / TL) * (D / TL);
-    {
+    if (tc_supported(f.dk, f.dv, f.chunk, f.dtype)) {
+        // the reverse scan on the tensor cores at the same bf16-mode precision
+        if ((e = tc_rscan_launch(a.dout, a.dq, X, f.gamma, f.B, f.H, f.T, R, error_word_ptr(), st)) != cudaSuccess)
+            return e;
+    } else {
+        constexpr int TL = D < 64 ? D : 64;
+        constexpr int tiles = 2 * (D / TL) * (D / TL);
         LaunchTimer timer(kKindBwdRscan, st);
         simt_rscan_kernel<D, D, CH><<<dim3(tiles, BH), kThreads, 0, st>>>(a.dout, a.dq, X, f.gamma, f.T, nc, R);
     }
