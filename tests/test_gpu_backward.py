@@ -58,6 +58,8 @@ CASES = [
     ("bf16", 128, 64, 200, 2, 1, 15, 0.0),
     ("bf16", 64, 64, 150, 1, 2, 15, 0.0),
     ("f32", 64, 32, 64, 1, 1, 3, 0.0),
+    # 96 sequences: the tensor-core scans carry both states in one CTA per sequence
+    ("bf16", 128, 64, 100, 6, 16, 6, 0.0),
 ]
 
 
